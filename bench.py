@@ -1,0 +1,316 @@
+"""Benchmark: masked attention forward TFLOP/s on attended pairs (bf16), B200.
+
+One step = the whole hot path on one batch: plan the dense causal (N, N) mask
+(bfa_plan_dense: classify + lists + order) and run the fused forward (bfa_fwd)
+for B=4, H=Hkv=32, N=8192, D=128.  FLOPs are counted on attended pairs only:
+4 * D * nnz per (batch, head), nnz = N (N + 1) / 2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bfa|reference]
+
+Multi-GPU (torchrun): every rank runs its own full workload (weak scaling, no
+collective on the data path); value = all ranks' FLOPs / max-over-ranks time.
+``--impl reference`` times the CPU float64 oracle on the host cores instead (rank
+0 only), on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "masked attn fwd TFLOP/s on attended pairs (bf16), % of B200 tensor peak"
+WORKLOAD = dict(workload="causal_8192", B=4, H=32, Hkv=32, N=8192, D=128, mask="dense causal (N,N) bool",
+                plan="bfa_plan_dense per step", layout="BSHD")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _attended_flops(N, D, BH):
+    nnz = N * (N + 1) // 2
+    return 4.0 * D * nnz * BH, nnz
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        srt = sorted(sm)
+        loaded = [x for x in srt if x > 0.5 * max(srt)] or srt
+        return {"sm_mhz": loaded[len(loaded) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_oracle_sample(w, n_heads=4, rows=None):
+    """Time the float64 oracle on a bounded sample: ``n_heads`` (b, h) pairs, all rows."""
+    from oracle import attention as oa
+    M = w["mask"].numpy()
+    N, D = w["N"], w["D"]
+    pairs = [(b, h) for b in range(w["B"]) for h in range(w["H"])][:n_heads]
+    t0 = time.perf_counter()
+    for (b, h) in pairs:
+        q = w["q"][b, :, h]
+        MM = M
+        if rows is not None:
+            q, MM = q[:rows], M[:rows]
+        oa.masked_attention(q, w["k"][b, :, h], w["v"][b, :, h], MM)
+    dt = time.perf_counter() - t0
+    nnz = int(M.sum()) if rows is None else int(M[:rows].sum())
+    flops = 4.0 * D * nnz * len(pairs)
+    return flops / dt / 1e12, dt, len(pairs)
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import workloads
+    w = workloads.causal_8192()
+    times, vals = [], []
+    per_step_heads = 2
+    for i in range(args.warmup + args.steps):
+        v, dt, n = cpu_oracle_sample(w, n_heads=per_step_heads)
+        if i >= args.warmup:
+            times.append(dt)
+            vals.append(v)
+    value = sum(vals) / len(vals)
+    cores = _threads_used()
+    sample = f"{per_step_heads} of 128 (batch, head) pairs per step, all 8192 rows, float64 NumPy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism=f"dp{args.gpus}"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_bfa(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import mask_skipping_flashattention_b200 as bfa
+    import workloads
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = workloads.causal_8192()
+    B, H, N, D = w["B"], w["H"], w["N"], w["D"]
+    q, k, v = w["q"].to(dev), w["k"].to(dev), w["v"].to(dev)
+    mask = w["mask"].to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    flops, nnz = _attended_flops(N, D, B * H)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        plan = bfa.plan_dense(mask)
+        if ev is not None:
+            ev[1].record(stream)
+        bfa.fwd(plan, q, k, v, out=out, lse=lse)
+        if ev is not None:
+            ev[2].record(stream)
+        plan.destroy()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    fwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    plan_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms, fwd_ms, plan_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, fwd_ms, plan_ms = t.tolist()
+    ms_per_step = ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: H2D of q/k/v/mask from
+    # pinned memory, plan + forward, D2H of out and lse, every step
+    hq, hk, hv = w["q"].pin_memory(), w["k"].pin_memory(), w["v"].pin_memory()
+    hm = w["mask"].pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hm))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        mask.copy_(hm, non_blocking=True)
+        plan = bfa.plan_dense(mask)
+        bfa.fwd(plan, q, k, v, out=out, lse=lse)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        plan.destroy()
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    peaks, src = _peaks()
+    fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(WORKLOAD, global_batch=B * world, seq_len=N, parallelism=f"dp{world}",
+                       attended_pairs_per_head=nnz, gflop_per_step=flops / 1e9,
+                       l2="inputs larger than L2 (q, k, v 268 MB each, mask 67 MB); no flush"),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "kernel": "bfa_fwd_kernel<128>", "achieved": fwd_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": fwd_tflops / peak, "peak_source": f"{src} bf16_tflops (burst)",
+                     "frac_of_sustained": fwd_tflops / peaks.get("bf16_tflops_sustained", peak),
+                     "traffic": None},
+        "fwd_ms": fwd_ms, "plan_ms": plan_ms,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v_cpu, dt, n = cpu_oracle_sample(w, n_heads=2)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": _threads_used(), "kind": "oracle",
+                                "sample": f"{n} of 128 (batch, head) pairs, all 8192 rows, {dt:.1f} s float64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["bfa", "reference"], default="bfa")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_bfa(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,228 @@
+/*
+ * bfa.h -- C ABI of the mask-aware fused attention forward for NVIDIA B200 (sm_100a).
+ *
+ * The library computes O = softmax(scale * Q K^T + mask) V and the natural-log
+ * LSE of every query row, where the boolean mask (True = attend) is never
+ * materialised inside the score loop.  A mask is first turned into a *plan*:
+ * for every 128-row query tile, the ascending list of 128-column key tiles that
+ * hold at least one attended pair, each marked full (every in-range pair
+ * attended) or partial, plus 32-bit packed fine masks for the partial tiles of a
+ * dense mask.  The forward kernel then visits only the listed tiles, runs full
+ * tiles with no mask work, and masks partial tiles from the packed bits, from the
+ * block-id predicate, or from positions.
+ *
+ * Sources (page title, section):
+ *   - BinFlash, "Efficiently Dispatching FlashAttention For Partially Filled
+ *     Attention Masks": coarse block mask + 32-bit packed fine mask, pre-sorted
+ *     non-empty key-block list per query row, all-True blocks with no mask loads,
+ *     all-False blocks skipped; mask (N, N) bool, True = attend; scale 1/sqrt(D).
+ *   - opentau.policies.flash_attn_cuda, make_att_block_ids / flash_attn_blockmask:
+ *     attend(i, j) = q_valid[i] & k_valid[j] & (k_blk[j] <= q_blk[i]); cross
+ *     columns carry k_blk = INT32_MIN; q (B, Sq, H, D), k/v (B, Sk, Hkv, D),
+ *     H % Hkv == 0; output has the dtype of q; is_available / load_error.
+ *   - tensorplay.nn.attention.varlen, "Packed layout": (total_tokens, H, D)
+ *     packing with int32 cumulative lengths starting at 0; under-stated max
+ *     lengths are an error; window_size, out= form, CUDA-only.
+ *   - flashinfer.attention.prims_ts.block_sparse_attention, Parameters: BSR
+ *     block_indptr [B, Hkv, ceil(Sq/q_block_size)+1] / block_indices, canonical
+ *     rows validated synchronously, mask_type dense|causal, plan once outside
+ *     graph capture and capture only the run, caller-owned out.
+ *   - tensorplay.nn.attention.omni_attention, "Outputs": return_lse.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer unless stated otherwise; a host
+ *     pointer is rejected with BFA_ERR_NOT_DEVICE before anything is launched.
+ *   - The caller owns every input and output buffer.  The library owns plans.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     stream-ordered on it.  bfa_fwd never synchronises and may be captured in a
+ *     CUDA graph; the planners may synchronise once (see each).
+ *   - Errors: a negative bfa_status; bfa_last_error() gives a message (per thread).
+ *     Argument errors are detected on the host before any launch.
+ *   - Tiles are 128 x 128 (BFA_TILE).  bf16 q/k/v/out, head dim D in {64, 128}.
+ */
+#ifndef BFA_H_
+#define BFA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct bfa_plan bfa_plan; /* opaque, library-owned, freed by bfa_plan_destroy */
+
+typedef enum bfa_status {
+  BFA_OK = 0,
+  BFA_ERR_INVALID_ARG = -1,      /* shape, stride, alignment or value out of range      */
+  BFA_ERR_UNSUPPORTED = -2,      /* valid request this build does not implement         */
+  BFA_ERR_NOT_DEVICE = -3,       /* a pointer that must be device memory is not         */
+  BFA_ERR_NONCANONICAL_BSR = -4, /* BSR rows not sorted / unique / in range             */
+  BFA_ERR_CAPACITY = -5,         /* sizes beyond what the library can index or allocate */
+  BFA_ERR_CUDA = -6,             /* a CUDA runtime call failed                          */
+  BFA_ERR_TIMEOUT = -7           /* a device-side wait ran past its bound               */
+} bfa_status;
+
+enum { BFA_TILE = 128 };
+
+typedef enum bfa_plan_kind {
+  BFA_PLAN_DENSE = 1,      /* from a dense (Sq, Sk) bool mask, shared by every batch and head   */
+  BFA_PLAN_BLOCKIDS = 2,   /* from per-token block ids and validity, per batch / sequence       */
+  BFA_PLAN_POSITIONAL = 3, /* causal (+ window) on token positions, per batch / sequence        */
+  BFA_PLAN_BSR = 4         /* from BSR routing, per (batch, kv head)                            */
+} bfa_plan_kind;
+
+/* Host-side description of a plan (no synchronisation needed to read it). */
+typedef struct bfa_plan_info {
+  int32_t kind;           /* bfa_plan_kind                                                        */
+  int32_t varlen;         /* 1: packed THD layout through cu_seqlens                              */
+  int32_t n_groups;       /* row groups: 1 (dense), B (blockids/positional), n_seq (varlen),
+                             B*Hkv (BSR)                                                          */
+  int32_t n_rows;         /* query-tile rows over all groups                                      */
+  int64_t grid_tiles;     /* (row, key tile) positions over all groups = size of the class grid   */
+  int32_t batch;          /* B of the plan (0 for dense plans: any B)                             */
+  int32_t hkv;            /* BSR only: kv heads of the routing; else 0                            */
+  int32_t sq, sk;         /* batched: per-batch lengths; varlen: total packed tokens              */
+  int32_t max_kv_tiles;   /* longest key-tile count of a group                                    */
+  int32_t window_left;    /* -1: no window                                                        */
+  int32_t causal;         /* positional / BSR plans: 1 if kv_idx <= q_idx is applied             */
+} bfa_plan_info;
+
+/* Library version string. */
+const char* bfa_version(void);
+
+/* Message of the last failed call on this thread ("" if none).  The analogue of
+ * opentau's load_error(): a diagnostic string, valid until the next call. */
+const char* bfa_last_error(void);
+
+/* 1 if a device of compute capability 10.0 is present and the kernels can load,
+ * else 0 (message in bfa_last_error).  Mirrors opentau's is_available(). */
+int bfa_is_available(void);
+
+/*
+ * Block ids from padding and block-opening flags (opentau make_att_block_ids).
+ *   pad_masks [B, N] u8 (nonzero = real token), att_masks [B, N] u8 (nonzero =
+ *   the token opens a new block, zero = it continues the current one).
+ *   q_blk[b, i] = number of block openings in att_masks[b, 0..i] (inclusive), so
+ *   tokens before the first opening get id 0.  With n_cross > 0, n_cross key
+ *   columns with id INT32_MIN and validity cross_pad[B, n_cross] are prepended.
+ * Outputs (caller-owned, device): q_blk [B, N] i32, k_blk [B, n_cross + N] i32,
+ *   q_valid [B, N] u8, k_valid [B, n_cross + N] u8.  Row-major, contiguous.
+ * Stream-ordered, no synchronisation.
+ */
+bfa_status bfa_make_block_ids(const uint8_t* pad_masks, const uint8_t* att_masks, int B, int N,
+                              int n_cross, const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk,
+                              uint8_t* q_valid, uint8_t* k_valid, void* stream);
+
+/*
+ * Plan from a dense bool mask (BinFlash preprocessing).
+ *   mask: device, Sq rows of Sk bytes (nonzero = attend), row r at
+ *   mask + r * mask_row_stride (bytes, >= Sk).  Shared by every batch and head.
+ * Tile classes are decided over the in-range pairs of each tile; partial tiles
+ * get 128 rows x 4 uint32 words, bit b of word w = column 32w + b (LSB first).
+ * Stream-ordered, no synchronisation; the mask may be freed once the stream has
+ * passed this call.
+ */
+bfa_status bfa_plan_dense(const uint8_t* mask, int64_t mask_row_stride, int Sq, int Sk, bfa_plan** out,
+                          void* stream);
+
+/*
+ * Plan from the compact block-id form (opentau) or from positions.
+ *   q_blk [B, Sq] / k_blk [B, Sk] i32 (batched) or [total_q] / [total_k] (varlen).
+ *     Both NULL: identity positions local to each sequence, i.e. causal
+ *     kv_idx <= q_idx (top-left aligned).
+ *   q_valid / k_valid u8, same indexing; NULL = all valid.
+ *   cu_seqlens_q / cu_seqlens_k: device i32 [B + 1] starting at 0 for the packed
+ *     THD layout (tensorplay varlen), or NULL for the batched layout.  In varlen
+ *     mode B is the number of sequences, Sq / Sk are ignored, and max_q / max_k
+ *     must be >= every sequence length (under-stating is BFA_ERR_INVALID_ARG).
+ *   window_left: -1 = off; else keys with 0 <= q_pos - k_pos < window_left are
+ *     kept (window of past keys including the query's own position).  Requires
+ *     positional ids and no validity masks.
+ * The kernel evaluates attend(i, j) = q_valid[i] & k_valid[j] & (k_blk[j] <= q_blk[i])
+ * (or the position rule) on partial tiles; the plan keeps its own copy of the ids.
+ * Varlen mode reads cu_seqlens back to the host once (one synchronisation).
+ */
+bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
+                             const uint8_t* k_valid, int B, int Sq, int Sk, const int32_t* cu_seqlens_q,
+                             const int32_t* cu_seqlens_k, int max_q, int max_k, int window_left,
+                             bfa_plan** out, void* stream);
+
+/*
+ * Plan from BSR routing (flashinfer block_sparse_attention).
+ *   indptr [B, Hkv, ceil(Sq/q_block)+1] i32: absolute offsets into indices, each
+ *   (b, hkv) slice non-decreasing; indices [n_indices] i32: KV block ids, each
+ *   row strictly increasing in [0, ceil(Skv/kv_block)).
+ *   q_block == kv_block == 128 (BFA_TILE) in this build.
+ *   causal != 0 applies kv_idx <= q_idx on absolute positions inside the selected
+ *   blocks (mask_type "causal"): blocks below the diagonal become full, blocks on
+ *   it partial, blocks above it are dropped.
+ * Query head h uses the routing of kv head h / (H / Hkv).
+ * Validation runs on the device and is read back synchronously (one sync), like
+ * the page's plan step; non-canonical rows give BFA_ERR_NONCANONICAL_BSR.
+ */
+bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
+                        int Sq, int Skv, int q_block, int kv_block, int causal, bfa_plan** out,
+                        void* stream);
+
+/*
+ * Fused masked attention forward with a prebuilt plan.
+ *   q: batched [B, Sq, H, D] or packed [total_q, H, D]; k, v: [B, Sk, Hkv, D] or
+ *   [total_k, Hkv, D]; bf16; the D axis contiguous.  *_strides = {batch, token,
+ *   head} in elements (batch stride ignored for packed plans); strides and base
+ *   addresses must be multiples of 16 bytes.
+ *   H % Hkv == 0 (query head h reads kv head h / (H / Hkv)); D in {64, 128}.
+ *   scale <= 0 selects 1/sqrt(D).
+ *   out: caller-owned bf16, same logical shape as q, strides o_strides.
+ *   lse: caller-owned f32 or NULL; batched [B, H, Sq], packed [H, total_q],
+ *   natural log.  Rows with no attended key get out = 0 and lse = -inf.
+ *   For dense plans B is free; otherwise B must equal the plan's batch /
+ *   sequence count, and for BSR plans Hkv must equal the routing's.
+ * Asynchronous: a device-side timeout is reported by bfa_plan_device_status().
+ */
+bfa_status bfa_fwd(const bfa_plan* plan, const void* q, const void* k, const void* v,
+                   const int64_t q_strides[3], const int64_t k_strides[3], const int64_t v_strides[3],
+                   int B, int H, int Hkv, int D, float scale, void* out, const int64_t o_strides[3],
+                   float* lse, void* stream);
+
+/* Host-side plan description (no sync). */
+bfa_status bfa_plan_get_info(const bfa_plan* plan, bfa_plan_info* info);
+
+/* Tile statistics over the whole class grid (BinFlash's dispatch statistics);
+ * synchronises `stream`.  n_full + n_partial = number of listed tiles. */
+bfa_status bfa_plan_stats(const bfa_plan* plan, int64_t* n_full, int64_t* n_partial, int64_t* n_empty,
+                          void* stream);
+
+/*
+ * Copy a plan to HOST buffers (for parity checks); synchronises `stream`.
+ * Sizes: row_ptr [n_rows + 1], kv_tile / partial [n_full + n_partial],
+ * fine [n_partial * 512] uint32 (dense plans; partial tiles in list order, 128
+ * rows x 4 words each) or NULL, order [n_rows] (longest row first, ties by row
+ * index), classes [grid_tiles] (0 empty, 1 partial, 2 full; groups in order,
+ * each group row-major over (query tile, key tile)).  Any pointer may be NULL.
+ */
+bfa_status bfa_plan_export(const bfa_plan* plan, int32_t* row_ptr, int32_t* kv_tile, uint8_t* partial,
+                           uint32_t* fine, int32_t* order, uint8_t* classes, void* stream);
+
+/* Synchronise `stream` and report BFA_ERR_TIMEOUT if a kernel that used the plan
+ * hit its wait bound since the last call (the flag is then cleared). */
+bfa_status bfa_plan_device_status(const bfa_plan* plan, void* stream);
+
+/* Free a plan in stream order on the stream it was built on.  Work on other
+ * streams that reads the plan must be ordered before this call.  NULL is a no-op. */
+void bfa_plan_destroy(bfa_plan* plan);
+
+/* Bound, in nanoseconds, on every device-side wait of the kernels launched after
+ * this call (default 1e9, i.e. one second).  0 restores the default. */
+void bfa_set_wait_timeout_ns(uint64_t ns);
+
+/* Launch a one-thread-block kernel that waits, with the current bound, on a
+ * barrier phase that nothing completes, and synchronise.  Returns
+ * BFA_ERR_TIMEOUT when the bounded wait gives up as designed (and the context
+ * stays usable), BFA_OK never.  Exercises the failure path without a fault. */
+bfa_status bfa_selftest_wait_timeout(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BFA_H_ */

@@ -1,0 +1,256 @@
+"""Mask-aware fused attention forward for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libbfa.so`` (``include/bfa.h``).  The
+binding only marshals torch tensors into device pointers, sizes, strides and the
+current CUDA stream; every step of the computation runs in the library's CUDA
+kernels.  There is no CPU path: CPU tensors are rejected by the library.
+
+    plan = plan_dense(mask)                      # (Sq, Sk) bool, True = attend
+    out, lse = fwd(plan, q, k, v)                # q (B, Sq, H, D), k/v (B, Sk, Hkv, D)
+
+Other mask sources: ``plan_blockids`` (opentau block ids, positions, varlen,
+sliding window) and ``plan_bsr`` (BSR routing); ``make_att_block_ids`` builds
+block ids from padding and block-opening flags.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import BfaError, PlanInfo
+
+__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_bsr", "fwd", "make_att_block_ids",
+           "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "library_path"]
+
+TILE = 128
+KIND_NAMES = {1: "dense", 2: "blockids", 3: "positional", 4: "bsr"}
+
+library_path = _lib.LIB_PATH
+_L = _lib.load()
+
+
+def _stream(stream=None):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _u8(t):
+    if t is None:
+        return None
+    if t.dtype == torch.bool:
+        return t
+    return (t != 0)
+
+
+def is_available():
+    """True if a B200-class device is present and the kernels load (opentau is_available)."""
+    return bool(_L.bfa_is_available())
+
+
+def load_error():
+    """Message of the last failed library call on this thread, or None."""
+    m = _L.bfa_last_error().decode(errors="replace")
+    return m or None
+
+
+def set_wait_timeout_ns(ns):
+    _L.bfa_set_wait_timeout_ns(int(ns))
+
+
+def selftest_wait_timeout(stream=None):
+    """Run the library's bounded-wait self test; returns the status name."""
+    return _lib.STATUS.get(_L.bfa_selftest_wait_timeout(_stream(stream)))
+
+
+class Plan:
+    """A library-owned tile plan; freed when garbage collected or by ``destroy()``."""
+
+    def __init__(self, handle, stream):
+        self._h = handle
+        self._stream = stream
+        info = PlanInfo()
+        _lib.check(_L.bfa_plan_get_info(self._h, ctypes.byref(info)))
+        self.info = {f: getattr(info, f) for f, _ in PlanInfo._fields_}
+        self.kind = KIND_NAMES[self.info["kind"]]
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise RuntimeError("plan was destroyed")
+        return self._h
+
+    def destroy(self):
+        if self._h is not None:
+            _L.bfa_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+    def stats(self, stream=None):
+        f, p, e = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _lib.check(_L.bfa_plan_stats(self.handle, ctypes.byref(f), ctypes.byref(p), ctypes.byref(e),
+                                     _stream(stream)))
+        return f.value, p.value, e.value
+
+    def device_status(self, stream=None):
+        """Raise BfaError(BFA_ERR_TIMEOUT) if a kernel using this plan hit its wait bound."""
+        _lib.check(_L.bfa_plan_device_status(self.handle, _stream(stream)))
+
+    def export(self, stream=None):
+        """Host copy: row_ptr, kv_tile, partial, fine (dense plans), order, classes."""
+        n_full, n_part, _ = self.stats(stream)
+        R = self.info["n_rows"]
+        nnz = n_full + n_part
+        row_ptr = np.zeros(R + 1, np.int32)
+        kv_tile = np.zeros(max(nnz, 1), np.int32)
+        partial = np.zeros(max(nnz, 1), np.uint8)
+        fine = np.zeros((max(n_part, 1), TILE, 4), np.uint32) if self.kind == "dense" else None
+        order = np.zeros(max(R, 1), np.int32)
+        classes = np.zeros(max(self.info["grid_tiles"], 1), np.uint8)
+        P = lambda a: a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+        _lib.check(_L.bfa_plan_export(self.handle, P(row_ptr), P(kv_tile), P(partial), P(fine), P(order),
+                                      P(classes), _stream(stream)))
+        out = dict(row_ptr=row_ptr, kv_tile=kv_tile[:nnz], partial=partial[:nnz], order=order[:R],
+                   classes=classes[:self.info["grid_tiles"]])
+        if fine is not None:
+            out["fine"] = fine[:n_part]
+        return out
+
+
+def make_att_block_ids(pad_masks, att_masks, n_cross_att_tokens=None, cross_att_pad_masks=None, stream=None):
+    """(q_blk, k_blk, q_valid, k_valid) from padding and block-opening flags (opentau).
+
+    pad_masks / att_masks: (B, N) bool or integer CUDA tensors; cross columns with
+    block id INT32_MIN are prepended when ``n_cross_att_tokens`` is given.
+    """
+    pad = _u8(pad_masks).contiguous()
+    att = _u8(att_masks).contiguous()
+    B, N = pad.shape
+    nc = int(n_cross_att_tokens or 0)
+    cpad = _u8(cross_att_pad_masks).contiguous() if nc else None
+    dev = pad.device
+    q_blk = torch.empty((B, N), dtype=torch.int32, device=dev)
+    k_blk = torch.empty((B, nc + N), dtype=torch.int32, device=dev)
+    q_valid = torch.empty((B, N), dtype=torch.bool, device=dev)
+    k_valid = torch.empty((B, nc + N), dtype=torch.bool, device=dev)
+    _lib.check(_L.bfa_make_block_ids(_ptr(pad), _ptr(att), B, N, nc, _ptr(cpad), _ptr(q_blk), _ptr(k_blk),
+                                     _ptr(q_valid), _ptr(k_valid), _stream(stream)))
+    return q_blk, k_blk, q_valid, k_valid
+
+
+def plan_dense(mask, stream=None):
+    """Plan from a dense (Sq, Sk) bool CUDA mask (True = attend), shared by all batches/heads."""
+    if mask.dim() != 2:
+        raise ValueError("mask must be 2-D (Sq, Sk)")
+    m = mask if mask.dtype in (torch.bool, torch.uint8) else (mask != 0)
+    if m.stride(1) != 1:
+        m = m.contiguous()
+    h = ctypes.c_void_p()
+    st = _stream(stream)
+    _lib.check(_L.bfa_plan_dense(_ptr(m), m.stride(0), m.shape[0], m.shape[1], ctypes.byref(h), st))
+    return Plan(h, st)
+
+
+def plan_blockids(q_blk=None, k_blk=None, q_valid=None, k_valid=None, *, B=None, Sq=None, Sk=None,
+                  cu_seqlens_q=None, cu_seqlens_k=None, max_q=0, max_k=0, window_left=-1, stream=None):
+    """Plan from block ids / validity (opentau) or, with ids None, from causal positions.
+
+    Batched: ids (B, Sq) / (B, Sk).  Varlen: ids over packed tokens, ``cu_seqlens_*``
+    int32 (B + 1,) starting at 0, ``max_q`` / ``max_k`` >= every sequence length.
+    ``window_left`` > 0 keeps keys with 0 <= q_pos - k_pos < window_left.
+    """
+    varlen = cu_seqlens_q is not None
+    if varlen:
+        B = cu_seqlens_q.numel() - 1
+        Sq = Sk = 0
+    elif q_blk is not None:
+        B, Sq = q_blk.shape
+        Sk = k_blk.shape[1]
+    elif q_valid is not None:
+        B, Sq = q_valid.shape
+        Sk = k_valid.shape[1] if k_valid is not None else Sk
+    for t in (q_blk, k_blk):
+        if t is not None and t.dtype != torch.int32:
+            raise TypeError("block ids must be int32")
+    qv = _u8(q_valid).contiguous() if q_valid is not None else None
+    kv = _u8(k_valid).contiguous() if k_valid is not None else None
+    qb = q_blk.contiguous() if q_blk is not None else None
+    kb = k_blk.contiguous() if k_blk is not None else None
+    cq = cu_seqlens_q.to(torch.int32).contiguous() if varlen else None
+    ck = (cu_seqlens_k if cu_seqlens_k is not None else cu_seqlens_q).to(torch.int32).contiguous() if varlen else None
+    h = ctypes.c_void_p()
+    st = _stream(stream)
+    _lib.check(_L.bfa_plan_blockids(_ptr(qb), _ptr(kb), _ptr(qv), _ptr(kv), int(B), int(Sq or 0), int(Sk or 0),
+                                    _ptr(cq), _ptr(ck), int(max_q), int(max_k), int(window_left),
+                                    ctypes.byref(h), st))
+    return Plan(h, st)
+
+
+def plan_bsr(block_indptr, block_indices, Sq, Skv, q_block_size=TILE, kv_block_size=TILE, causal=False,
+             stream=None):
+    """Plan from BSR routing: indptr (B, Hkv, ceil(Sq/q_block)+1) int32, indices int32."""
+    ip = block_indptr.to(torch.int32).contiguous()
+    ix = block_indices.to(torch.int32).contiguous()
+    B, Hkv, _ = ip.shape
+    h = ctypes.c_void_p()
+    st = _stream(stream)
+    _lib.check(_L.bfa_plan_bsr(_ptr(ip), _ptr(ix) if ix.numel() else None, ix.numel(), B, Hkv, int(Sq), int(Skv),
+                               int(q_block_size), int(kv_block_size), 1 if causal else 0, ctypes.byref(h), st))
+    return Plan(h, st)
+
+
+def _strides3(t):
+    if t.dim() == 4:
+        return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+    if t.dim() == 3:
+        return (ctypes.c_int64 * 3)(0, t.stride(0), t.stride(1))
+    raise ValueError("expected a 4-D (B, S, H, D) or 3-D (T, H, D) tensor")
+
+
+def fwd(plan, q, k, v, scale=None, out=None, return_lse=True, lse=None, stream=None):
+    """Masked attention forward; returns (out, lse or None).
+
+    Batched q (B, Sq, H, D), k/v (B, Sk, Hkv, D); packed (varlen plans) q (Tq, H, D),
+    k/v (Tk, Hkv, D).  bf16, last dim contiguous, D in {64, 128}.
+    """
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("q, k, v must be bfloat16")
+        if t.stride(-1) != 1:
+            raise ValueError("the head dim of q, k, v must be contiguous")
+    packed = q.dim() == 3
+    if packed:
+        B = plan.info["batch"]
+        _, H, D = q.shape
+        Hkv = k.shape[1]
+        lse_shape = (H, q.shape[0])
+    else:
+        B, Sq, H, D = q.shape
+        Hkv = k.shape[2]
+        lse_shape = (B, H, Sq)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    sc = float(scale) if scale is not None else 0.0
+    _lib.check(_L.bfa_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _strides3(q), _strides3(k), _strides3(v),
+                          int(B), int(H), int(Hkv), int(D), ctypes.c_float(sc), _ptr(out), _strides3(out),
+                          _ptr(lse), _stream(stream)))
+    return out, lse

@@ -1,0 +1,717 @@
+// Host side of the C ABI declared in include/bfa.h: argument validation, plan
+// allocation and layout, TMA tensor maps, and the kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/bfa.h"
+#include "fwd_params.cuh"
+#include "plan_types.cuh"
+
+#define BFA_API extern "C" __attribute__((visibility("default")))
+
+namespace bfa {
+
+// kernels (planner.cu, fwd.cu)
+cudaError_t launch_dense_classify(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* cls, uint32_t* fine,
+                                  cudaStream_t s);
+cudaError_t launch_blockid_classify(const GroupInfo* groups, int n_groups, int max_tiles_q, int max_tiles_k,
+                                    const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
+                                    const uint8_t* k_valid, int batched, int Sq, int Sk, int window, int copy_ids,
+                                    int32_t* qid, uint8_t* qv, int32_t* kid, uint32_t* kbits, uint8_t* cls,
+                                    cudaStream_t s);
+cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, int64_t n_indices,
+                                const GroupInfo* groups, int n_groups, int nqt, int causal, uint8_t* cls,
+                                uint32_t* err, int32_t* max_width, cudaStream_t s);
+cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
+                        int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
+                        int32_t* order, cudaStream_t s);
+cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
+                                  const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
+                                  uint8_t* k_valid, cudaStream_t s);
+
+
+}  // namespace bfa
+
+using namespace bfa;
+
+// ----------------------------------------------------------------------------
+// plan object
+// ----------------------------------------------------------------------------
+struct bfa_plan {
+  int kind = 0, varlen = 0, batch = 0, hkv = 0, sq = 0, sk = 0, window = -1, causal = 0;
+  int n_groups = 0, n_rows = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
+  int64_t grid_tiles = 0;
+  std::vector<GroupInfo> groups_h;
+  cudaStream_t stream = nullptr;
+  void* slab = nullptr;
+  // device arrays inside the slab
+  GroupInfo* groups = nullptr;
+  int32_t* row_group = nullptr;
+  uint8_t* cls = nullptr;
+  int32_t* row_cnt = nullptr;
+  int32_t* row_ptr = nullptr;
+  int32_t* kv_tile = nullptr;
+  int32_t* part = nullptr;
+  uint32_t* fine = nullptr;
+  int32_t* order = nullptr;
+  int32_t* qid = nullptr;
+  uint8_t* qvalid = nullptr;
+  int32_t* kid = nullptr;
+  uint32_t* kbits = nullptr;
+  uint32_t* err = nullptr;
+  int32_t* max_width = nullptr;
+};
+
+namespace {
+
+thread_local std::string g_err;
+uint64_t g_wait_ns = 1000000000ull;
+
+bfa_status fail(bfa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+bfa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BFA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define BFA_CUDA(call, what)                  \
+  do {                                        \
+    cudaError_t e_ = (call);                  \
+    if (e_ != cudaSuccess) {                  \
+      cleanup();                              \
+      return cuda_fail(e_, what);             \
+    }                                         \
+  } while (0)
+
+// BFA_ERR_NOT_DEVICE unless p is device (or managed) memory.
+bfa_status need_device(const void* p, const char* name, bool allow_null = false) {
+  if (p == nullptr) {
+    if (allow_null) return BFA_OK;
+    return fail(BFA_ERR_INVALID_ARG, "%s is NULL", name);
+  }
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(BFA_ERR_NOT_DEVICE, "%s is not a device pointer (%s)", name, cudaGetErrorString(e));
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(BFA_ERR_NOT_DEVICE, "%s is not device memory (CPU tensors are not supported)", name);
+  return BFA_OK;
+}
+
+inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct SlabLayout {
+  size_t off = 0;
+  template <typename T>
+  size_t take(size_t count) {
+    const size_t o = off;
+    off = align256(off + count * sizeof(T));
+    return o;
+  }
+};
+
+// Allocate and carve the plan slab; uploads groups and row_group.
+bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t kid_elems, int64_t kbit_words) {
+  SlabLayout L;
+  const int64_t cap_tiles = std::max<int64_t>(P->grid_tiles, 1);
+  const size_t o_groups = L.take<GroupInfo>(std::max(P->n_groups, 1));
+  const size_t o_rowg = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_cls = L.take<uint8_t>(cap_tiles);
+  const size_t o_cnt = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_ptr = L.take<int32_t>(P->n_rows + 1);
+  const size_t o_kv = L.take<int32_t>(cap_tiles);
+  const size_t o_part = L.take<int32_t>(cap_tiles);
+  const size_t o_ord = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_err = L.take<uint32_t>(1);
+  const size_t o_mw = L.take<int32_t>(1);
+  const size_t o_qid = L.take<int32_t>(std::max<int64_t>(qid_elems, 1));
+  const size_t o_qv = L.take<uint8_t>(std::max<int64_t>(qid_elems, 1));
+  const size_t o_kid = L.take<int32_t>(std::max<int64_t>(kid_elems, 1));
+  const size_t o_kb = L.take<uint32_t>(std::max<int64_t>(kbit_words, 1));
+  const size_t o_fine = L.take<uint32_t>(with_fine ? static_cast<size_t>(cap_tiles) * kFineWordsPerTile : 1);
+  cudaError_t e = cudaMallocAsync(&P->slab, L.off, P->stream);
+  if (e != cudaSuccess) return fail(BFA_ERR_CAPACITY, "plan allocation of %zu bytes failed: %s", L.off,
+                                    cudaGetErrorString(e));
+  uint8_t* base = static_cast<uint8_t*>(P->slab);
+  P->groups = reinterpret_cast<GroupInfo*>(base + o_groups);
+  P->row_group = reinterpret_cast<int32_t*>(base + o_rowg);
+  P->cls = base + o_cls;
+  P->row_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
+  P->row_ptr = reinterpret_cast<int32_t*>(base + o_ptr);
+  P->kv_tile = reinterpret_cast<int32_t*>(base + o_kv);
+  P->part = reinterpret_cast<int32_t*>(base + o_part);
+  P->order = reinterpret_cast<int32_t*>(base + o_ord);
+  P->err = reinterpret_cast<uint32_t*>(base + o_err);
+  P->max_width = reinterpret_cast<int32_t*>(base + o_mw);
+  P->qid = reinterpret_cast<int32_t*>(base + o_qid);
+  P->qvalid = base + o_qv;
+  P->kid = reinterpret_cast<int32_t*>(base + o_kid);
+  P->kbits = reinterpret_cast<uint32_t*>(base + o_kb);
+  P->fine = reinterpret_cast<uint32_t*>(base + o_fine);
+
+  std::vector<int32_t> rg(std::max(P->n_rows, 1), 0);
+  for (int g = 0; g < P->n_groups; ++g)
+    for (int r = 0; r < P->groups_h[g].nqt; ++r) rg[P->groups_h[g].row0 + r] = g;
+  if (P->n_groups > 0) {
+    e = cudaMemcpyAsync(P->groups, P->groups_h.data(), sizeof(GroupInfo) * P->n_groups, cudaMemcpyHostToDevice,
+                        P->stream);
+    if (e != cudaSuccess) return cuda_fail(e, "upload plan groups");
+  }
+  e = cudaMemcpyAsync(P->row_group, rg.data(), sizeof(int32_t) * rg.size(), cudaMemcpyHostToDevice, P->stream);
+  if (e != cudaSuccess) return cuda_fail(e, "upload plan rows");
+  e = cudaMemsetAsync(P->err, 0, 2 * 256, P->stream);  // err and max_width slots
+  if (e != cudaSuccess) return cuda_fail(e, "clear plan status");
+  return BFA_OK;
+}
+
+void free_plan(bfa_plan* P) {
+  if (!P) return;
+  if (P->slab) cudaFreeAsync(P->slab, P->stream);
+  delete P;
+}
+
+// Finish the plan: groups laid out, classes written -> lists and order.
+bfa_status build_rows(bfa_plan* P) {
+  if (P->n_rows == 0) {
+    cudaError_t e = cudaMemsetAsync(P->row_ptr, 0, sizeof(int32_t), P->stream);
+    return e == cudaSuccess ? BFA_OK : cuda_fail(e, "empty plan");
+  }
+  if (P->max_nkt + 1 > 50000) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
+  cudaError_t e = launch_rows(P->groups, P->row_group, P->cls, P->n_rows, P->max_nkt, P->row_cnt, P->row_ptr,
+                              P->kv_tile, P->part, P->order, P->stream);
+  return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
+}
+
+void finalize_layout(bfa_plan* P) {
+  int row = 0;
+  int64_t cls = 0;
+  P->max_nkt = 0;
+  P->max_nqt = 0;
+  for (auto& g : P->groups_h) {
+    g.row0 = row;
+    g.cls_off = cls;
+    row += g.nqt;
+    cls += static_cast<int64_t>(g.nqt) * g.nkt;
+    P->max_nkt = std::max(P->max_nkt, g.nkt);
+    P->max_nqt = std::max(P->max_nqt, g.nqt);
+  }
+  P->n_rows = row;
+  P->grid_tiles = cls;
+  P->n_groups = static_cast<int>(P->groups_h.size());
+}
+
+GroupInfo make_group(int q_off, int q_len, int k_off, int k_len, int b, int hkv) {
+  GroupInfo g;
+  std::memset(&g, 0, sizeof(g));
+  g.q_off = q_off;
+  g.q_len = q_len;
+  g.k_off = k_off;
+  g.k_len = k_len;
+  g.b = b;
+  g.hkv = hkv;
+  g.nqt = cdiv(q_len, kTile);
+  g.nkt = cdiv(k_len, kTile);
+  return g;
+}
+
+bfa_status check_capacity(const bfa_plan* P, bool with_fine) {
+  if (P->grid_tiles >= (int64_t(1) << 31)) return fail(BFA_ERR_CAPACITY, "class grid of %lld tiles exceeds int32",
+                                                       (long long)P->grid_tiles);
+  if (with_fine && P->grid_tiles * 2048 > (int64_t(64) << 30))
+    return fail(BFA_ERR_CAPACITY, "fine-mask capacity %lld bytes too large", (long long)(P->grid_tiles * 2048));
+  return BFA_OK;
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------------------
+// C ABI
+// ----------------------------------------------------------------------------
+BFA_API const char* bfa_version(void) { return "bfa 0.1 (sm_100a)"; }
+
+BFA_API const char* bfa_last_error(void) { return g_err.c_str(); }
+
+BFA_API int bfa_is_available(void) {
+  int n = 0;
+  cudaError_t e = cudaGetDeviceCount(&n);
+  if (e != cudaSuccess || n == 0) {
+    cudaGetLastError();
+    fail(BFA_ERR_CUDA, "no CUDA device: %s", e == cudaSuccess ? "count is 0" : cudaGetErrorString(e));
+    return 0;
+  }
+  int dev = 0, major = 0, minor = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) {
+    fail(BFA_ERR_UNSUPPORTED, "device is sm_%d%d; these kernels are built for sm_100a only", major, minor);
+    return 0;
+  }
+  e = probe_fwd_kernels();
+  if (e != cudaSuccess) {
+    fail(BFA_ERR_CUDA, "kernel image does not load: %s", cudaGetErrorString(e));
+    return 0;
+  }
+  return 1;
+}
+
+BFA_API void bfa_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : 1000000000ull; }
+
+BFA_API bfa_status bfa_make_block_ids(const uint8_t* pad_masks, const uint8_t* att_masks, int B, int N, int n_cross,
+                                      const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
+                                      uint8_t* k_valid, void* stream) {
+  if (B <= 0 || N <= 0 || n_cross < 0) return fail(BFA_ERR_INVALID_ARG, "bad sizes B=%d N=%d n_cross=%d", B, N, n_cross);
+  bfa_status s;
+  if ((s = need_device(pad_masks, "pad_masks")) || (s = need_device(att_masks, "att_masks")) ||
+      (s = need_device(q_blk, "q_blk")) || (s = need_device(k_blk, "k_blk")) ||
+      (s = need_device(q_valid, "q_valid")) || (s = need_device(k_valid, "k_valid")))
+    return s;
+  if (n_cross > 0 && (s = need_device(cross_pad, "cross_pad"))) return s;
+  cudaError_t e = launch_make_block_ids(pad_masks, att_masks, B, N, n_cross, cross_pad, q_blk, k_blk, q_valid,
+                                        k_valid, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BFA_OK : cuda_fail(e, "make_block_ids kernel");
+}
+
+BFA_API bfa_status bfa_plan_dense(const uint8_t* mask, int64_t ld, int Sq, int Sk, bfa_plan** out, void* stream) {
+  if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (Sq <= 0 || Sk <= 0) return fail(BFA_ERR_INVALID_ARG, "Sq=%d Sk=%d must be positive", Sq, Sk);
+  if (ld < Sk) return fail(BFA_ERR_INVALID_ARG, "mask_row_stride %lld < Sk %d", (long long)ld, Sk);
+  bfa_status s = need_device(mask, "mask");
+  if (s) return s;
+  bfa_plan* P = new bfa_plan();
+  auto cleanup = [&]() { free_plan(P); };
+  P->kind = BFA_PLAN_DENSE;
+  P->stream = static_cast<cudaStream_t>(stream);
+  P->sq = Sq;
+  P->sk = Sk;
+  P->mask_mode = MASK_BITS;
+  P->groups_h.push_back(make_group(0, Sq, 0, Sk, -1, -1));
+  finalize_layout(P);
+  if ((s = check_capacity(P, true))) { cleanup(); return s; }
+  if ((s = alloc_plan(P, true, 0, 0, 0))) { cleanup(); return s; }
+  BFA_CUDA(launch_dense_classify(mask, ld, Sq, Sk, P->cls, P->fine, P->stream), "dense classify kernel");
+  if ((s = build_rows(P))) { cleanup(); return s; }
+  *out = P;
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
+                                     const uint8_t* k_valid, int B, int Sq, int Sk, const int32_t* cu_q,
+                                     const int32_t* cu_k, int max_q, int max_k, int window_left, bfa_plan** out,
+                                     void* stream) {
+  if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (B <= 0) return fail(BFA_ERR_INVALID_ARG, "B=%d must be positive", B);
+  if ((q_blk == nullptr) != (k_blk == nullptr))
+    return fail(BFA_ERR_INVALID_ARG, "q_blk and k_blk must both be given or both be NULL");
+  if ((cu_q == nullptr) != (cu_k == nullptr))
+    return fail(BFA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must both be given or both be NULL");
+  if (window_left < -1 || window_left == 0) return fail(BFA_ERR_INVALID_ARG, "window_left=%d (use -1 or >= 1)", window_left);
+  const bool positional = q_blk == nullptr;
+  const bool have_valid = q_valid != nullptr || k_valid != nullptr;
+  if (window_left >= 1 && (!positional || have_valid))
+    return fail(BFA_ERR_UNSUPPORTED, "a window needs positional ids and no validity masks");
+  bfa_status s;
+  if ((s = need_device(q_blk, "q_blk", true)) || (s = need_device(k_blk, "k_blk", true)) ||
+      (s = need_device(q_valid, "q_valid", true)) || (s = need_device(k_valid, "k_valid", true)) ||
+      (s = need_device(cu_q, "cu_seqlens_q", true)) || (s = need_device(cu_k, "cu_seqlens_k", true)))
+    return s;
+  const bool varlen = cu_q != nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bfa_plan* P = new bfa_plan();
+  auto cleanup = [&]() { free_plan(P); };
+  P->kind = positional && !have_valid ? BFA_PLAN_POSITIONAL : BFA_PLAN_BLOCKIDS;
+  P->mask_mode = positional && !have_valid ? MASK_POS : MASK_BLOCKID;
+  P->causal = 1;
+  P->window = window_left >= 1 ? window_left : -1;
+  P->varlen = varlen;
+  P->batch = B;
+  P->stream = st;
+  if (varlen) {
+    std::vector<int32_t> cq(B + 1), ck(B + 1);
+    BFA_CUDA(cudaMemcpyAsync(cq.data(), cu_q, sizeof(int32_t) * (B + 1), cudaMemcpyDeviceToHost, st), "read cu_seqlens_q");
+    BFA_CUDA(cudaMemcpyAsync(ck.data(), cu_k, sizeof(int32_t) * (B + 1), cudaMemcpyDeviceToHost, st), "read cu_seqlens_k");
+    BFA_CUDA(cudaStreamSynchronize(st), "read cu_seqlens");
+    if (cq[0] != 0 || ck[0] != 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "cu_seqlens must start at 0"); }
+    for (int i = 0; i < B; ++i) {
+      const int lq = cq[i + 1] - cq[i], lk = ck[i + 1] - ck[i];
+      if (lq < 0 || lk < 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "cu_seqlens decreases at sequence %d", i); }
+      if (lq > max_q || lk > max_k) {
+        cleanup();
+        return fail(BFA_ERR_INVALID_ARG, "sequence %d has lengths (%d, %d) above max_q=%d / max_k=%d", i, lq, lk,
+                    max_q, max_k);
+      }
+      P->groups_h.push_back(make_group(cq[i], lq, ck[i], lk, 0, -1));
+    }
+    P->sq = cq[B];
+    P->sk = ck[B];
+  } else {
+    if (Sq <= 0 || Sk <= 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "Sq=%d Sk=%d must be positive", Sq, Sk); }
+    for (int b = 0; b < B; ++b) P->groups_h.push_back(make_group(0, Sq, 0, Sk, b, -1));
+    P->sq = Sq;
+    P->sk = Sk;
+  }
+  finalize_layout(P);
+  // padded per-group id copies (block-id mode only)
+  int64_t qe = 0, ke = 0, kw = 0;
+  const bool copy_ids = P->mask_mode == MASK_BLOCKID;
+  for (auto& g : P->groups_h) {
+    g.qid_off = static_cast<int32_t>(qe);
+    g.kid_off = static_cast<int32_t>(ke);
+    g.kbit_off = static_cast<int32_t>(kw);
+    if (copy_ids) {
+      qe += static_cast<int64_t>(g.nqt) * kTile;
+      ke += static_cast<int64_t>(g.nkt) * kTile;
+      kw += static_cast<int64_t>(g.nkt) * kWordsPerTileRow;
+    }
+  }
+  if (qe >= (int64_t(1) << 31) || ke >= (int64_t(1) << 31)) { cleanup(); return fail(BFA_ERR_CAPACITY, "too many tokens"); }
+  if ((s = check_capacity(P, false))) { cleanup(); return s; }
+  if ((s = alloc_plan(P, false, qe, ke, kw))) { cleanup(); return s; }
+  if (P->n_groups > 0) {
+    BFA_CUDA(launch_blockid_classify(P->groups, P->n_groups, P->max_nqt, P->max_nkt, q_blk, k_blk, q_valid, k_valid,
+                                     varlen ? 0 : 1, P->sq, P->sk, P->window, copy_ids ? 1 : 0, P->qid, P->qvalid,
+                                     P->kid, P->kbits, P->cls, st),
+             "block-id classify kernel");
+  }
+  if ((s = build_rows(P))) { cleanup(); return s; }
+  *out = P;
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
+                                int Sq, int Skv, int q_block, int kv_block, int causal, bfa_plan** out,
+                                void* stream) {
+  if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (B <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || n_indices < 0)
+    return fail(BFA_ERR_INVALID_ARG, "bad sizes B=%d Hkv=%d Sq=%d Skv=%d n_indices=%lld", B, Hkv, Sq, Skv,
+                (long long)n_indices);
+  if (q_block != kTile || kv_block != kTile)
+    return fail(BFA_ERR_UNSUPPORTED, "q_block=%d kv_block=%d: this build needs both equal to %d", q_block, kv_block,
+                kTile);
+  bfa_status s;
+  if ((s = need_device(indptr, "block_indptr"))) return s;
+  if (n_indices > 0 && (s = need_device(indices, "block_indices"))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bfa_plan* P = new bfa_plan();
+  auto cleanup = [&]() { free_plan(P); };
+  P->kind = BFA_PLAN_BSR;
+  P->mask_mode = MASK_POS;
+  P->causal = causal ? 1 : 0;
+  P->window = -1;
+  P->batch = B;
+  P->hkv = Hkv;
+  P->sq = Sq;
+  P->sk = Skv;
+  P->stream = st;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hkv; ++h) P->groups_h.push_back(make_group(0, Sq, 0, Skv, b, h));
+  finalize_layout(P);
+  if ((s = check_capacity(P, false))) { cleanup(); return s; }
+  if ((s = alloc_plan(P, false, 0, 0, 0))) { cleanup(); return s; }
+  BFA_CUDA(cudaMemsetAsync(P->cls, 0, static_cast<size_t>(std::max<int64_t>(P->grid_tiles, 1)), st), "clear classes");
+  BFA_CUDA(launch_bsr_classify(indptr, indices, n_indices, P->groups, P->n_groups, cdiv(Sq, kTile), P->causal, P->cls,
+                               P->err, P->max_width, st),
+           "BSR classify kernel");
+  uint32_t err = 0;
+  BFA_CUDA(cudaMemcpyAsync(&err, P->err, sizeof(err), cudaMemcpyDeviceToHost, st), "read BSR status");
+  BFA_CUDA(cudaStreamSynchronize(st), "BSR validation");
+  if (err) {
+    cleanup();
+    return fail(BFA_ERR_NONCANONICAL_BSR, "BSR routing is not canonical (%s)",
+                (err & DEVERR_BSR_RANGE) ? "row offsets out of range or decreasing"
+                                          : "block ids unsorted, duplicated or out of range");
+  }
+  if ((s = build_rows(P))) { cleanup(); return s; }
+  *out = P;
+  return BFA_OK;
+}
+
+// ----------------------------------------------------------------------------
+// forward launch: TMA tensor maps + kernel parameters
+// ----------------------------------------------------------------------------
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  }
+  return fn;
+}
+
+// 4-D map over (d, head, token, batch) of a bf16 tensor, box = 64 d x 1 head x
+// 128 tokens x 1 batch, 128-byte swizzle: one 16 KB panel of a 128 x D tile.
+bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int64_t tokens, int batch, int64_t s_head,
+               int64_t s_tok, int64_t s_batch, std::string* why) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  if (s_batch == 0 || batch == 1) s_batch = std::max<int64_t>(s_tok * std::max<int64_t>(tokens, 1), 8);
+  if (s_head == 0) s_head = 8;  // a single head: any aligned stride
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(tokens),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_head) * 2, static_cast<cuuint64_t>(s_tok) * 2,
+                           static_cast<cuuint64_t>(s_batch) * 2};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "tensor map rejected (CUresult %d) for strides (%lld, %lld, %lld)", (int)r,
+             (long long)s_head, (long long)s_tok, (long long)s_batch);
+    *why = buf;
+    return false;
+  }
+  return true;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t* qs,
+                                 const int64_t* ks, const int64_t* vs, int B, int H, int Hkv, int D, float scale,
+                                 void* out, const int64_t* os, float* lse, uint64_t wait_ns, cudaStream_t st,
+                                 std::string* why) {
+  const int bq = P->varlen ? 1 : B;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why) ||
+      !make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], why) ||
+      !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], why))
+    return cudaErrorInvalidValue;
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.plan.groups = P->groups;
+  p.plan.row_group = P->row_group;
+  p.plan.row_ptr = P->row_ptr;
+  p.plan.kv_tile = P->kv_tile;
+  p.plan.part = P->part;
+  p.plan.fine = P->fine;
+  p.plan.order = P->order;
+  p.plan.qid = P->qid;
+  p.plan.qvalid = P->qvalid;
+  p.plan.kid = P->kid;
+  p.plan.kbits = P->kbits;
+  p.plan.err = P->err;
+  p.plan.n_rows = P->n_rows;
+  p.plan.n_groups = P->n_groups;
+  p.plan.mask_mode = P->mask_mode;
+  p.plan.causal = P->causal;
+  p.plan.window = P->window;
+  p.plan.kind = P->kind;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? H / Hkv : H);
+  // Keep enough replicas of a row together to fill about two waves of CTAs, but
+  // no more heads than keep their K/V resident in L2 (about 64 MB).
+  const int64_t waves = 2LL * sm_count() * 2;
+  int chunk = static_cast<int>(std::min<int64_t>(p.rep, std::max<int64_t>(1, (waves + P->n_rows - 1) / std::max(P->n_rows, 1))));
+  const int64_t kv_head_bytes = std::max<int64_t>(1, static_cast<int64_t>(P->sk) * D * 4);
+  const int64_t l2_heads = std::max<int64_t>(1, (64LL << 20) / kv_head_bytes) * std::max(1, H / Hkv);
+  chunk = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(chunk, l2_heads)));
+  p.head_chunk = chunk;
+  p.varlen = P->varlen;
+  p.Sq_lse = P->sq;
+  const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.o_sb = P->varlen ? 0 : os[0];
+  p.o_ss = os[1];
+  p.o_sh = os[2];
+  p.lse = lse;
+  p.wait_ns = wait_ns;
+  const int64_t n_work = static_cast<int64_t>(P->n_rows) * p.rep;
+  return launch_fwd(D, tq, tk, tv, p, n_work, st);
+}
+
+}  // namespace
+
+BFA_API bfa_status bfa_fwd(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t qs[3],
+                           const int64_t ks[3], const int64_t vs[3], int B, int H, int Hkv, int D, float scale,
+                           void* out, const int64_t os[3], float* lse, void* stream) {
+  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  if (!qs || !ks || !vs || !os) return fail(BFA_ERR_INVALID_ARG, "strides are NULL");
+  if (D != 64 && D != 128) return fail(BFA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", D);
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0) return fail(BFA_ERR_INVALID_ARG, "H=%d must be a positive multiple of Hkv=%d", H, Hkv);
+  if (B <= 0) return fail(BFA_ERR_INVALID_ARG, "B=%d must be positive", B);
+  if (P->kind != BFA_PLAN_DENSE && B != P->batch)
+    return fail(BFA_ERR_INVALID_ARG, "B=%d does not match the plan's %d", B, P->batch);
+  if (P->kind == BFA_PLAN_BSR && Hkv != P->hkv)
+    return fail(BFA_ERR_INVALID_ARG, "Hkv=%d does not match the BSR routing's %d", Hkv, P->hkv);
+  bfa_status s;
+  if ((s = need_device(q, "q")) || (s = need_device(k, "k")) || (s = need_device(v, "v")) ||
+      (s = need_device(out, "out")) || (s = need_device(lse, "lse", true)))
+    return s;
+  const int64_t* all[4] = {qs, ks, vs, os};
+  for (int t = 0; t < 4; ++t)
+    for (int i = 0; i < 3; ++i) {
+      if (P->varlen && i == 0) continue;
+      if (all[t][i] < 0 || all[t][i] % 8 != 0)
+        return fail(BFA_ERR_INVALID_ARG, "stride %lld is not a non-negative multiple of 8 elements", (long long)all[t][i]);
+    }
+  const void* ptrs[4] = {q, k, v, out};
+  for (int t = 0; t < 4; ++t)
+    if (reinterpret_cast<uintptr_t>(ptrs[t]) & 15u) return fail(BFA_ERR_INVALID_ARG, "tensor base is not 16-byte aligned");
+  std::string why;
+  cudaError_t e = fwd_launch_from_host(P, q, k, v, qs, ks, vs, B, H, Hkv, D, scale, out, os, lse, g_wait_ns,
+                                       static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) {
+    if (!why.empty()) return fail(BFA_ERR_INVALID_ARG, "%s", why.c_str());
+    return cuda_fail(e, "forward kernel");
+  }
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_get_info(const bfa_plan* P, bfa_plan_info* info) {
+  if (!P || !info) return fail(BFA_ERR_INVALID_ARG, "NULL argument");
+  info->kind = P->kind;
+  info->varlen = P->varlen;
+  info->n_groups = P->n_groups;
+  info->n_rows = P->n_rows;
+  info->grid_tiles = P->grid_tiles;
+  info->batch = P->kind == BFA_PLAN_DENSE ? 0 : P->batch;
+  info->hkv = P->hkv;
+  info->sq = P->sq;
+  info->sk = P->sk;
+  info->max_kv_tiles = P->max_nkt;
+  info->window_left = P->window;
+  info->causal = P->causal;
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_stats(const bfa_plan* P, int64_t* n_full, int64_t* n_partial, int64_t* n_empty,
+                                  void* stream) {
+  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<uint8_t> cls(static_cast<size_t>(P->grid_tiles));
+  auto cleanup = []() {};
+  if (P->grid_tiles > 0) {
+    BFA_CUDA(cudaMemcpyAsync(cls.data(), P->cls, cls.size(), cudaMemcpyDeviceToHost, st), "read classes");
+  }
+  BFA_CUDA(cudaStreamSynchronize(st), "plan stats");
+  int64_t c[3] = {0, 0, 0};
+  for (uint8_t x : cls) c[x < 3 ? x : 0]++;
+  if (n_empty) *n_empty = c[0];
+  if (n_partial) *n_partial = c[1];
+  if (n_full) *n_full = c[2];
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_export(const bfa_plan* P, int32_t* row_ptr, int32_t* kv_tile, uint8_t* partial,
+                                   uint32_t* fine, int32_t* order, uint8_t* classes, void* stream) {
+  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto cleanup = []() {};
+  std::vector<int32_t> rp(P->n_rows + 1);
+  BFA_CUDA(cudaMemcpyAsync(rp.data(), P->row_ptr, sizeof(int32_t) * rp.size(), cudaMemcpyDeviceToHost, st), "read row_ptr");
+  BFA_CUDA(cudaStreamSynchronize(st), "export");
+  const int64_t nnz = rp[P->n_rows];
+  std::vector<int32_t> part(nnz);
+  if (nnz > 0) BFA_CUDA(cudaMemcpyAsync(part.data(), P->part, sizeof(int32_t) * nnz, cudaMemcpyDeviceToHost, st), "read parts");
+  if (row_ptr) std::memcpy(row_ptr, rp.data(), sizeof(int32_t) * rp.size());
+  if (kv_tile && nnz > 0)
+    BFA_CUDA(cudaMemcpyAsync(kv_tile, P->kv_tile, sizeof(int32_t) * nnz, cudaMemcpyDeviceToHost, st), "read lists");
+  if (order && P->n_rows > 0)
+    BFA_CUDA(cudaMemcpyAsync(order, P->order, sizeof(int32_t) * P->n_rows, cudaMemcpyDeviceToHost, st), "read order");
+  if (classes && P->grid_tiles > 0)
+    BFA_CUDA(cudaMemcpyAsync(classes, P->cls, static_cast<size_t>(P->grid_tiles), cudaMemcpyDeviceToHost, st), "read classes");
+  std::vector<uint32_t> fine_all;
+  const bool want_fine = fine && P->mask_mode == MASK_BITS && P->grid_tiles > 0;
+  if (want_fine) {
+    fine_all.resize(static_cast<size_t>(P->grid_tiles) * kFineWordsPerTile);
+    BFA_CUDA(cudaMemcpyAsync(fine_all.data(), P->fine, fine_all.size() * sizeof(uint32_t), cudaMemcpyDeviceToHost, st),
+             "read fine masks");
+  }
+  BFA_CUDA(cudaStreamSynchronize(st), "export");
+  int64_t np = 0;
+  for (int64_t e = 0; e < nnz; ++e) {
+    if (partial) partial[e] = part[e] >= 0 ? 1 : 0;
+    if (part[e] >= 0) {
+      if (want_fine)
+        std::memcpy(fine + np * kFineWordsPerTile, fine_all.data() + static_cast<int64_t>(part[e]) * kFineWordsPerTile,
+                    sizeof(uint32_t) * kFineWordsPerTile);
+      ++np;
+    }
+  }
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_device_status(const bfa_plan* P, void* stream) {
+  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto cleanup = []() {};
+  uint32_t err = 0;
+  BFA_CUDA(cudaMemcpyAsync(&err, P->err, sizeof(err), cudaMemcpyDeviceToHost, st), "read device status");
+  BFA_CUDA(cudaStreamSynchronize(st), "device status");
+  if (err & DEVERR_TIMEOUT) {
+    BFA_CUDA(cudaMemsetAsync(P->err, 0, sizeof(uint32_t), st), "clear device status");
+    BFA_CUDA(cudaStreamSynchronize(st), "device status");
+    return fail(BFA_ERR_TIMEOUT, "a device-side wait exceeded its bound");
+  }
+  return BFA_OK;
+}
+
+BFA_API void bfa_plan_destroy(bfa_plan* P) { free_plan(P); }
+
+BFA_API bfa_status bfa_selftest_wait_timeout(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* d = nullptr;
+  auto cleanup = [&]() {
+    if (d) cudaFreeAsync(d, st);
+  };
+  BFA_CUDA(cudaMallocAsync(&d, sizeof(uint32_t), st), "selftest alloc");
+  BFA_CUDA(cudaMemsetAsync(d, 0, sizeof(uint32_t), st), "selftest clear");
+  BFA_CUDA(launch_wait_selftest(d, g_wait_ns, st), "selftest kernel");
+  uint32_t h = 0;
+  BFA_CUDA(cudaMemcpyAsync(&h, d, sizeof(h), cudaMemcpyDeviceToHost, st), "selftest read");
+  BFA_CUDA(cudaStreamSynchronize(st), "selftest");
+  cleanup();
+  if (h & DEVERR_TIMEOUT) return fail(BFA_ERR_TIMEOUT, "bounded wait gave up as designed");
+  return BFA_OK;
+}
+

@@ -1,0 +1,33 @@
+// Parameters of the fused forward kernel (filled on the host, passed by value).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "plan_types.cuh"
+
+namespace bfa {
+
+struct FwdParams {
+  PlanDev plan;
+  int32_t B, H, Hkv, D;
+  int32_t rep;          // (batch, head) replicas that share one plan row
+  int32_t head_chunk;   // replicas kept together in the work order (K/V reuse in L2)
+  int32_t varlen;
+  int32_t Sq_lse;       // batched: per-batch query length (lse row pitch); varlen: total_q
+  float scale_log2;     // softmax scale * log2(e)
+  __nv_bfloat16* out;
+  int64_t o_sb, o_ss, o_sh;
+  float* lse;
+  uint64_t wait_ns;
+};
+
+int fwd_smem_bytes(int D);
+cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, int64_t n_work, cudaStream_t s);
+cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s);
+cudaError_t probe_fwd_kernels();
+
+}  // namespace bfa

@@ -1,0 +1,65 @@
+// Plan layout shared by the host code, the planner kernels and the forward kernel.
+#pragma once
+
+#include <cstdint>
+
+namespace bfa {
+
+constexpr int kTile = 128;             // query and key tile edge
+constexpr int kWordsPerTileRow = 4;    // 128 columns / 32 bits
+constexpr int kFineWordsPerTile = kTile * kWordsPerTileRow;  // 512 uint32 = 2 KB
+
+enum MaskMode : int32_t {
+  MASK_BITS = 0,     // partial tiles carry packed fine masks (dense plans)
+  MASK_BLOCKID = 1,  // partial tiles evaluate q_valid & k_valid & (k_blk <= q_blk)
+  MASK_POS = 2       // partial tiles evaluate causal (+ window) on positions
+};
+
+enum DevErr : uint32_t {
+  DEVERR_TIMEOUT = 1u,       // a bounded wait gave up
+  DEVERR_BSR_RANGE = 2u,     // BSR offsets out of range / decreasing
+  DEVERR_BSR_ORDER = 4u,     // BSR ids unsorted, duplicated or out of range
+};
+
+// One row group: a batch (batched plans), a sequence (varlen plans), a
+// (batch, kv head) pair (BSR plans) or the single shared group of a dense plan.
+struct GroupInfo {
+  int32_t q_off;      // first query token of the group along the token axis
+  int32_t q_len;      // query tokens
+  int32_t k_off;      // first key token
+  int32_t k_len;      // key tokens
+  int32_t b;          // batch index used for strides (-1: any batch, dense plans)
+  int32_t hkv;        // BSR: kv head of the routing; -1: every head
+  int32_t row0;       // first plan row of the group
+  int32_t nqt;        // query tiles
+  int32_t nkt;        // key tiles
+  int32_t qid_off;    // block-id plans: offset of the group's padded q ids / validity
+  int32_t kid_off;    // block-id plans: offset of the group's padded k ids
+  int32_t kbit_off;   // block-id plans: word offset of the group's k validity bits
+  int64_t cls_off;    // offset of the group's (nqt x nkt) class grid
+};
+static_assert(sizeof(GroupInfo) == 56, "GroupInfo layout");
+
+// Device view of a plan (pointers into the plan's slab).
+struct PlanDev {
+  const GroupInfo* groups;
+  const int32_t* row_group;  // [n_rows]
+  const int32_t* row_ptr;    // [n_rows + 1]
+  const int32_t* kv_tile;    // [listed tiles]
+  const int32_t* part;       // [listed tiles]: -1 full, else the tile's class-grid index
+  const uint32_t* fine;      // [grid_tiles * 512] (dense plans) indexed by grid index
+  const int32_t* order;      // [n_rows] longest first
+  const int32_t* qid;        // padded q block ids  (block-id plans)
+  const uint8_t* qvalid;     // padded q validity   (block-id plans)
+  const int32_t* kid;        // padded k block ids  (block-id plans)
+  const uint32_t* kbits;     // padded k validity bits (block-id plans)
+  uint32_t* err;             // device error word
+  int32_t n_rows;
+  int32_t n_groups;
+  int32_t mask_mode;
+  int32_t causal;
+  int32_t window;            // -1 off
+  int32_t kind;
+};
+
+}  // namespace bfa

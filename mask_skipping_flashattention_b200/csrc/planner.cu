@@ -1,0 +1,442 @@
+// Mask planner kernels: turn a dense mask, block ids / positions, or BSR routing
+// into the tile plan (class grid -> per-row ascending key-tile lists -> longest
+// first row order), plus packed fine masks for the partial tiles of dense masks.
+//
+// The method is BinFlash's preprocessing ("Efficiently Dispatching FlashAttention
+// For Partially Filled Attention Masks": coarse block mask + 32-bit packed fine
+// mask + pre-sorted non-empty key-block lists), with the block-id rule of
+// opentau flash_attn_cuda and the BSR routing of flashinfer block_sparse_attention
+// as the other two mask sources.  Everything is deterministic: counts are integer
+// reductions, lists come from ballot prefix sums, and the order is a stable
+// counting sort.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "plan_types.cuh"
+
+namespace bfa {
+
+// ----------------------------------------------------------------------------
+// dense mask -> classes + fine words
+// ----------------------------------------------------------------------------
+// Grid (ceil(nkt / 4), nqt); 256 threads.  A CTA reads a 128-row band of 4 key
+// tiles (512 columns): lane L of a warp covers 16 columns (tile L / 8, chunk L % 8)
+// with one 16-byte load per row, so each warp instruction reads 512 contiguous
+// mask bytes.  Each warp owns 16 rows.
+constexpr int kDenseTilesPerCta = 4;
+
+__device__ __forceinline__ uint32_t nz_bytes4(uint32_t x) {
+  // bit k (k < 4) set iff byte k of x is nonzero
+  uint32_t t = x | (x >> 4);
+  t |= t >> 2;
+  t |= t >> 1;
+  t &= 0x01010101u;
+  return ((t * 0x01020408u) >> 24) & 0xFu;
+}
+
+__global__ void __launch_bounds__(256) k_dense_classify(const uint8_t* __restrict__ mask, int64_t ld, int Sq,
+                                                        int Sk, int nkt, uint8_t* __restrict__ cls,
+                                                        uint32_t* __restrict__ fine, int vec_ok) {
+  __shared__ uint32_t words[kDenseTilesPerCta][kTile][kWordsPerTileRow];  // 8 KB
+  __shared__ int tile_cnt[kDenseTilesPerCta];
+  const int qt = blockIdx.y;
+  const int kt0 = blockIdx.x * kDenseTilesPerCta;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < kDenseTilesPerCta) tile_cnt[threadIdx.x] = 0;
+  const int t = lane >> 3, chunk = lane & 7;
+  const int64_t col0 = static_cast<int64_t>(kt0 + t) * kTile + chunk * 16;
+  const int rows_here = min(kTile, Sq - qt * kTile);
+
+  uint32_t m16[16];
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) {
+    const int r = warp * 16 + rr;
+    uint32_t m = 0;
+    if (r < rows_here && col0 < Sk) {
+      const uint8_t* p = mask + static_cast<int64_t>(qt * kTile + r) * ld + col0;
+      if (vec_ok && col0 + 16 <= Sk) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        m = nz_bytes4(v.x) | (nz_bytes4(v.y) << 4) | (nz_bytes4(v.z) << 8) | (nz_bytes4(v.w) << 12);
+      } else {
+        for (int c = 0; c < 16; ++c)
+          if (col0 + c < Sk && p[c] != 0) m |= 1u << c;
+      }
+    }
+    m16[rr] = m;
+  }
+  int cnt = 0;
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) {
+    const uint32_t hi = __shfl_down_sync(0xffffffffu, m16[rr], 1);
+    cnt += __popc(m16[rr]);
+    if ((chunk & 1) == 0) words[t][warp * 16 + rr][chunk >> 1] = m16[rr] | (hi << 16);
+  }
+  // reduce the counts of the 8 lanes of each tile
+  cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
+  cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
+  cnt += __shfl_xor_sync(0xffffffffu, cnt, 4);
+  __syncthreads();  // tile_cnt zeroed
+  if (chunk == 0) atomicAdd(&tile_cnt[t], cnt);
+  __syncthreads();
+  for (int tt = 0; tt < kDenseTilesPerCta; ++tt) {
+    const int kt = kt0 + tt;
+    if (kt >= nkt) break;
+    const int cols = min(kTile, Sk - kt * kTile);
+    const int n_in = rows_here * cols;
+    const int c = tile_cnt[tt];
+    const int klass = (c == 0) ? 0 : (c == n_in ? 2 : 1);
+    const int64_t gidx = static_cast<int64_t>(qt) * nkt + kt;
+    if (threadIdx.x == 0) cls[gidx] = static_cast<uint8_t>(klass);
+    if (klass == 1) {
+      uint32_t* dst = fine + gidx * kFineWordsPerTile;
+      const uint32_t* src = &words[tt][0][0];
+      for (int i = threadIdx.x; i < kFineWordsPerTile; i += blockDim.x) dst[i] = src[i];
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// block ids / positions -> padded id copies + classes (one CTA per group)
+// ----------------------------------------------------------------------------
+struct TileStat {
+  int32_t lo, hi;   // min / max id over valid in-range tokens of the tile
+  int32_t any, all; // any valid, all in-range tokens valid
+};
+
+__device__ __forceinline__ void warp_minmax(int32_t& lo, int32_t& hi, int32_t& any, int32_t& all) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  any = __any_sync(0xffffffffu, any);
+  all = __all_sync(0xffffffffu, all);
+}
+
+// Stats of one tile of `len` tokens starting at local index `t0`; copies the ids
+// and validity into the padded arrays when requested.  One warp.
+__device__ TileStat tile_stats(const int32_t* ids, const uint8_t* valid, int tok0, int len, int t0,
+                               int32_t* out_id, uint8_t* out_valid, uint32_t* out_bits, int lane) {
+  int32_t lo = INT32_MAX, hi = INT32_MIN, any = 0, all = 1;
+  for (int c = 0; c < kTile / 32; ++c) {
+    const int j = t0 + c * 32 + lane;   // local index
+    const bool in = j < len;
+    int32_t id = in ? (ids ? ids[tok0 + j] : j) : INT32_MAX;
+    const bool v = in && (valid ? valid[tok0 + j] != 0 : true);
+    if (v) {
+      lo = min(lo, id);
+      hi = max(hi, id);
+      any = 1;
+    }
+    if (in && !v) all = 0;
+    if (out_id) out_id[t0 + c * 32 + lane] = in ? id : INT32_MAX;
+    if (out_valid) out_valid[t0 + c * 32 + lane] = v ? 1 : 0;
+    const uint32_t bits = __ballot_sync(0xffffffffu, v);
+    if (out_bits && lane == 0) out_bits[(t0 >> 5) + c] = bits;
+  }
+  warp_minmax(lo, hi, any, all);
+  return TileStat{lo, hi, any, all};
+}
+
+__global__ void __launch_bounds__(256) k_blockid_classify(const GroupInfo* __restrict__ groups,
+                                                          const int32_t* __restrict__ q_blk,
+                                                          const int32_t* __restrict__ k_blk,
+                                                          const uint8_t* __restrict__ q_valid,
+                                                          const uint8_t* __restrict__ k_valid, int batched,
+                                                          int Sq, int Sk, int window, int copy_ids,
+                                                          int32_t* qid, uint8_t* qv, int32_t* kid,
+                                                          uint32_t* kbits, uint8_t* cls) {
+  extern __shared__ TileStat st[];  // nqt + nkt entries
+  const GroupInfo g = groups[blockIdx.x];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  // token offsets of the group inside the caller's id / validity arrays
+  const int qtok = batched ? g.b * Sq : g.q_off;
+  const int ktok = batched ? g.b * Sk : g.k_off;
+  TileStat* sq = st;
+  TileStat* sk = st + g.nqt;
+  for (int qt = warp; qt < g.nqt; qt += nw)
+    sq[qt] = tile_stats(q_blk, q_valid, qtok, g.q_len, qt * kTile, copy_ids ? qid + g.qid_off : nullptr,
+                        copy_ids ? qv + g.qid_off : nullptr, nullptr, lane);
+  for (int kt = warp; kt < g.nkt; kt += nw)
+    sk[kt] = tile_stats(k_blk, k_valid, ktok, g.k_len, kt * kTile, copy_ids ? kid + g.kid_off : nullptr,
+                        nullptr, copy_ids ? kbits + g.kbit_off : nullptr, lane);
+  __syncthreads();
+  const int64_t n = static_cast<int64_t>(g.nqt) * g.nkt;
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) {
+    const int qt = static_cast<int>(e / g.nkt), kt = static_cast<int>(e % g.nkt);
+    const TileStat a = sq[qt], b = sk[kt];
+    // attend(i, j) = valid_i & valid_j & id_j <= id_i   [& i - j < window on positions]
+    bool exists = a.any && b.any && b.lo <= a.hi;
+    bool full = a.all && b.all && b.hi <= a.lo;
+    if (window >= 0) {
+      // positions: i - j ranges over [lo_q - hi_k, hi_q - lo_k] without gaps
+      exists = exists && (a.lo - b.hi) < window;
+      full = full && (a.hi - b.lo) < window;
+    }
+    cls[g.cls_off + e] = static_cast<uint8_t>(exists ? (full ? 2 : 1) : 0);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// BSR routing -> validation + classes (one thread per BSR row)
+// ----------------------------------------------------------------------------
+__global__ void k_bsr_classify(const int32_t* __restrict__ indptr, const int32_t* __restrict__ indices,
+                               int64_t n_indices, const GroupInfo* __restrict__ groups, int n_groups,
+                               int nqt, int causal, uint8_t* cls, uint32_t* err, int32_t* max_width) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= static_cast<int64_t>(n_groups) * nqt) return;
+  const int grp = static_cast<int>(gid / nqt), qt = static_cast<int>(gid % nqt);
+  const GroupInfo g = groups[grp];
+  const int32_t* ip = indptr + static_cast<int64_t>(grp) * (nqt + 1);
+  const int32_t a = ip[qt], b = ip[qt + 1];
+  if (a < 0 || b < a || static_cast<int64_t>(b) > n_indices) {
+    atomicOr(err, DEVERR_BSR_RANGE);
+    return;
+  }
+  atomicMax(max_width, b - a);
+  const int i0 = qt * kTile, i1 = min(g.q_len, i0 + kTile) - 1;
+  int32_t prev = -1;
+  for (int32_t e = a; e < b; ++e) {
+    const int32_t kt = indices[e];
+    if (kt <= prev || kt >= g.nkt) {
+      atomicOr(err, DEVERR_BSR_ORDER);
+      return;
+    }
+    prev = kt;
+    int klass = 2;
+    if (causal) {
+      const int j0 = kt * kTile, j1 = min(g.k_len, j0 + kTile) - 1;
+      klass = (j0 > i1) ? 0 : (j1 <= i0 ? 2 : 1);
+    }
+    cls[g.cls_off + static_cast<int64_t>(qt) * g.nkt + kt] = static_cast<uint8_t>(klass);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// classes -> CSR lists + longest-first order (one CTA of 1024 threads)
+// ----------------------------------------------------------------------------
+// Dynamic shared memory: (max_nkt + 1) ints of bucket counters.
+__global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ groups,
+                                               const int32_t* __restrict__ row_group,
+                                               const uint8_t* __restrict__ cls, int n_rows, int max_nkt,
+                                               int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_ptr,
+                                               int32_t* __restrict__ kv_tile, int32_t* __restrict__ part,
+                                               int32_t* __restrict__ order) {
+  extern __shared__ int32_t bucket[];  // [max_nkt + 1]
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  // 1. count the listed tiles of every row (warp per row, ballot + popc)
+  for (int r = warp; r < n_rows; r += nw) {
+    const GroupInfo g = groups[row_group[r]];
+    const uint8_t* c = cls + g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
+    int n = 0;
+    for (int k0 = 0; k0 < g.nkt; k0 += 32) {
+      const int kt = k0 + lane;
+      n += __popc(__ballot_sync(0xffffffffu, kt < g.nkt && c[kt] != 0));
+    }
+    if (lane == 0) row_cnt[r] = n;
+  }
+  for (int i = tid; i <= max_nkt; i += blockDim.x) bucket[i] = 0;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+
+  // 2. exclusive scan of the counts -> row_ptr; bucket histogram of the counts
+  for (int base = 0; base < n_rows; base += blockDim.x) {
+    const int r = base + tid;
+    const int v = r < n_rows ? row_cnt[r] : 0;
+    if (r < n_rows) atomicAdd(&bucket[v], 1);
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int incl = x + (warp ? warp_sums[warp - 1] : 0) + carry;
+    if (r < n_rows) row_ptr[r] = incl - v;
+    __syncthreads();
+    if (tid == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  if (tid == 0) row_ptr[n_rows] = carry;
+  __syncthreads();
+
+  // 3. write each row's ascending list (warp per row)
+  for (int r = warp; r < n_rows; r += nw) {
+    const GroupInfo g = groups[row_group[r]];
+    const int64_t rowoff = g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
+    const uint8_t* c = cls + rowoff;
+    int out = row_ptr[r];
+    for (int k0 = 0; k0 < g.nkt; k0 += 32) {
+      const int kt = k0 + lane;
+      const int klass = kt < g.nkt ? c[kt] : 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, klass != 0);
+      if (klass != 0) {
+        const int pos = out + __popc(bal & lt_mask);
+        kv_tile[pos] = kt;
+        part[pos] = (klass == 1) ? static_cast<int32_t>(rowoff + kt) : -1;
+      }
+      out += __popc(bal);
+    }
+  }
+
+  // 4. longest-first stable order: counting sort over the counts.
+  //    bucket[k] <- first output slot of count k (descending counts)
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int k = max_nkt; k >= 0; --k) {
+      const int h = bucket[k];
+      bucket[k] = acc;
+      acc += h;
+    }
+  }
+  __syncthreads();
+  //    rows are placed chunk by chunk, warp by warp, so equal counts keep row order
+  for (int base = 0; base < n_rows; base += blockDim.x) {
+    const int r = base + tid;
+    const int key = r < n_rows ? row_cnt[r] : -1;
+    const uint32_t same = __match_any_sync(0xffffffffu, key);
+    const int rank = __popc(same & lt_mask);
+    const bool leader = rank == 0;
+    for (int w = 0; w < nw; ++w) {
+      if (warp == w && key >= 0) {
+        const int slot = bucket[key] + rank;
+        order[slot] = r;
+      }
+      __syncthreads();
+      if (warp == w && key >= 0 && leader) bucket[key] += __popc(same);
+      __syncthreads();
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// make_att_block_ids: inclusive running count of block openings (CTA per batch)
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_make_block_ids(const uint8_t* __restrict__ pad,
+                                                         const uint8_t* __restrict__ att, int N, int n_cross,
+                                                         const uint8_t* __restrict__ cross_pad,
+                                                         int32_t* __restrict__ q_blk, int32_t* __restrict__ k_blk,
+                                                         uint8_t* __restrict__ q_valid,
+                                                         uint8_t* __restrict__ k_valid) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t Nk = static_cast<int64_t>(n_cross) + N;
+  for (int j = tid; j < n_cross; j += blockDim.x) {
+    k_blk[b * Nk + j] = INT32_MIN;
+    k_valid[b * Nk + j] = cross_pad[static_cast<int64_t>(b) * n_cross + j] != 0;
+  }
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < N; base += blockDim.x) {
+    const int i = base + tid;
+    const int v = (i < N && att[static_cast<int64_t>(b) * N + i] != 0) ? 1 : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int incl = x + (warp ? warp_sums[warp - 1] : 0) + carry;
+    if (i < N) {
+      const int64_t qi = static_cast<int64_t>(b) * N + i;
+      const uint8_t pv = pad[qi] != 0;
+      q_blk[qi] = incl;
+      q_valid[qi] = pv;
+      k_blk[b * Nk + n_cross + i] = incl;
+      k_valid[b * Nk + n_cross + i] = pv;
+    }
+    __syncthreads();
+    if (tid == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// launchers (host)
+// ----------------------------------------------------------------------------
+cudaError_t launch_dense_classify(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* cls, uint32_t* fine,
+                                  cudaStream_t s) {
+  const int nqt = (Sq + kTile - 1) / kTile, nkt = (Sk + kTile - 1) / kTile;
+  const int vec_ok = ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (ld & 15) == 0) ? 1 : 0;
+  dim3 grid((nkt + kDenseTilesPerCta - 1) / kDenseTilesPerCta, nqt);
+  k_dense_classify<<<grid, 256, 0, s>>>(mask, ld, Sq, Sk, nkt, cls, fine, vec_ok);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_blockid_classify(const GroupInfo* groups, int n_groups, int max_tiles_q, int max_tiles_k,
+                                    const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
+                                    const uint8_t* k_valid, int batched, int Sq, int Sk, int window, int copy_ids,
+                                    int32_t* qid, uint8_t* qv, int32_t* kid, uint32_t* kbits, uint8_t* cls,
+                                    cudaStream_t s) {
+  const size_t smem = sizeof(TileStat) * static_cast<size_t>(max_tiles_q + max_tiles_k);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_blockid_classify, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k_blockid_classify<<<n_groups, 256, smem, s>>>(groups, q_blk, k_blk, q_valid, k_valid, batched, Sq, Sk,
+                                                 window, copy_ids, qid, qv, kid, kbits, cls);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, int64_t n_indices,
+                                const GroupInfo* groups, int n_groups, int nqt, int causal, uint8_t* cls,
+                                uint32_t* err, int32_t* max_width, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(n_groups) * nqt;
+  const int threads = 128;
+  k_bsr_classify<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(
+      indptr, indices, n_indices, groups, n_groups, nqt, causal, cls, err, max_width);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
+                        int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
+                        int32_t* order, cudaStream_t s) {
+  const size_t smem = sizeof(int32_t) * static_cast<size_t>(max_nkt + 1);
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
+                                  const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
+                                  uint8_t* k_valid, cudaStream_t s) {
+  k_make_block_ids<<<B, 1024, 0, s>>>(pad, att, N, n_cross, cross_pad, q_blk, k_blk, q_valid, k_valid);
+  return cudaGetLastError();
+}
+
+}  // namespace bfa

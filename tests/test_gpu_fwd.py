@@ -1,0 +1,254 @@
+"""GPU forward parity: outputs and LSE against the float64 oracle.
+
+Tolerance (bf16 N(0, 1) inputs, fp32 accumulation): output max-abs 1e-2, LSE
+max-abs 1e-3, and -inf LSE exactly where a row attends no key.  Small workloads
+are compared on every output; the full-size workloads on sampled rows of
+sampled heads, in the same call the bench times.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from helpers import check_bshd, compare_rows, sample_rows
+from oracle import attention as oa
+from oracle import masks as om
+
+pytestmark = pytest.mark.gpu
+
+bfa = pytest.importorskip("mask_skipping_flashattention_b200")
+
+
+def _cuda(x):
+    return torch.as_tensor(np.ascontiguousarray(x)).cuda()
+
+
+def _rand(shape, seed):
+    return workloads.randn_bf16(shape, seed)
+
+
+# ---------------------------------------------------------------- tiny / block-causal
+@pytest.mark.parametrize("form", ["dense", "blockids"])
+def test_tiny_blockcausal(form):
+    w = workloads.tiny_blockcausal()
+    ids_ref = om.make_att_block_ids(w["pad_masks"], w["att_masks"])
+    M = om.blockid_dense(*ids_ref)[0]
+    if form == "dense":
+        P = bfa.plan_dense(_cuda(M))
+    else:
+        P = bfa.plan_blockids(*bfa.make_att_block_ids(_cuda(w["pad_masks"]), _cuda(w["att_masks"])))
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), scale=w["scale"])
+    torch.cuda.synchronize()
+    P.device_status()
+    pairs = [(0, 0), (0, 1)]
+    check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: M, w["scale"], pairs, where=form)
+    # padded query rows attend nothing: output 0 and LSE -inf
+    assert torch.all(out[0, 240:] == 0) and torch.all(torch.isneginf(lse[0, :, 240:]))
+
+
+def test_blockcausal_gqa_cross_columns():
+    w = workloads.blockcausal_gqa()
+    ids = bfa.make_att_block_ids(_cuda(w["pad_masks"]), _cuda(w["att_masks"]), w["n_cross"],
+                                 _cuda(w["cross_pad_masks"]))
+    P = bfa.plan_blockids(*ids)
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+    torch.cuda.synchronize()
+    dense = om.blockid_dense(*om.make_att_block_ids(w["pad_masks"], w["att_masks"], w["n_cross"],
+                                                    w["cross_pad_masks"]))
+    pairs = [(b, h) for b in range(w["B"]) for h in range(w["H"])]
+    check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: dense[b], None, pairs, where="cfg3")
+
+
+# ---------------------------------------------------------------- causal 8192
+def test_causal_8192_reduced_heads_all_rows():
+    w = workloads.causal_8192(B=1, H=2)
+    P = bfa.plan_dense(w["mask"].cuda())
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+    torch.cuda.synchronize()
+    M = w["mask"].numpy()
+    check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: M, None, [(0, 0), (0, 1)],
+               where="causal full rows")
+
+
+def test_causal_8192_full_size_sampled():
+    """The bench workload (B=4, H=32, N=8192) in the bench's launch; sampled rows."""
+    w = workloads.causal_8192()
+    mask = w["mask"].cuda()
+    q, k, v = w["q"].cuda(), w["k"].cuda(), w["v"].cuda()
+    P = bfa.plan_dense(mask)
+    out, lse = bfa.fwd(P, q, k, v)
+    torch.cuda.synchronize()
+    P.device_status()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    rows = sample_rows(8192, 48, 7, must=(0, 1, 127, 128, 4095, 8191))
+    M = w["mask"].numpy()
+    pairs = [(0, 0), (1, 17), (2, 31), (3, 5)]
+    check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: M, None, pairs, rows=rows,
+               where="causal full size")
+
+
+# ---------------------------------------------------------------- varlen
+def _varlen_check(out, lse, w, window, heads, rows_per_seq=None):
+    cu = w["cu_seqlens"]
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        M = om.positional_dense(b - a, b - a, causal=True, window=window)
+        rows = None if rows_per_seq is None else sample_rows(b - a, rows_per_seq, s, must=(0, b - a - 1))
+        for h in heads:
+            g = h // (w["H"] // w["Hkv"])
+            qq = w["q"][a:b, h]
+            MM = M
+            if rows is not None:
+                qq, MM = qq[rows], M[rows]
+            O, L = oa.masked_attention(qq, w["k"][a:b, g], w["v"][a:b, g], MM)
+            og = out[a:b, h] if rows is None else out[a:b, h][rows]
+            lg = lse[h, a:b] if rows is None else lse[h, a:b][rows]
+            compare_rows(og, lg, O, L, where=f"varlen seq {s} head {h} window {window}")
+
+
+@pytest.mark.parametrize("window", [-1, 1024])
+def test_varlen_workload(window):
+    w = workloads.varlen_16()
+    cu = _cuda(w["cu_seqlens"])
+    P = bfa.plan_blockids(cu_seqlens_q=cu, cu_seqlens_k=cu, max_q=w["max_len"], max_k=w["max_len"],
+                          window_left=window)
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+    torch.cuda.synchronize()
+    _varlen_check(out.cpu(), lse.cpu(), w, window, heads=[0, 13, 31], rows_per_seq=96)
+
+
+def test_varlen_small_all_rows():
+    rng = np.random.default_rng(2)
+    lens = [1, 127, 128, 129, 300, 0, 5]
+    cu = np.zeros(len(lens) + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    T, H, Hkv, D = int(cu[-1]), 4, 2, 64
+    w = dict(cu_seqlens=cu, H=H, Hkv=Hkv, q=_rand((T, H, D), 11), k=_rand((T, Hkv, D), 12),
+             v=_rand((T, Hkv, D), 13))
+    for window in (-1, 3):
+        P = bfa.plan_blockids(cu_seqlens_q=_cuda(cu), cu_seqlens_k=_cuda(cu), max_q=300, max_k=300,
+                              window_left=window)
+        out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+        torch.cuda.synchronize()
+        _varlen_check(out.cpu(), lse.cpu(), w, window, heads=range(H))
+
+
+# ---------------------------------------------------------------- BSR and dense union
+def test_bsr_workload_sampled():
+    w = workloads.bsr_16384()
+    P = bfa.plan_bsr(_cuda(w["block_indptr"]), _cuda(w["block_indices"]), w["S"], w["S"], causal=True)
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+    torch.cuda.synchronize()
+    rows = sample_rows(w["S"], 40, 3, must=(0, 127, 128, 16383))
+    pairs = [(0, 0), (0, 9), (1, 31)]
+    out_c, lse_c = out.cpu(), lse.cpu()
+    for (b, h) in pairs:
+        g = h // 4
+        M = om.bsr_dense(w["block_indptr"][b:b + 1, g:g + 1], w["block_indices"], w["S"], w["S"], 128, 128,
+                         causal=True)[0, 0]
+        check_bshd(out_c, lse_c, w["q"], w["k"], w["v"], lambda bb, hh: M, None, [(b, h)], rows=rows,
+                   where="bsr")
+
+
+def test_union_workload_sampled():
+    w = workloads.union_16384()
+    P = bfa.plan_dense(w["mask"].cuda())
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+    torch.cuda.synchronize()
+    M = w["mask"].numpy()
+    rows = sample_rows(w["S"], 40, 4, must=(0, 63, 64, 2047, 16383))
+    check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: M, None, [(0, 0), (1, 30)],
+               rows=rows, where="union")
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Sq,Sk", [(1, 1), (77, 300), (300, 77), (256, 256), (129, 1000)])
+def test_dense_ragged_gqa(D, Sq, Sk):
+    rng = np.random.default_rng(Sq * 13 + Sk + D)
+    B, H, Hkv = 2, 4, 2
+    M = rng.random((Sq, Sk)) < 0.6
+    M[0] = False                      # a fully masked row
+    if Sq > 3:
+        M[3] = False
+        M[3, Sk - 1] = True           # a single attended key, at the edge
+    q, k, v = _rand((B, Sq, H, D), 1), _rand((B, Sk, Hkv, D), 2), _rand((B, Sk, Hkv, D), 3)
+    P = bfa.plan_dense(_cuda(M))
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda(), scale=0.3)
+    torch.cuda.synchronize()
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M, 0.3, pairs, where=f"ragged D={D}")
+    assert torch.all(out[:, 0] == 0) and torch.all(torch.isneginf(lse[:, :, 0]))
+
+
+def test_all_true_and_empty_masks():
+    B, H, S, D = 1, 2, 384, 128
+    q, k, v = _rand((B, S, H, D), 4), _rand((B, S, H, D), 5), _rand((B, S, H, D), 6)
+    for M in (np.ones((S, S), bool), np.zeros((S, S), bool)):
+        P = bfa.plan_dense(_cuda(M))
+        out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+        torch.cuda.synchronize()
+        check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M, None, [(0, 0), (0, 1)], where="all/none")
+    assert torch.all(out == 0)
+
+
+def test_bhsd_strides_and_out_buffer():
+    B, H, S, D = 2, 3, 200, 128
+    qh = _rand((B, H, S, D), 7).cuda()
+    kh = _rand((B, H, S, D), 8).cuda()
+    vh = _rand((B, H, S, D), 9).cuda()
+    q, k, v = (t.transpose(1, 2) for t in (qh, kh, vh))      # BSHD views of BHSD storage
+    M = om.positional_dense(S, S, causal=True)
+    P = bfa.plan_dense(_cuda(M))
+    big = torch.zeros((B, S, H, 2 * D), dtype=torch.bfloat16, device="cuda")
+    out = big[..., D:]
+    bfa.fwd(P, q, k, v, out=out, return_lse=False)
+    torch.cuda.synchronize()
+    assert torch.all(big[..., :D] == 0)
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    check_bshd(out.cpu(), None, q.cpu(), k.cpu(), v.cpu(), lambda b, h: M, None, pairs, where="bhsd")
+
+
+def test_default_scale_matches_explicit():
+    B, H, S, D = 1, 1, 256, 64
+    q, k, v = _rand((B, S, H, D), 21).cuda(), _rand((B, S, H, D), 22).cuda(), _rand((B, S, H, D), 23).cuda()
+    P = bfa.plan_dense(_cuda(om.positional_dense(S, S)))
+    o1, l1 = bfa.fwd(P, q, k, v)
+    o2, l2 = bfa.fwd(P, q, k, v, scale=1.0 / math.sqrt(D))
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_error_paths():
+    B, H, S, D = 1, 4, 128, 128
+    q, k, v = _rand((B, S, H, D), 1).cuda(), _rand((B, S, 3, D), 2).cuda(), _rand((B, S, 3, D), 3).cuda()
+    P = bfa.plan_dense(_cuda(np.ones((S, S), bool)))
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.fwd(P, q, k, v)                                   # H % Hkv != 0
+    assert e.value.status == "BFA_ERR_INVALID_ARG"
+    q96 = torch.zeros((B, S, H, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.fwd(P, q96, q96, q96)
+    assert e.value.status == "BFA_ERR_UNSUPPORTED"
+    qc = torch.zeros((B, S, H, D), dtype=torch.bfloat16)
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.fwd(P, qc, qc, qc, out=torch.zeros_like(qc.cuda()))
+    assert e.value.status == "BFA_ERR_NOT_DEVICE"
+    Pb = bfa.plan_blockids(B=2, Sq=S, Sk=S)
+    qq = torch.zeros((3, S, H, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.fwd(Pb, qq, qq, qq)                               # batch mismatch
+    assert e.value.status == "BFA_ERR_INVALID_ARG"
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    bfa.set_wait_timeout_ns(50_000_000)
+    try:
+        assert bfa.selftest_wait_timeout() == "BFA_ERR_TIMEOUT"
+    finally:
+        bfa.set_wait_timeout_ns(0)
+    # the context is still usable
+    test_default_scale_matches_explicit()

@@ -1,0 +1,222 @@
+"""GPU planner parity: every plan is compared bit for bit with the oracle's plan.
+
+The oracle plan of any mask form is the plan of its dense mask (built by the
+oracle's own builders); the GPU planners get the compact forms (dense bytes,
+block ids, positions, BSR routing) through the C ABI.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from helpers import assert_plan_equal, oracle_plan_for_groups
+from oracle import masks as om
+
+pytestmark = pytest.mark.gpu
+
+bfa = pytest.importorskip("mask_skipping_flashattention_b200")
+
+
+def _cuda(x, dtype=None):
+    t = torch.as_tensor(np.ascontiguousarray(x))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+# ---------------------------------------------------------------- dense plans
+@pytest.mark.parametrize("shape,density", [
+    ((1, 1), 1.0), ((1, 1), 0.0), ((5, 300), 0.5), ((128, 128), 0.999), ((129, 257), 0.3),
+    ((300, 200), 0.001), ((1000, 1300), 0.05), ((513, 129), 1.0), ((2048, 2048), 0.0),
+])
+def test_dense_plan_random(shape, density):
+    rng = np.random.default_rng(shape[0] * 7 + shape[1])
+    M = rng.random(shape) < density
+    if shape[0] >= 256 and shape[1] >= 256:
+        M[:128, :128] = True         # a full tile
+        M[128:256, 128:256] = False  # an empty tile
+    got = bfa.plan_dense(_cuda(M)).export()
+    assert_plan_equal(got, oracle_plan_for_groups([M]))
+
+
+def test_dense_plan_strided_and_uint8_mask():
+    rng = np.random.default_rng(3)
+    big = rng.random((300, 512)) < 0.2
+    t = _cuda(big)[:, :333]                    # row stride 512 bytes, 333 columns
+    got = bfa.plan_dense(t).export()
+    assert_plan_equal(got, oracle_plan_for_groups([big[:, :333]]))
+    t2 = _cuda(big.astype(np.uint8) * 7)[:, 1:300]   # nonzero bytes, unaligned base
+    got = bfa.plan_dense(t2).export()
+    assert_plan_equal(got, oracle_plan_for_groups([big[:, 1:300]]))
+
+
+def test_dense_plan_tiny_blockcausal():
+    w = workloads.tiny_blockcausal()
+    ids = om.make_att_block_ids(w["pad_masks"], w["att_masks"])
+    M = om.blockid_dense(*ids)[0]
+    assert_plan_equal(bfa.plan_dense(_cuda(M)).export(), oracle_plan_for_groups([M]))
+
+
+def test_dense_plan_causal_8192():
+    w = workloads.causal_8192(with_qkv=False)
+    P = bfa.plan_dense(w["mask"].cuda())
+    assert P.stats() == (2016, 64, 2016)
+    assert_plan_equal(P.export(), oracle_plan_for_groups([w["mask"].numpy()]))
+
+
+def test_dense_plan_union_16384():
+    w = workloads.union_16384(with_qkv=False)
+    M = w["mask"]
+    P = bfa.plan_dense(M.cuda())
+    assert_plan_equal(P.export(), oracle_plan_for_groups([M.numpy()]))
+
+
+# ---------------------------------------------------------------- block ids
+def test_make_block_ids_matches_oracle():
+    w = workloads.blockcausal_gqa()
+    ref = om.make_att_block_ids(w["pad_masks"], w["att_masks"], w["n_cross"], w["cross_pad_masks"])
+    got = bfa.make_att_block_ids(_cuda(w["pad_masks"]), _cuda(w["att_masks"]), w["n_cross"],
+                                 _cuda(w["cross_pad_masks"]))
+    for g, r in zip(got, ref):
+        np.testing.assert_array_equal(g.cpu().numpy().astype(np.int64), np.asarray(r).astype(np.int64))
+
+
+@pytest.mark.parametrize("name", ["tiny_blockcausal", "blockcausal_gqa"])
+def test_blockid_plan_matches_dense_oracle(name):
+    w = workloads.get(name)
+    nc = w.get("n_cross")
+    ref_ids = om.make_att_block_ids(w["pad_masks"], w["att_masks"], nc, w.get("cross_pad_masks"))
+    dense = om.blockid_dense(*ref_ids)
+    ids = bfa.make_att_block_ids(_cuda(w["pad_masks"]), _cuda(w["att_masks"]), nc,
+                                 _cuda(w["cross_pad_masks"]) if nc else None)
+    P = bfa.plan_blockids(*ids)
+    assert P.kind == "blockids"
+    ref = oracle_plan_for_groups(list(dense))
+    assert_plan_equal(P.export(), ref)
+    # the block-id planner's classes equal the dense planner's on the materialised mask
+    for b in range(dense.shape[0]):
+        Pd = bfa.plan_dense(_cuda(dense[b])).export()
+        nq, nk = ref["cls"][b].shape
+        np.testing.assert_array_equal(P.export()["classes"][b * nq * nk:(b + 1) * nq * nk], Pd["classes"])
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_blockid_plan_random_ragged(seed):
+    rng = np.random.default_rng(40 + seed)
+    B, Sq, Sk = 3, int(rng.integers(1, 700)), int(rng.integers(1, 900))
+    qb = np.sort(rng.integers(0, 6, size=(B, Sq)), axis=1).astype(np.int32)
+    kb = rng.integers(-3, 8, size=(B, Sk)).astype(np.int32)
+    kb[:, : min(5, Sk)] = np.iinfo(np.int32).min
+    qv = rng.random((B, Sq)) < (0.9 if seed % 2 else 1.0)
+    kv = rng.random((B, Sk)) < 0.8
+    P = bfa.plan_blockids(_cuda(qb), _cuda(kb), _cuda(qv), _cuda(kv))
+    dense = om.blockid_dense(qb, kb, qv, kv)
+    assert_plan_equal(P.export(), oracle_plan_for_groups(list(dense)))
+
+
+def test_positional_batched_plan():
+    P = bfa.plan_blockids(B=2, Sq=1000, Sk=1000)
+    assert P.kind == "positional"
+    M = om.positional_dense(1000, 1000, causal=True)
+    assert_plan_equal(P.export(), oracle_plan_for_groups([M, M]))
+
+
+def test_positional_with_validity_uses_predicate_plan():
+    rng = np.random.default_rng(5)
+    qv = rng.random((2, 300)) < 0.9
+    P = bfa.plan_blockids(q_valid=_cuda(qv), k_valid=_cuda(np.ones((2, 300), bool)), B=2, Sq=300, Sk=300)
+    assert P.kind == "blockids"
+    masks = [om.positional_dense(300, 300) & qv[b][:, None] for b in range(2)]
+    assert_plan_equal(P.export(), oracle_plan_for_groups(masks))
+
+
+# ---------------------------------------------------------------- varlen
+def _varlen_oracle(cu_q, cu_k, window):
+    masks = []
+    for s in range(len(cu_q) - 1):
+        lq, lk = int(cu_q[s + 1] - cu_q[s]), int(cu_k[s + 1] - cu_k[s])
+        masks.append(om.positional_dense(lq, lk, causal=True, window=window))
+    return masks
+
+
+@pytest.mark.parametrize("window", [-1, 1024])
+def test_varlen_plan_workload(window):
+    w = workloads.varlen_16()
+    cu = _cuda(w["cu_seqlens"])
+    P = bfa.plan_blockids(cu_seqlens_q=cu, cu_seqlens_k=cu, max_q=w["max_len"], max_k=w["max_len"],
+                          window_left=window)
+    assert P.info["varlen"] == 1 and P.info["n_groups"] == 16
+    assert_plan_equal(P.export(), oracle_plan_for_groups(_varlen_oracle(w["cu_seqlens"], w["cu_seqlens"], window)))
+
+
+@pytest.mark.parametrize("window", [-1, 1, 7, 200])
+def test_varlen_plan_ragged_unequal(window):
+    cq = np.array([0, 3, 3, 260, 900, 901], dtype=np.int32)     # includes an empty sequence
+    ck = np.array([0, 130, 131, 131, 700, 1000], dtype=np.int32)
+    P = bfa.plan_blockids(cu_seqlens_q=_cuda(cq), cu_seqlens_k=_cuda(ck), max_q=640, max_k=600,
+                          window_left=window)
+    assert_plan_equal(P.export(), oracle_plan_for_groups(_varlen_oracle(cq, ck, window)))
+
+
+def test_varlen_understated_max_is_an_error():
+    cu = _cuda(np.array([0, 100, 300], dtype=np.int32))
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.plan_blockids(cu_seqlens_q=cu, cu_seqlens_k=cu, max_q=150, max_k=300)
+    assert e.value.status == "BFA_ERR_INVALID_ARG"
+
+
+# ---------------------------------------------------------------- BSR
+def _bsr_oracle(indptr, indices, S, causal):
+    D = om.bsr_dense(indptr, indices, S, S, 128, 128, causal=causal)
+    return [D[b, h] for b in range(D.shape[0]) for h in range(D.shape[1])]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bsr_plan_small(causal):
+    indptr, indices = workloads.bsr_routing(2, 3, 9, 77)
+    S = 9 * 128 - 50                       # ragged last block
+    P = bfa.plan_bsr(_cuda(indptr), _cuda(indices), S, S, causal=causal)
+    assert_plan_equal(P.export(), oracle_plan_for_groups(_bsr_oracle(indptr, indices, S, causal)))
+
+
+def test_bsr_plan_workload_one_head_group_full_size():
+    w = workloads.bsr_16384(with_qkv=False)
+    P = bfa.plan_bsr(_cuda(w["block_indptr"]), _cuda(w["block_indices"]), w["S"], w["S"], causal=True)
+    n_full, n_part, n_empty = P.stats()
+    assert n_part == 2 * 8 * 128 and n_full == 2 * 8 * 1984
+    got = P.export()
+    # full bit-exact check on the first two (b, hkv) groups; lists of all groups by counts
+    ip, ix = w["block_indptr"][:1, :2], w["block_indices"]
+    ref = oracle_plan_for_groups(_bsr_oracle(ip, ix, w["S"], True))
+    R = 2 * 128
+    np.testing.assert_array_equal(got["row_ptr"][:R + 1], ref["row_ptr"])
+    np.testing.assert_array_equal(got["kv_tile"][:ref["kv_tile"].size], ref["kv_tile"])
+    np.testing.assert_array_equal(got["partial"][:ref["partial"].size], ref["partial"])
+    counts = np.diff(got["row_ptr"])
+    exp = np.array([i // 4 + 1 for _ in range(16) for i in range(128)])
+    np.testing.assert_array_equal(counts, exp)
+    order = got["order"]
+    assert np.all(np.diff(counts[order]) <= 0)
+    ties = np.diff(counts[order]) == 0
+    assert np.all(np.diff(order)[ties] > 0)
+
+
+def test_bsr_noncanonical_rejected():
+    indptr = np.array([[[0, 2, 3]]], dtype=np.int32)
+    for bad in ([1, 0, 1], [1, 1, 1], [0, 1, 2]):
+        with pytest.raises(bfa.BfaError) as e:
+            bfa.plan_bsr(_cuda(indptr), _cuda(np.array(bad, np.int32)), 256, 256)
+        assert e.value.status == "BFA_ERR_NONCANONICAL_BSR"
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.plan_bsr(_cuda(np.array([[[0, 3, 2]]], np.int32)), _cuda(np.array([0, 1, 1], np.int32)), 256, 256)
+    assert e.value.status == "BFA_ERR_NONCANONICAL_BSR"
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.plan_bsr(_cuda(indptr), _cuda(np.array([0, 1, 1], np.int32)), 256, 256, q_block_size=64)
+    assert e.value.status == "BFA_ERR_UNSUPPORTED"
+
+
+def test_plan_rejects_host_memory():
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.plan_dense(torch.ones(8, 8, dtype=torch.bool))
+    assert e.value.status == "BFA_ERR_NOT_DEVICE"
