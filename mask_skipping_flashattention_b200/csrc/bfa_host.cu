@@ -36,6 +36,8 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
 cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
                                   const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
                                   uint8_t* k_valid, cudaStream_t s);
+cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
+                                       GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s);
 
 
 }  // namespace bfa
@@ -49,6 +51,9 @@ struct bfa_plan {
   int kind = 0, varlen = 0, batch = 0, hkv = 0, sq = 0, sk = 0, window = -1, causal = 0;
   int n_groups = 0, n_rows = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
   int64_t grid_tiles = 0;
+  bool regular = false;   // every group the same shape: the group table is built on the device
+  int regular_hkv = 1;    // groups per batch of a regular layout (BSR: Hkv)
+  bool copy_ids = false;
   std::vector<GroupInfo> groups_h;
   cudaStream_t stream = nullptr;
   void* slab = nullptr;
@@ -115,6 +120,33 @@ bfa_status need_device(const void* p, const char* name, bool allow_null = false)
   return BFA_OK;
 }
 
+// Stream-ordered pool for plan memory, one per device.  Its release threshold
+// is unbounded, so building and freeing plans in a loop reuses the same memory
+// instead of returning it to the driver at every synchronisation.
+cudaError_t plan_pool(cudaMemPool_t* out) {
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!pools[dev]) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t thr = UINT64_MAX;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+    if (e != cudaSuccess) return e;
+    pools[dev] = pool;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
+}
+
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -147,7 +179,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   const size_t o_kid = L.take<int32_t>(std::max<int64_t>(kid_elems, 1));
   const size_t o_kb = L.take<uint32_t>(std::max<int64_t>(kbit_words, 1));
   const size_t o_fine = L.take<uint32_t>(with_fine ? static_cast<size_t>(cap_tiles) * kFineWordsPerTile : 1);
-  cudaError_t e = cudaMallocAsync(&P->slab, L.off, P->stream);
+  cudaMemPool_t pool;
+  cudaError_t e = plan_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "plan memory pool");
+  e = cudaMallocFromPoolAsync(&P->slab, L.off, pool, P->stream);
   if (e != cudaSuccess) return fail(BFA_ERR_CAPACITY, "plan allocation of %zu bytes failed: %s", L.off,
                                     cudaGetErrorString(e));
   uint8_t* base = static_cast<uint8_t*>(P->slab);
@@ -167,16 +202,24 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->kbits = reinterpret_cast<uint32_t*>(base + o_kb);
   P->fine = reinterpret_cast<uint32_t*>(base + o_fine);
 
-  std::vector<int32_t> rg(std::max(P->n_rows, 1), 0);
-  for (int g = 0; g < P->n_groups; ++g)
-    for (int r = 0; r < P->groups_h[g].nqt; ++r) rg[P->groups_h[g].row0 + r] = g;
-  if (P->n_groups > 0) {
-    e = cudaMemcpyAsync(P->groups, P->groups_h.data(), sizeof(GroupInfo) * P->n_groups, cudaMemcpyHostToDevice,
-                        P->stream);
-    if (e != cudaSuccess) return cuda_fail(e, "upload plan groups");
+  if (P->regular) {
+    e = launch_init_regular_groups(P->groups_h[0], P->n_groups, P->regular_hkv, P->kind == BFA_PLAN_BSR ? 1 : 0,
+                                   P->copy_ids ? 1 : 0, P->groups, P->row_group, P->n_rows, P->stream);
+    if (e != cudaSuccess) return cuda_fail(e, "plan group table kernel");
+  } else {
+    // irregular (varlen) layouts: the planner has synchronised already to read
+    // the sequence lengths, so a pageable upload costs nothing extra here
+    std::vector<int32_t> rg(std::max(P->n_rows, 1), 0);
+    for (int g = 0; g < P->n_groups; ++g)
+      for (int r = 0; r < P->groups_h[g].nqt; ++r) rg[P->groups_h[g].row0 + r] = g;
+    if (P->n_groups > 0) {
+      e = cudaMemcpyAsync(P->groups, P->groups_h.data(), sizeof(GroupInfo) * P->n_groups, cudaMemcpyHostToDevice,
+                          P->stream);
+      if (e != cudaSuccess) return cuda_fail(e, "upload plan groups");
+    }
+    e = cudaMemcpyAsync(P->row_group, rg.data(), sizeof(int32_t) * rg.size(), cudaMemcpyHostToDevice, P->stream);
+    if (e != cudaSuccess) return cuda_fail(e, "upload plan rows");
   }
-  e = cudaMemcpyAsync(P->row_group, rg.data(), sizeof(int32_t) * rg.size(), cudaMemcpyHostToDevice, P->stream);
-  if (e != cudaSuccess) return cuda_fail(e, "upload plan rows");
   e = cudaMemsetAsync(P->err, 0, 2 * 256, P->stream);  // err and max_width slots
   if (e != cudaSuccess) return cuda_fail(e, "clear plan status");
   return BFA_OK;
@@ -305,6 +348,7 @@ BFA_API bfa_status bfa_plan_dense(const uint8_t* mask, int64_t ld, int Sq, int S
   P->sk = Sk;
   P->mask_mode = MASK_BITS;
   P->groups_h.push_back(make_group(0, Sq, 0, Sk, -1, -1));
+  P->regular = true;
   finalize_layout(P);
   if ((s = check_capacity(P, true))) { cleanup(); return s; }
   if ((s = alloc_plan(P, true, 0, 0, 0))) { cleanup(); return s; }
@@ -370,10 +414,12 @@ BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk,
     P->sq = Sq;
     P->sk = Sk;
   }
+  P->regular = !varlen;
+  P->copy_ids = P->mask_mode == MASK_BLOCKID;
   finalize_layout(P);
   // padded per-group id copies (block-id mode only)
   int64_t qe = 0, ke = 0, kw = 0;
-  const bool copy_ids = P->mask_mode == MASK_BLOCKID;
+  const bool copy_ids = P->copy_ids;
   for (auto& g : P->groups_h) {
     g.qid_off = static_cast<int32_t>(qe);
     g.kid_off = static_cast<int32_t>(ke);
@@ -426,6 +472,8 @@ BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, i
   P->stream = st;
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < Hkv; ++h) P->groups_h.push_back(make_group(0, Sq, 0, Skv, b, h));
+  P->regular = true;
+  P->regular_hkv = Hkv;
   finalize_layout(P);
   if ((s = check_capacity(P, false))) { cleanup(); return s; }
   if ((s = alloc_plan(P, false, 0, 0, 0))) { cleanup(); return s; }

@@ -7,15 +7,16 @@
 // longest-first row order, so the hardware's in-order CTA dispatch balances SMs
 // by the number of non-empty tiles.
 //
-// Warp roles (192 threads):
+// Warp roles (256 threads, two CTAs per SM):
 //   warp 0      TMA producer: Q once, then K_u / V_u of every listed tile u
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer:
 //                 S_u = Q K_u^T   (SS: both operands in shared memory, K-major)
 //                 O  += P_u V_u   (TS: P_u read from TMEM, V_u MN-major in smem)
-//   warps 2..5  softmax: one query row per thread; S_u from TMEM, mask on partial
-//               and edge tiles, online base-2 softmax in fp32, P_u written back to
-//               TMEM over S_u as packed bf16, lazy rescale of O in TMEM; epilogue
-//               O / l -> bf16 and LSE.
+//   warps 2..3  idle (they give their registers to the softmax warpgroup)
+//   warps 4..7  softmax: one query row per thread, the whole S row in registers;
+//               mask on partial and edge tiles only, online base-2 softmax in
+//               fp32, P_u written back to TMEM over S_u as packed bf16, lazy
+//               rescale of O in TMEM; epilogue O / l -> bf16 and LSE.
 //
 // TMEM (256 columns): S / P at columns [0, 128), O at [128, 128 + D).
 // Shared memory: Q, K, V tiles (128 x D bf16 each) in 64-column panels with the
@@ -35,7 +36,16 @@ using namespace ptx;
 
 
 
-constexpr int kThreads = 192;
+// 256 threads: warpgroup 0 = warp 0 TMA producer, warp 1 MMA issuer (warps 2-3
+// idle), warpgroup 1 = softmax.  Two CTAs per SM: 128 registers per thread at
+// launch, redistributed so the softmax holds a whole S row in registers.  The
+// split must add up to the launch allocation: 128 * kRegsWG0 + 128 * kRegsWG1 ==
+// 256 * kRegsLaunch (checked against the compiled kernel before launching).
+constexpr int kThreads = 256;
+constexpr int kRegsLaunch = 128;
+constexpr uint32_t kRegsWG0 = 56;
+constexpr uint32_t kRegsWG1 = 200;
+static_assert(128 * kRegsWG0 + 128 * kRegsWG1 == kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
 
 template <int D>
@@ -195,74 +205,79 @@ __global__ void __launch_bounds__(kThreads, 2)
   const Work wk = wk_s;
   const uint64_t cap = p.wait_ns;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && wk.n > 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const int qs = wk.q_off + wk.qt * kTile;
-      mbar_expect_tx(bar(BQ), C::kTileBytes);
-#pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_4d(smem_u32(sQ + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h, qs, wk.b);
-      int last_k = -1, last_v = -1;  // last issued phase of each full barrier
-      for (int u = 0; u < wk.n; ++u) {
-        const int kt = p.plan.kv_tile[wk.e0 + u];
-        const int ks = wk.k_off + kt * kTile;
-        if (u > 0 && !mbar_wait(bar(BKE), (u - 1) & 1, cap, &abort_flag)) break;
-        mbar_expect_tx(bar(BKF), C::kTileBytes);
+  if (warp < 4) {
+    // ============================================================ warpgroup 0
+    regs_dec<kRegsWG0>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0 && wk.n > 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        const int qs = wk.q_off + wk.qt * kTile;
+        mbar_expect_tx(bar(BQ), C::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_4d(smem_u32(sK + pn * 16384), &tmK, bar(BKF), pn * 64, wk.hk, ks, wk.b);
-        last_k = u;
-        if (u > 0 && !mbar_wait(bar(BVE), (u - 1) & 1, cap, &abort_flag)) break;
-        mbar_expect_tx(bar(BVF), C::kTileBytes);
+          tma_load_4d(smem_u32(sQ + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h, qs, wk.b);
+        int last_k = -1, last_v = -1;  // last issued phase of each full barrier
+        for (int u = 0; u < wk.n; ++u) {
+          const int kt = p.plan.kv_tile[wk.e0 + u];
+          const int ks = wk.k_off + kt * kTile;
+          if (u > 0 && !mbar_wait(bar(BKE), (u - 1) & 1, cap, &abort_flag)) break;
+          mbar_expect_tx(bar(BKF), C::kTileBytes);
 #pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_4d(smem_u32(sV + pn * 16384), &tmV, bar(BVF), pn * 64, wk.hk, ks, wk.b);
-        last_v = u;
-      }
-      // before the CTA can exit, every copy it issued must have landed (bounded;
-      // on the normal path these phases completed long ago)
-      volatile int no_abort = 0;
-      mbar_wait(bar(BQ), 0, cap, &no_abort);
-      if (last_k >= 0) mbar_wait(bar(BKF), last_k & 1, cap, &no_abort);
-      if (last_v >= 0) mbar_wait(bar(BVF), last_v & 1, cap, &no_abort);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && wk.n > 0) {
-      const uint32_t tS = tmem + C::kColS, tO = tmem + C::kColO;
-      bool ok = mbar_wait(bar(BQ), 0, cap, &abort_flag);
-      for (int u = 0; ok && u < wk.n; ++u) {
-        if (!mbar_wait(bar(BKF), u & 1, cap, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_4d(smem_u32(sK + pn * 16384), &tmK, bar(BKF), pn * 64, wk.hk, ks, wk.b);
+          last_k = u;
+          if (u > 0 && !mbar_wait(bar(BVE), (u - 1) & 1, cap, &abort_flag)) break;
+          mbar_expect_tx(bar(BVF), C::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tS, smem_desc(smem_u32(sQ + off), 16, 1024), smem_desc(smem_u32(sK + off), 16, 1024),
-                  C::kIdescQK, kk > 0);
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_4d(smem_u32(sV + pn * 16384), &tmV, bar(BVF), pn * 64, wk.hk, ks, wk.b);
+          last_v = u;
         }
-        umma_commit(bar(BS));
-        umma_commit(bar(BKE));
-        if (!mbar_wait(bar(BP), u & 1, cap, &abort_flag)) { ok = false; break; }
-        if (!mbar_wait(bar(BVF), u & 1, cap, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tO, tS + kk * 8, smem_desc(smem_u32(sV + kk * 2048), 16384, 1024), C::kIdescPV,
-                  (u > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(BVE));
+        // every copy this CTA issued must land before it can exit (bounded; on the
+        // normal path these phases completed long ago)
+        volatile int no_abort = 0;
+        mbar_wait(bar(BQ), 0, cap, &no_abort);
+        if (last_k >= 0) mbar_wait(bar(BKF), last_k & 1, cap, &no_abort);
+        if (last_v >= 0) mbar_wait(bar(BVF), last_v & 1, cap, &no_abort);
       }
-      if (ok) umma_commit(bar(BO));
-      // every MMA issued must be finished before TMEM is released (bounded)
-      umma_commit(bar(BDONE));
-      volatile int no_abort = 0;
-      mbar_wait(bar(BDONE), 0, cap, &no_abort);
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0 && wk.n > 0) {
+        const uint32_t tS = tmem + C::kColS, tO = tmem + C::kColO;
+        bool ok = mbar_wait(bar(BQ), 0, cap, &abort_flag);
+        for (int u = 0; ok && u < wk.n; ++u) {
+          if (!mbar_wait(bar(BKF), u & 1, cap, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_ss(tS, smem_desc(smem_u32(sQ + off), 16, 1024), smem_desc(smem_u32(sK + off), 16, 1024),
+                    C::kIdescQK, kk > 0);
+          }
+          umma_commit(bar(BS));
+          umma_commit(bar(BKE));
+          if (!mbar_wait(bar(BP), u & 1, cap, &abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar(BVF), u & 1, cap, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tO, tS + kk * 8, smem_desc(smem_u32(sV + kk * 2048), 16384, 1024), C::kIdescPV,
+                    (u > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(BVE));
+        }
+        if (ok) umma_commit(bar(BO));
+        // every MMA issued must be finished before TMEM is released (bounded)
+        umma_commit(bar(BDONE));
+        volatile int no_abort = 0;
+        mbar_wait(bar(BDONE), 0, cap, &no_abort);
+      }
     }
   } else {
-    // ------------------------------------------------------------ softmax
+    // ============================================================ warpgroup 1: softmax
+    regs_inc<kRegsWG1>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tS = tmem_addr(tmem + C::kColS, quarter * 32, 0);
@@ -270,31 +285,43 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    int kt_next = wk.n > 0 ? p.plan.kv_tile[wk.e0] : 0;
+    int part_next = wk.n > 0 ? p.plan.part[wk.e0] : -1;
     for (int u = 0; u < wk.n; ++u) {
-      const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
-      if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit
-      tc_fence_after();
-      const int e = wk.e0 + u;
-      const int kt = p.plan.kv_tile[e];
-      const int part = p.plan.part[e];
+      const int kt = kt_next, part = part_next;
+      if (u + 1 < wk.n) {  // next list entry, off the critical path
+        kt_next = p.plan.kv_tile[wk.e0 + u + 1];
+        part_next = p.plan.part[wk.e0 + u + 1];
+      }
       const bool masked = part >= 0 || (kt + 1) * kTile > wk.k_len;
       uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (masked) row_mask_words(p, wk, row, kt, part, am);
-      // pass 1: row max of the masked scores, 32 columns at a time
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tS + cc * 32, r);
-        tmem_wait_ld();
-        reg_fence(r);
-        const uint32_t w = cc == 0 ? am[0] : cc == 1 ? am[1] : cc == 2 ? am[2] : am[3];
+
+      const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
+      if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit
+      tc_fence_after();
+      // the whole S row in registers: four loads in flight, one wait
+      uint32_t sr[128];
+      tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      reg_fence(sr);
+      float* s = reinterpret_cast<float*>(sr);
+      if (masked) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float x = ((w >> j) & 1u) ? __uint_as_float(r[j]) : -INFINITY;
-          mx = fmaxf(mx, x);
-        }
+        for (int j = 0; j < 128; ++j)
+          if (!((am[j >> 5] >> (j & 31)) & 1u)) s[j] = -INFINITY;
       }
+      // row max, 8 independent chains
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int j = 8; j < 128; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mnew = fmaxf(m, mx * c);
       // The reference max m only moves when some row of the warp grew by more
       // than 2^8; then every row of the warp moves to its true running max (alpha
@@ -318,34 +345,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         m = mnew;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
-      // pass 2: p = 2^(s*c - m), packed to bf16 pairs over the first 64 columns of S
-      float rs = 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tS + cc * 32, r);
-        tmem_wait_ld();
-        reg_fence(r);
-        const uint32_t w = cc == 0 ? am[0] : cc == 1 ? am[1] : cc == 2 ? am[2] : am[3];
-        uint32_t pk[16];
+      // p = 2^(s*c - m), 4 independent row-sum chains; packed bf16 pairs go to
+      // the first 64 columns of S (the A operand of the P V product)
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[64];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float s0 = ((w >> (2 * j)) & 1u) ? __uint_as_float(r[2 * j]) : -INFINITY;
-          const float s1 = ((w >> (2 * j + 1)) & 1u) ? __uint_as_float(r[2 * j + 1]) : -INFINITY;
-          const float p0 = ex2_approx(fmaf(s0, c, -mref));
-          const float p1 = ex2_approx(fmaf(s1, c, -mref));
-          rs += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
-        }
-        tmem_st_32x32b_x16(tS + cc * 16, pk);
+      for (int j = 0; j < 64; ++j) {
+        const float p0 = ex2_approx(fmaf(s[2 * j], c, -mref));
+        const float p1 = ex2_approx(fmaf(s[2 * j + 1], c, -mref));
+        rs[j & 3] += p0 + p1;
+        pk[j] = pack_bf16x2(p0, p1);
       }
-      l += rs;
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BP));
     }
-    // ------------------------------------------------------------ epilogue
+    // ---------------------------------------------------------- epilogue
     if (ok && wk.n > 0) {
       const bool got = mbar_wait(bar(BO), 0, cap, &abort_flag);
       ok = !__any_sync(0xffffffffu, !got);
@@ -417,6 +436,16 @@ __global__ void k_wait_selftest(uint32_t* err, uint64_t cap) {
 // ----------------------------------------------------------------------------
 int fwd_smem_bytes(int D) { return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes; }
 
+// The setmaxnreg split is only safe if every thread is launched with exactly
+// kRegsLaunch registers; refuse to launch otherwise.
+template <typename K>
+static cudaError_t check_regs(K kernel) {
+  cudaFuncAttributes a;
+  cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+  if (e != cudaSuccess) return e;
+  return a.numRegs == kRegsLaunch ? cudaSuccess : cudaErrorInvalidKernelImage;
+}
+
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int64_t n_work, cudaStream_t s) {
   if (n_work <= 0) return cudaSuccess;
@@ -424,8 +453,9 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
   if (D == 64) {
     static bool set = false;
     if (!set) {
-      cudaError_t e = cudaFuncSetAttribute(bfa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           Cfg<64>::kSmemBytes);
+      cudaError_t e = check_regs(bfa_fwd_kernel<64>);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(bfa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<64>::kSmemBytes);
       if (e != cudaSuccess) return e;
       set = true;
     }
@@ -433,8 +463,10 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
   } else {
     static bool set = false;
     if (!set) {
-      cudaError_t e = cudaFuncSetAttribute(bfa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           Cfg<128>::kSmemBytes);
+      cudaError_t e = check_regs(bfa_fwd_kernel<128>);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(bfa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg<128>::kSmemBytes);
       if (e != cudaSuccess) return e;
       set = true;
     }

@@ -382,8 +382,39 @@ __global__ void __launch_bounds__(1024) k_make_block_ids(const uint8_t* __restri
 }
 
 // ----------------------------------------------------------------------------
+// group table of a regular layout (every group the same shape): group g is
+// batch g / n_hkv and, for BSR plans, kv head g % n_hkv
+// ----------------------------------------------------------------------------
+__global__ void k_init_regular_groups(GroupInfo tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
+                                      GroupInfo* __restrict__ groups, int32_t* __restrict__ row_group,
+                                      int n_rows) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n_groups) {
+    GroupInfo g = tmpl;
+    g.b = (tmpl.b < 0) ? -1 : i / n_hkv;
+    g.hkv = bsr ? i % n_hkv : -1;
+    g.row0 = i * tmpl.nqt;
+    g.cls_off = static_cast<int64_t>(i) * tmpl.nqt * tmpl.nkt;
+    g.qid_off = copy_ids ? i * tmpl.nqt * kTile : 0;
+    g.kid_off = copy_ids ? i * tmpl.nkt * kTile : 0;
+    g.kbit_off = copy_ids ? i * tmpl.nkt * kWordsPerTileRow : 0;
+    groups[i] = g;
+  }
+  if (i < n_rows) row_group[i] = tmpl.nqt > 0 ? i / tmpl.nqt : 0;
+}
+
+// ----------------------------------------------------------------------------
 // launchers (host)
 // ----------------------------------------------------------------------------
+cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
+                                       GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s) {
+  const int n = n_groups > n_rows ? n_groups : n_rows;
+  if (n <= 0) return cudaSuccess;
+  k_init_regular_groups<<<(n + 255) / 256, 256, 0, s>>>(tmpl, n_groups, n_hkv, bsr, copy_ids, groups, row_group,
+                                                       n_rows);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dense_classify(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* cls, uint32_t* fine,
                                   cudaStream_t s) {
   const int nqt = (Sq + kTile - 1) / kTile, nkt = (Sk + kTile - 1) / kTile;

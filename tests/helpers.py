@@ -62,6 +62,17 @@ def check_bshd(out, lse, q, k, v, mask_for, scale, pairs, rows=None, where=""):
     return worst
 
 
+# Worst-case error of the bf16 path, used where the softmax is far peakier than
+# the default scale makes it: P is rounded to bf16 before P V (relative error at
+# most u = 2^-8 per weight, so at most u * max|v| on a weighted mean of v) and the
+# output is rounded to bf16 (at most u * |O|); fp32 accumulation adds ~1e-5.
+BF16_U = 2.0 ** -8
+
+
+def peaked_bound(O_ref, vmax):
+    return BF16_U * (np.abs(O_ref) + vmax) + 1e-4
+
+
 def sample_rows(n, k, seed, must=()):
     rng = np.random.default_rng(seed)
     r = set(int(x) for x in rng.choice(n, size=min(k, n), replace=False))
