@@ -74,7 +74,7 @@ def load():
         return _lib
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libbfa.so not found at {LIB_PATH}; build it with "
-                          "`python -m mask_skipping_flashattention_b200.build` (nvcc, sm_100a)")
+                          "`python mask_skipping_flashattention_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

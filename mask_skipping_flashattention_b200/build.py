@@ -1,6 +1,7 @@
 """Build ``libbfa.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m mask_skipping_flashattention_b200.build [--force] [--verbose]``.
+Usage: ``python mask_skipping_flashattention_b200/build.py [--force] [--verbose]`` (run by path:
+importing the package would load the library being rebuilt).
 Objects go to ``_build/`` at the repository root; the shared library is written
 next to this file so that it travels with the source tree.
 """
