@@ -221,6 +221,35 @@ void bfa_set_wait_timeout_ns(uint64_t ns);
  * stays usable), BFA_OK never.  Exercises the failure path without a fault. */
 bfa_status bfa_selftest_wait_timeout(void* stream);
 
+/*
+ * Dense-mask planner that allocates nothing.  The source pages have no
+ * counterpart: this entry point exists for callers that cannot let a library
+ * allocate device memory -- for example a serving process whose memory manager
+ * reserves the whole GPU up front, or code that must keep a fixed device-memory
+ * footprint.  It computes the same plan as bfa_plan_dense, but as plain arrays
+ * in buffers the caller owns, and calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   Inputs: mask / mask_row_stride / Sq / Sk as for bfa_plan_dense.
+ *   Outputs (device, caller-owned; nqt = ceil(Sq/128), nkt = ceil(Sk/128)):
+ *     classes [nqt * nkt] u8 (0 empty, 1 partial, 2 full), row_ptr [nqt + 1],
+ *     kv_tile [nqt * nkt] i32 and part [nqt * nkt] i32 (-1 full, else the tile's
+ *     index in classes), used up to row_ptr[nqt]; fine [nqt * nkt * 512] u32,
+ *     written at the class-grid index of every partial tile; order [nqt].
+ *   Limits: nqt <= BFA_NOALLOC_MAX_ROWS and nkt <= BFA_NOALLOC_MAX_KV_TILES, else
+ *     BFA_ERR_CAPACITY before anything is launched.
+ * Its scratch (group table, row map, per-row counts: 256 + 8 * BFA_NOALLOC_MAX_ROWS
+ * bytes) is a device array inside the library that every GPU loading the library
+ * holds until exit.  The first call on a device looks up that array's address,
+ * so make that first call before any stream capture.  All calls share the one
+ * array: calls that overlap on the GPU (on different streams) race and must be
+ * ordered by the caller.  Each call writes every scratch word it reads, so the
+ * previous call's contents do not matter.  Stream-ordered, no synchronisation.
+ */
+enum { BFA_NOALLOC_MAX_ROWS = 4096, BFA_NOALLOC_MAX_KV_TILES = 16384 };
+bfa_status bfa_plan_dense_noalloc(const uint8_t* mask, int64_t mask_row_stride, int Sq, int Sk,
+                                  uint8_t* classes, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
+                                  uint32_t* fine, int32_t* order, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

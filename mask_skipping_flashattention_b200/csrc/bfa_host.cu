@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -763,3 +764,78 @@ BFA_API bfa_status bfa_selftest_wait_timeout(void* stream) {
   return BFA_OK;
 }
 
+
+// ----------------------------------------------------------------------------
+// Dense planner that allocates nothing
+// ----------------------------------------------------------------------------
+// For callers that cannot let the library allocate device memory, for example a
+// serving process whose memory manager has reserved the whole GPU up front, or
+// code that must keep a fixed, known device-memory footprint.  The caller passes
+// the mask and every output buffer; the planner's own scratch (the group table,
+// the row -> group map and the per-row tile counts) lives in the file-scope
+// device array below, which every GPU that loads the library holds until the
+// process exits.
+namespace {
+
+constexpr int kNoAllocMaxRows = BFA_NOALLOC_MAX_ROWS;
+constexpr size_t kNoAllocScratchBytes = 256 + 2 * sizeof(int32_t) * kNoAllocMaxRows;
+static_assert(sizeof(GroupInfo) <= 256, "group table slot");
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+uint8_t* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device (set up once per
+// device, with that device current).  In host code the array's name is only a
+// host-side stand-in, so the address must come from cudaGetSymbolAddress.
+bfa_status noalloc_scratch(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "current device");
+  if (dev < 0 || dev >= 64) return fail(BFA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "scratch symbol address");
+    g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return BFA_OK;
+}
+
+}  // namespace
+
+BFA_API bfa_status bfa_plan_dense_noalloc(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* classes,
+                                          int32_t* row_ptr, int32_t* kv_tile, int32_t* part, uint32_t* fine,
+                                          int32_t* order, void* stream) {
+  if (Sq <= 0 || Sk <= 0) return fail(BFA_ERR_INVALID_ARG, "Sq=%d Sk=%d must be positive", Sq, Sk);
+  if (ld < Sk) return fail(BFA_ERR_INVALID_ARG, "mask_row_stride %lld < Sk %d", (long long)ld, Sk);
+  const int nqt = cdiv(Sq, kTile), nkt = cdiv(Sk, kTile);
+  if (nqt > kNoAllocMaxRows || nkt > BFA_NOALLOC_MAX_KV_TILES)
+    return fail(BFA_ERR_CAPACITY, "%d x %d tiles exceed the no-allocation limits (%d query tiles, %d key tiles)",
+                nqt, nkt, kNoAllocMaxRows, BFA_NOALLOC_MAX_KV_TILES);
+  bfa_status s;
+  if ((s = need_device(mask, "mask")) || (s = need_device(classes, "classes")) ||
+      (s = need_device(row_ptr, "row_ptr")) || (s = need_device(kv_tile, "kv_tile")) ||
+      (s = need_device(part, "part")) || (s = need_device(fine, "fine")) || (s = need_device(order, "order")))
+    return s;
+  uint8_t* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch))) return s;
+  GroupInfo* groups = reinterpret_cast<GroupInfo*>(scratch);
+  int32_t* row_group = reinterpret_cast<int32_t*>(scratch + 256);
+  int32_t* row_cnt = row_group + kNoAllocMaxRows;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto cleanup = []() {};
+  // every scratch word the kernels read is written first in this call, so the
+  // previous call's contents never leak into this one
+  GroupInfo g = make_group(0, Sq, 0, Sk, -1, -1);
+  g.row0 = 0;
+  g.cls_off = 0;
+  BFA_CUDA(launch_init_regular_groups(g, 1, 1, 0, 0, groups, row_group, nqt, st), "group table kernel");
+  BFA_CUDA(launch_dense_classify(mask, ld, Sq, Sk, classes, fine, st), "dense classify kernel");
+  BFA_CUDA(launch_rows(groups, row_group, classes, nqt, nkt, row_cnt, row_ptr, kv_tile, part, order, st),
+           "plan rows kernel");
+  return BFA_OK;
+}
