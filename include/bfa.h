@@ -85,6 +85,7 @@ typedef struct bfa_plan_info {
   int32_t max_kv_tiles;   /* longest key-tile count of a group                                    */
   int32_t window_left;    /* -1: no window                                                        */
   int32_t causal;         /* positional / BSR plans: 1 if kv_idx <= q_idx is applied             */
+  int32_t n_pairs;        /* work pairs: consecutive query tiles (2i, 2i+1) of one group          */
 } bfa_plan_info;
 
 /* Library version string. */
@@ -202,6 +203,14 @@ bfa_status bfa_plan_stats(const bfa_plan* plan, int64_t* n_full, int64_t* n_part
  */
 bfa_status bfa_plan_export(const bfa_plan* plan, int32_t* row_ptr, int32_t* kv_tile, uint8_t* partial,
                            uint32_t* fine, int32_t* order, uint8_t* classes, void* stream);
+
+/* Copy the plan's work pairs to HOST buffers (synchronises `stream`).  A work
+ * pair is two consecutive query tiles (2i, 2i+1) of one group that one CTA of the
+ * forward can run together; pair_row [n_pairs] holds the first row, bit-inverted
+ * (~row) when the group has no second tile; pair_order [n_pairs] lists the pairs
+ * longest first (by their total listed tiles), ties by pair index.  Either pointer
+ * may be NULL. */
+bfa_status bfa_plan_export_pairs(const bfa_plan* plan, int32_t* pair_row, int32_t* pair_order, void* stream);
 
 /* Synchronise `stream` and report BFA_ERR_TIMEOUT if a kernel that used the plan
  * hit its wait bound since the last call (the flag is then cleared). */

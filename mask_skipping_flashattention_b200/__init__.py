@@ -127,6 +127,12 @@ class Plan:
                                       P(classes), _stream(stream)))
         out = dict(row_ptr=row_ptr, kv_tile=kv_tile[:nnz], partial=partial[:nnz], order=order[:R],
                    classes=classes[:self.info["grid_tiles"]])
+        n_pairs = self.info["n_pairs"]
+        pair_row = np.zeros(max(n_pairs, 1), np.int32)
+        pair_order = np.zeros(max(n_pairs, 1), np.int32)
+        _lib.check(_L.bfa_plan_export_pairs(self.handle, P(pair_row), P(pair_order), _stream(stream)))
+        out["pair_row"] = pair_row[:n_pairs]
+        out["pair_order"] = pair_order[:n_pairs]
         if fine is not None:
             out["fine"] = fine[:n_part]
         return out

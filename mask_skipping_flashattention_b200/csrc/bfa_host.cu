@@ -33,7 +33,8 @@ cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, i
                                 uint32_t* err, int32_t* max_width, cudaStream_t s);
 cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
-                        int32_t* order, cudaStream_t s);
+                        int32_t* order, cudaStream_t s, int32_t* pair_row = nullptr, int32_t* pair_cost = nullptr,
+                        int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr);
 cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
                                   const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
                                   uint8_t* k_valid, cudaStream_t s);
@@ -50,7 +51,7 @@ using namespace bfa;
 // ----------------------------------------------------------------------------
 struct bfa_plan {
   int kind = 0, varlen = 0, batch = 0, hkv = 0, sq = 0, sk = 0, window = -1, causal = 0;
-  int n_groups = 0, n_rows = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
+  int n_groups = 0, n_rows = 0, n_pairs = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
   int64_t grid_tiles = 0;
   bool regular = false;   // every group the same shape: the group table is built on the device
   int regular_hkv = 1;    // groups per batch of a regular layout (BSR: Hkv)
@@ -68,6 +69,10 @@ struct bfa_plan {
   int32_t* part = nullptr;
   uint32_t* fine = nullptr;
   int32_t* order = nullptr;
+  int32_t* pair_row = nullptr;    // first row of each work pair (~row: single-row pair)
+  int32_t* pair_cost = nullptr;   // listed tiles of the pair
+  int32_t* pair_order = nullptr;  // longest-first order of the pairs
+  int32_t* pair_idx = nullptr;    // scratch: pair index of each row
   int32_t* qid = nullptr;
   uint8_t* qvalid = nullptr;
   int32_t* kid = nullptr;
@@ -148,6 +153,8 @@ cudaError_t plan_pool(cudaMemPool_t* out) {
   return cudaSuccess;
 }
 
+constexpr int kMaxKvTiles = 16384;  // key tiles per row: the row kernel's shared-memory buckets
+
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -173,6 +180,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   const size_t o_kv = L.take<int32_t>(cap_tiles);
   const size_t o_part = L.take<int32_t>(cap_tiles);
   const size_t o_ord = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_prow = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_pcost = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_pord = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_pidx = L.take<int32_t>(std::max(P->n_rows, 1));
   const size_t o_err = L.take<uint32_t>(1);
   const size_t o_mw = L.take<int32_t>(1);
   const size_t o_qid = L.take<int32_t>(std::max<int64_t>(qid_elems, 1));
@@ -195,6 +206,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->kv_tile = reinterpret_cast<int32_t*>(base + o_kv);
   P->part = reinterpret_cast<int32_t*>(base + o_part);
   P->order = reinterpret_cast<int32_t*>(base + o_ord);
+  P->pair_row = reinterpret_cast<int32_t*>(base + o_prow);
+  P->pair_cost = reinterpret_cast<int32_t*>(base + o_pcost);
+  P->pair_order = reinterpret_cast<int32_t*>(base + o_pord);
+  P->pair_idx = reinterpret_cast<int32_t*>(base + o_pidx);
   P->err = reinterpret_cast<uint32_t*>(base + o_err);
   P->max_width = reinterpret_cast<int32_t*>(base + o_mw);
   P->qid = reinterpret_cast<int32_t*>(base + o_qid);
@@ -238,9 +253,10 @@ bfa_status build_rows(bfa_plan* P) {
     cudaError_t e = cudaMemsetAsync(P->row_ptr, 0, sizeof(int32_t), P->stream);
     return e == cudaSuccess ? BFA_OK : cuda_fail(e, "empty plan");
   }
-  if (P->max_nkt + 1 > 50000) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
+  if (P->max_nkt > kMaxKvTiles) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
   cudaError_t e = launch_rows(P->groups, P->row_group, P->cls, P->n_rows, P->max_nkt, P->row_cnt, P->row_ptr,
-                              P->kv_tile, P->part, P->order, P->stream);
+                              P->kv_tile, P->part, P->order, P->stream, P->pair_row, P->pair_cost,
+                              P->pair_order, P->pair_idx);
   return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
 }
 
@@ -249,10 +265,12 @@ void finalize_layout(bfa_plan* P) {
   int64_t cls = 0;
   P->max_nkt = 0;
   P->max_nqt = 0;
+  P->n_pairs = 0;
   for (auto& g : P->groups_h) {
     g.row0 = row;
     g.cls_off = cls;
     row += g.nqt;
+    P->n_pairs += (g.nqt + 1) / 2;
     cls += static_cast<int64_t>(g.nqt) * g.nkt;
     P->max_nkt = std::max(P->max_nkt, g.nkt);
     P->max_nqt = std::max(P->max_nqt, g.nqt);
@@ -596,14 +614,24 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.Hkv = Hkv;
   p.D = D;
   p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? H / Hkv : H);
-  // Keep enough replicas of a row together to fill about two waves of CTAs, but
-  // no more heads than keep their K/V resident in L2 (about 64 MB).
-  const int64_t waves = 2LL * sm_count() * 2;
-  int chunk = static_cast<int>(std::min<int64_t>(p.rep, std::max<int64_t>(1, (waves + P->n_rows - 1) / std::max(P->n_rows, 1))));
+  p.plan.pair_row = P->pair_row;
+  p.plan.pair_order = P->pair_order;
+  p.plan.n_pairs = P->n_pairs;
+  // A CTA runs two query tiles that share K/V: two heads of one kv head on the
+  // same row when the GQA group is even (identical key lists), else two
+  // consecutive query tiles of one head.
+  p.pair_heads = ((H / Hkv) % 2 == 0) ? 1 : 0;
+  const int64_t units = p.pair_heads ? P->n_rows : P->n_pairs;
+  const int64_t items = p.pair_heads ? p.rep / 2 : p.rep;
+  // Keep enough replica units of a row together to fill about two waves of
+  // CTAs, but no more kv heads than stay resident in L2 (about 64 MB).
+  const int64_t waves = 2LL * sm_count();
+  int64_t chunk = std::min<int64_t>(items, std::max<int64_t>(1, (waves + units - 1) / std::max<int64_t>(units, 1)));
   const int64_t kv_head_bytes = std::max<int64_t>(1, static_cast<int64_t>(P->sk) * D * 4);
-  const int64_t l2_heads = std::max<int64_t>(1, (64LL << 20) / kv_head_bytes) * std::max(1, H / Hkv);
-  chunk = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(chunk, l2_heads)));
-  p.head_chunk = chunk;
+  const int64_t l2_kv_heads = std::max<int64_t>(1, (64LL << 20) / kv_head_bytes);
+  const int64_t units_per_kv_head = p.pair_heads ? std::max(1, (H / Hkv) / 2) : std::max(1, H / Hkv);
+  chunk = std::max<int64_t>(1, std::min<int64_t>(chunk, l2_kv_heads * units_per_kv_head));
+  p.head_chunk = static_cast<int>(chunk);
   p.varlen = P->varlen;
   p.Sq_lse = P->sq;
   const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
@@ -614,7 +642,7 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.o_sh = os[2];
   p.lse = lse;
   p.wait_ns = wait_ns;
-  const int64_t n_work = static_cast<int64_t>(P->n_rows) * p.rep;
+  const int64_t n_work = units * items;
   return launch_fwd(D, tq, tk, tv, p, n_work, st);
 }
 
@@ -670,6 +698,7 @@ BFA_API bfa_status bfa_plan_get_info(const bfa_plan* P, bfa_plan_info* info) {
   info->max_kv_tiles = P->max_nkt;
   info->window_left = P->window;
   info->causal = P->causal;
+  info->n_pairs = P->n_pairs;
   return BFA_OK;
 }
 
@@ -727,6 +756,22 @@ BFA_API bfa_status bfa_plan_export(const bfa_plan* P, int32_t* row_ptr, int32_t*
       ++np;
     }
   }
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_export_pairs(const bfa_plan* P, int32_t* pair_row, int32_t* pair_order, void* stream) {
+  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto cleanup = []() {};
+  if (P->n_pairs > 0) {
+    if (pair_row)
+      BFA_CUDA(cudaMemcpyAsync(pair_row, P->pair_row, sizeof(int32_t) * P->n_pairs, cudaMemcpyDeviceToHost, st),
+               "read pairs");
+    if (pair_order)
+      BFA_CUDA(cudaMemcpyAsync(pair_order, P->pair_order, sizeof(int32_t) * P->n_pairs, cudaMemcpyDeviceToHost, st),
+               "read pair order");
+  }
+  BFA_CUDA(cudaStreamSynchronize(st), "export pairs");
   return BFA_OK;
 }
 

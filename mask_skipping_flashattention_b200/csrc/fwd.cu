@@ -1,26 +1,32 @@
 // Fused mask-aware attention forward for sm_100a.
 //
-// One CTA computes one 128-row query tile of one (batch, head) against the key
-// tiles its plan row lists (BinFlash: iterate a pre-sorted list of non-empty key
-// blocks, run all-True blocks with no mask loads, apply the mask on partial
-// blocks only, skip all-False blocks).  Work items are taken in the plan's
-// longest-first row order, so the hardware's in-order CTA dispatch balances SMs
-// by the number of non-empty tiles.
+// Each CTA runs two 128-row query tiles ("slots") that share their keys and
+// values: either two heads of one kv head on the same query tile (GQA with an
+// even group), or two consecutive query tiles of one head.  The CTA walks the
+// union of the two tiles' plan lists (BinFlash: iterate a pre-sorted list of
+// non-empty key blocks, run all-True blocks with no mask loads, apply the mask on
+// partial blocks only, skip all-False blocks).  Work items are taken in the
+// plan's longest-first order, so the hardware's in-order CTA dispatch balances
+// SMs by the number of non-empty tiles.
 //
-// Warp roles (256 threads, two CTAs per SM):
-//   warp 0      TMA producer: Q once, then K_u / V_u of every listed tile u
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer:
-//                 S_u = Q K_u^T   (SS: both operands in shared memory, K-major)
-//                 O  += P_u V_u   (TS: P_u read from TMEM, V_u MN-major in smem)
-//   warps 2..3  idle (they give their registers to the softmax warpgroup)
-//   warps 4..7  softmax: one query row per thread, the whole S row in registers;
-//               mask on partial and edge tiles only, online base-2 softmax in
-//               fp32, P_u written back to TMEM over S_u as packed bf16, lazy
-//               rescale of O in TMEM; epilogue O / l -> bf16 and LSE.
+// Warp roles (384 threads, one CTA per SM):
+//   warp 0        TMA producer: Q of both slots, then K_u / V_u of every union
+//                 tile u into a two-stage ring
+//   warp 1        TMEM owner and single-thread tcgen05.mma issuer, ping-pong:
+//                   O0 += P0(u) V(u); S0 = Q0 K(u+1)^T; O1 += P1(u) V(u); S1 = Q1 K(u+1)^T
+//                 (S: SS, both operands K-major in shared memory; P V: TS, P is
+//                 the A operand in TMEM, V an MN-major shared-memory operand)
+//   warps 2..3    idle (they give their registers to the softmax warpgroups)
+//   warps 4..7    softmax of slot 0, warps 8..11 softmax of slot 1: one query
+//                 row per thread, the whole S row in registers; mask on partial
+//                 and edge tiles only, online base-2 softmax in fp32, P written
+//                 back to TMEM over S as packed bf16, lazy rescale of O in TMEM;
+//                 epilogue O / l -> bf16 and LSE.
+// While one slot's softmax runs, the tensor core works on the other slot.
 //
-// TMEM (256 columns): S / P at columns [0, 128), O at [128, 128 + D).
-// Shared memory: Q, K, V tiles (128 x D bf16 each) in 64-column panels with the
-// 128-byte swizzle that both TMA and the tensor core use.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// Shared memory: Q0, Q1 and two K and two V stages (128 x D bf16 each) in
+// 64-column panels with the 128-byte swizzle that TMA and the tensor core share.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -34,64 +40,93 @@ namespace bfa {
 
 using namespace ptx;
 
-
-
-// 256 threads: warpgroup 0 = warp 0 TMA producer, warp 1 MMA issuer (warps 2-3
-// idle), warpgroup 1 = softmax.  Two CTAs per SM: 128 registers per thread at
-// launch, redistributed so the softmax holds a whole S row in registers.  The
-// split must add up to the launch allocation: 128 * kRegsWG0 + 128 * kRegsWG1 ==
-// 256 * kRegsLaunch (checked against the compiled kernel before launching).
-constexpr int kThreads = 256;
-constexpr int kRegsLaunch = 128;
-constexpr uint32_t kRegsWG0 = 56;
-constexpr uint32_t kRegsWG1 = 200;
-static_assert(128 * kRegsWG0 + 128 * kRegsWG1 == kThreads * kRegsLaunch, "register split");
+// 128 * kRegsWG0 + 256 * kRegsSoftmax must equal kThreads * kRegsLaunch: the
+// increase draws only on the registers the block was launched with.  The
+// compiled kernel's launch count is checked before every first launch.
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;
+constexpr uint32_t kRegsWG0 = 72;
+constexpr uint32_t kRegsSoftmax = 216;
+static_assert(128 * kRegsWG0 + 256 * kRegsSoftmax == kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
+constexpr int kStages = 2;
 
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kSmemBytes = 3 * kTileBytes + 1024;
-  static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColO = 128;
+  static constexpr int kSmemBytes = (2 + 2 * kStages) * kTileBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);
 };
 
 struct Work {
-  int32_t e0, n;        // first listed tile and count
-  int32_t b, h, hk;
-  int32_t qt;           // query tile inside the group
+  int32_t row[2];       // plan row of each slot (-1: slot unused)
+  int32_t e0[2], n[2];  // first listed tile and count of each slot's row
+  int32_t qt[2];        // query tile inside the group
+  int32_t h[2];         // query head of each slot
+  int32_t b, hk;
+  int32_t same_row;     // both slots run the same row (so the same list)
   int32_t q_off, q_len, k_off, k_len;
   int32_t qid_off, kid_off, kbit_off;
 };
 
+// replica index -> (batch, head) of a plan row
+__device__ __forceinline__ void replica_bh(const FwdParams& p, const GroupInfo& g, int j, int& b, int& h) {
+  if (p.plan.kind == 1 /*BFA_PLAN_DENSE*/) {
+    b = j / p.H;
+    h = j % p.H;
+  } else if (p.plan.kind == 4 /*BFA_PLAN_BSR*/) {
+    b = g.b;
+    h = g.hkv * (p.H / p.Hkv) + j;
+  } else {
+    b = p.varlen ? 0 : g.b;
+    h = j;
+  }
+}
+
 __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk) {
-  const int64_t R = p.plan.n_rows;
+  const int64_t units = p.pair_heads ? p.plan.n_rows : p.plan.n_pairs;
+  const int64_t items = p.pair_heads ? p.rep / 2 : p.rep;  // replica units per row / pair
   const int64_t chunk = p.head_chunk;
-  const int64_t hg = w / (R * chunk);
-  const int64_t rem = w - hg * R * chunk;
-  const int64_t gs = min(chunk, static_cast<int64_t>(p.rep) - hg * chunk);
+  const int64_t hg = w / (units * chunk);
+  const int64_t rem = w - hg * units * chunk;
+  const int64_t gs = min(chunk, items - hg * chunk);
   const int i = static_cast<int>(rem / gs);
   const int j = static_cast<int>(hg * chunk + rem % gs);
-  const int row = p.plan.order[i];
-  const GroupInfo g = p.plan.groups[p.plan.row_group[row]];
-  wk.e0 = p.plan.row_ptr[row];
-  wk.n = p.plan.row_ptr[row + 1] - wk.e0;
-  wk.qt = row - g.row0;
-  if (p.plan.kind == 1 /*BFA_PLAN_DENSE*/) {
-    wk.b = j / p.H;
-    wk.h = j % p.H;
-  } else if (p.plan.kind == 4 /*BFA_PLAN_BSR*/) {
-    wk.b = g.b;
-    wk.h = g.hkv * (p.H / p.Hkv) + j;
+  int r0, r1;
+  if (p.pair_heads) {
+    r0 = r1 = p.plan.order[i];
   } else {
-    wk.b = p.varlen ? 0 : g.b;
-    wk.h = j;
+    const int pr = p.plan.pair_row[p.plan.pair_order[i]];
+    r0 = pr >= 0 ? pr : ~pr;
+    r1 = pr >= 0 ? r0 + 1 : -1;
   }
-  wk.hk = wk.h / (p.H / p.Hkv);
+  const GroupInfo g = p.plan.groups[p.plan.row_group[r0]];
+  wk.same_row = p.pair_heads;
+  wk.row[0] = r0;
+  wk.row[1] = r1;
+  for (int s = 0; s < 2; ++s) {
+    const int r = wk.row[s];
+    wk.e0[s] = r >= 0 ? p.plan.row_ptr[r] : 0;
+    wk.n[s] = r >= 0 ? p.plan.row_ptr[r + 1] - wk.e0[s] : 0;
+    wk.qt[s] = r >= 0 ? r - g.row0 : 0;
+  }
+  int b, h0, h1;
+  if (p.pair_heads) {
+    replica_bh(p, g, 2 * j, b, h0);
+    replica_bh(p, g, 2 * j + 1, b, h1);
+  } else {
+    replica_bh(p, g, j, b, h0);
+    h1 = h0;
+  }
+  wk.b = b;
+  wk.h[0] = h0;
+  wk.h[1] = h1;
+  wk.hk = h0 / (p.H / p.Hkv);
   wk.q_off = g.q_off;
   wk.q_len = g.q_len;
   wk.k_off = g.k_off;
@@ -101,11 +136,45 @@ __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk)
   wk.kbit_off = g.kbit_off;
 }
 
-// attend-bits of one query row against the 128 columns of key tile `kt`
-__device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& wk, int row, int kt, int part,
-                                               uint32_t (&am)[4]) {
+// Walk the union of the two slots' ascending key-tile lists.
+struct UnionWalk {
+  const int32_t* kv;
+  int ea, na, eb, nb, ia, ib;
+  bool same;
+  __device__ __forceinline__ void init(const FwdParams& p, const Work& wk) {
+    kv = p.plan.kv_tile;
+    ea = wk.e0[0];
+    na = wk.n[0];
+    eb = wk.e0[1];
+    nb = wk.n[1];
+    ia = ib = 0;
+    same = wk.same_row != 0;
+  }
+  // next tile: kt, and whether slot 0 / slot 1 have it; false at the end
+  __device__ __forceinline__ bool next(int& kt, bool& a, bool& b) {
+    if (same) {
+      if (ia >= na) return false;
+      kt = kv[ea + ia++];
+      a = b = true;
+      return true;
+    }
+    const int ka = ia < na ? kv[ea + ia] : 0x7fffffff;
+    const int kb = ib < nb ? kv[eb + ib] : 0x7fffffff;
+    if (ka == 0x7fffffff && kb == 0x7fffffff) return false;
+    kt = min(ka, kb);
+    a = ka == kt;
+    b = kb == kt;
+    ia += a;
+    ib += b;
+    return true;
+  }
+};
+
+// attend-bits of one query row (position qpos in its group) against the 128
+// columns of key tile `kt`
+__device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& wk, int qpos, int row, int kt,
+                                               int part, uint32_t (&am)[4]) {
   const int ncols = wk.k_len - kt * kTile;  // in-range columns (may exceed 128)
-  const int qpos = wk.qt * kTile + row;     // position of the row inside its group
   if (p.plan.mask_mode == MASK_BITS) {
     if (part >= 0) {
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.plan.fine + static_cast<int64_t>(part) * kFineWordsPerTile +
@@ -138,7 +207,7 @@ __device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& w
       am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
     }
   } else {  // MASK_POS: causal kv_pos <= q_pos, optional window q_pos - kv_pos < W
-    int hi = p.plan.causal ? (qpos - kt * kTile) : 127;            // last attended column
+    int hi = p.plan.causal ? (qpos - kt * kTile) : 127;                           // last attended column
     int lo = (p.plan.window >= 0) ? (qpos - kt * kTile - p.plan.window + 1) : 0;  // first attended column
     if (part < 0) { hi = 127; lo = 0; }
 #pragma unroll
@@ -161,17 +230,36 @@ __device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& w
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ __forceinline__ void issue_s(uint32_t tS, uint8_t* sQ, uint8_t* sK) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    umma_ss(tS, smem_desc(smem_u32(sQ + off), 16, 1024), smem_desc(smem_u32(sK + off), 16, 1024),
+            Cfg<D>::kIdescQK, kk > 0);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint8_t* sV, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    umma_ts(tO, tP + kk * 8, smem_desc(smem_u32(sV + kk * 2048), 16384, 1024), Cfg<D>::kIdescPV,
+            (acc || kk > 0) ? 1u : 0u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
     bfa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::kTileBytes;
-  uint8_t* sV = smem + 2 * C::kTileBytes;
+  uint8_t* const sQ0 = smem;
+  uint8_t* const sQ1 = smem + C::kTileBytes;
+  uint8_t* const sK0 = smem + 2 * C::kTileBytes;
+  uint8_t* const sV0 = smem + (2 + kStages) * C::kTileBytes;
 
-  enum { BQ = 0, BKF, BKE, BVF, BVE, BS, BP, BO, BDONE, NBAR };
+  enum { BQ = 0, BKF = 1, BKE = 3, BVF = 5, BVE = 7, BS = 9, BP = 11, BO = 13, BDONE = 14, NBAR = 15 };
   __shared__ __align__(8) uint64_t bars[NBAR];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -179,18 +267,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto sK = [&](int st) { return sK0 + st * C::kTileBytes; };
+  auto sV = [&](int st) { return sV0 + st * C::kTileBytes; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(bar(BQ), 1);
-    mbar_init(bar(BKF), 1);
-    mbar_init(bar(BKE), 1);
-    mbar_init(bar(BVF), 1);
-    mbar_init(bar(BVE), 1);
-    mbar_init(bar(BS), 1);
-    mbar_init(bar(BP), 4);
-    mbar_init(bar(BO), 1);
-    mbar_init(bar(BDONE), 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == BP || i == BP + 1) ? 4 : 1);
     fence_barrier_init();
     decode_work(p, blockIdx.x, wk_s);
   }
@@ -204,69 +286,121 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = tmem_slot;
   const Work wk = wk_s;
   const uint64_t cap = p.wait_ns;
+  const bool any_tiles = wk.n[0] + wk.n[1] > 0;
 
   if (warp < 4) {
     // ============================================================ warpgroup 0
     regs_dec<kRegsWG0>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      if (lane == 0 && wk.n > 0) {
+      if (lane == 0 && any_tiles) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        const int qs = wk.q_off + wk.qt * kTile;
-        mbar_expect_tx(bar(BQ), C::kTileBytes);
+        mbar_expect_tx(bar(BQ), ((wk.n[0] > 0 ? 1 : 0) + (wk.n[1] > 0 ? 1 : 0)) * C::kTileBytes);
+        for (int s = 0; s < 2; ++s) {
+          if (wk.n[s] == 0) continue;
+          const int qs = wk.q_off + wk.qt[s] * kTile;
+          uint8_t* dq = s ? sQ1 : sQ0;
 #pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_4d(smem_u32(sQ + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h, qs, wk.b);
-        int last_k = -1, last_v = -1;  // last issued phase of each full barrier
-        for (int u = 0; u < wk.n; ++u) {
-          const int kt = p.plan.kv_tile[wk.e0 + u];
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h[s], qs, wk.b);
+        }
+        UnionWalk walk;
+        walk.init(p, wk);
+        int kt;
+        bool ha, hb;
+        int u = 0;
+        int last_k[kStages] = {-1, -1}, last_v[kStages] = {-1, -1};  // last fill of each stage
+        while (walk.next(kt, ha, hb)) {
+          const int st = u & 1;
           const int ks = wk.k_off + kt * kTile;
-          if (u > 0 && !mbar_wait(bar(BKE), (u - 1) & 1, cap, &abort_flag)) break;
-          mbar_expect_tx(bar(BKF), C::kTileBytes);
+          if (u >= kStages && !mbar_wait(bar(BKE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
+          mbar_expect_tx(bar(BKF + st), C::kTileBytes);
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_4d(smem_u32(sK + pn * 16384), &tmK, bar(BKF), pn * 64, wk.hk, ks, wk.b);
-          last_k = u;
-          if (u > 0 && !mbar_wait(bar(BVE), (u - 1) & 1, cap, &abort_flag)) break;
-          mbar_expect_tx(bar(BVF), C::kTileBytes);
+            tma_load_4d(smem_u32(sK(st) + pn * 16384), &tmK, bar(BKF + st), pn * 64, wk.hk, ks, wk.b);
+          last_k[st] = u;
+          if (u >= kStages && !mbar_wait(bar(BVE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
+          mbar_expect_tx(bar(BVF + st), C::kTileBytes);
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_4d(smem_u32(sV + pn * 16384), &tmV, bar(BVF), pn * 64, wk.hk, ks, wk.b);
-          last_v = u;
+            tma_load_4d(smem_u32(sV(st) + pn * 16384), &tmV, bar(BVF + st), pn * 64, wk.hk, ks, wk.b);
+          last_v[st] = u;
+          ++u;
         }
         // every copy this CTA issued must land before it can exit (bounded; on the
         // normal path these phases completed long ago)
         volatile int no_abort = 0;
         mbar_wait(bar(BQ), 0, cap, &no_abort);
-        if (last_k >= 0) mbar_wait(bar(BKF), last_k & 1, cap, &no_abort);
-        if (last_v >= 0) mbar_wait(bar(BVF), last_v & 1, cap, &no_abort);
+        for (int st = 0; st < kStages; ++st) {
+          if (last_k[st] >= 0) mbar_wait(bar(BKF + st), (last_k[st] >> 1) & 1, cap, &no_abort);
+          if (last_v[st] >= 0) mbar_wait(bar(BVF + st), (last_v[st] >> 1) & 1, cap, &no_abort);
+        }
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
-      if (lane == 0 && wk.n > 0) {
-        const uint32_t tS = tmem + C::kColS, tO = tmem + C::kColO;
+      if (lane == 0 && any_tiles) {
+        const uint32_t tS0 = tmem + C::kColS0, tS1 = tmem + C::kColS1;
+        const uint32_t tO0 = tmem + C::kColO0, tO1 = tmem + C::kColO1;
+        UnionWalk walk;
+        walk.init(p, wk);
         bool ok = mbar_wait(bar(BQ), 0, cap, &abort_flag);
-        for (int u = 0; ok && u < wk.n; ++u) {
-          if (!mbar_wait(bar(BKF), u & 1, cap, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_ss(tS, smem_desc(smem_u32(sQ + off), 16, 1024), smem_desc(smem_u32(sK + off), 16, 1024),
-                    C::kIdescQK, kk > 0);
+        int cnt0 = 0, cnt1 = 0;           // P phases consumed per slot
+        bool started0 = false, started1 = false;
+        int kt;
+        bool a, b, na_, nb_;
+        bool have = ok && walk.next(kt, a, b);
+        if (have) {
+          ok = mbar_wait(bar(BKF + 0), 0, cap, &abort_flag);
+          if (ok) {
+            tc_fence_after();
+            if (a) { issue_s<D>(tS0, sQ0, sK(0)); umma_commit(bar(BS + 0)); }
+            if (b) { issue_s<D>(tS1, sQ1, sK(0)); umma_commit(bar(BS + 1)); }
+            umma_commit(bar(BKE + 0));
           }
-          umma_commit(bar(BS));
-          umma_commit(bar(BKE));
-          if (!mbar_wait(bar(BP), u & 1, cap, &abort_flag)) { ok = false; break; }
-          if (!mbar_wait(bar(BVF), u & 1, cap, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tO, tS + kk * 8, smem_desc(smem_u32(sV + kk * 2048), 16384, 1024), C::kIdescPV,
-                    (u > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar(BVE));
+        }
+        for (int u = 0; ok && have; ++u) {
+          const int st = u & 1, st1 = (u + 1) & 1;
+          const bool have_next = walk.next(kt, na_, nb_);
+          bool v_ready = false, k_ready = false;
+          // slot 0: O0 += P0(u) V(u), then S0 = Q0 K(u+1)^T over the consumed P0
+          if (a) {
+            if (!mbar_wait(bar(BP + 0), cnt0 & 1, cap, &abort_flag)) { ok = false; break; }
+            ++cnt0;
+            if (!mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+            v_ready = true;
+            tc_fence_after();
+            issue_pv<D>(tO0, tS0, sV(st), started0);
+            started0 = true;
+          }
+          if (have_next && na_) {
+            if (!mbar_wait(bar(BKF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+            k_ready = true;
+            tc_fence_after();
+            issue_s<D>(tS0, sQ0, sK(st1));
+            umma_commit(bar(BS + 0));
+          }
+          // slot 1: O1 += P1(u) V(u), then S1 = Q1 K(u+1)^T
+          if (b) {
+            if (!mbar_wait(bar(BP + 1), cnt1 & 1, cap, &abort_flag)) { ok = false; break; }
+            ++cnt1;
+            if (!v_ready && !mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv<D>(tO1, tS1, sV(st), started1);
+            started1 = true;
+          }
+          if (have_next && nb_) {
+            if (!k_ready && !mbar_wait(bar(BKF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_s<D>(tS1, sQ1, sK(st1));
+            umma_commit(bar(BS + 1));
+          }
+          if (have_next) umma_commit(bar(BKE + st1));
+          umma_commit(bar(BVE + st));
+          a = na_;
+          b = nb_;
+          have = have_next;
         }
         if (ok) umma_commit(bar(BO));
         // every MMA issued must be finished before TMEM is released (bounded)
@@ -276,132 +410,142 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   } else {
-    // ============================================================ warpgroup 1: softmax
-    regs_inc<kRegsWG1>();
+    // ============================================================ softmax warpgroups
+    regs_inc<kRegsSoftmax>();
+    const int slot = (warp >> 2) - 1;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const uint32_t tS = tmem_addr(tmem + C::kColS, quarter * 32, 0);
-    const uint32_t tO = tmem_addr(tmem + C::kColO, quarter * 32, 0);
-    const float c = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    int kt_next = wk.n > 0 ? p.plan.kv_tile[wk.e0] : 0;
-    int part_next = wk.n > 0 ? p.plan.part[wk.e0] : -1;
-    for (int u = 0; u < wk.n; ++u) {
-      const int kt = kt_next, part = part_next;
-      if (u + 1 < wk.n) {  // next list entry, off the critical path
-        kt_next = p.plan.kv_tile[wk.e0 + u + 1];
-        part_next = p.plan.part[wk.e0 + u + 1];
-      }
-      const bool masked = part >= 0 || (kt + 1) * kTile > wk.k_len;
-      uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (masked) row_mask_words(p, wk, row, kt, part, am);
+    const int my_row = slot ? wk.row[1] : wk.row[0];
+    if (my_row >= 0) {
+      const uint32_t tS = tmem_addr(tmem + (slot ? C::kColS1 : C::kColS0), quarter * 32, 0);
+      const uint32_t tO = tmem_addr(tmem + (slot ? C::kColO1 : C::kColO0), quarter * 32, 0);
+      const uint32_t barS = bar(BS + slot), barP = bar(BP + slot);
+      const int n = slot ? wk.n[1] : wk.n[0];
+      const int e0 = slot ? wk.e0[1] : wk.e0[0];
+      const int qpos = (slot ? wk.qt[1] : wk.qt[0]) * kTile + row;  // position of this row inside its group
+      const float c = p.scale_log2;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      int kt_next = n > 0 ? p.plan.kv_tile[e0] : 0;
+      int part_next = n > 0 ? p.plan.part[e0] : -1;
+      for (int t = 0; t < n; ++t) {
+        const int kt = kt_next, part = part_next;
+        if (t + 1 < n) {  // next list entry, off the critical path
+          kt_next = p.plan.kv_tile[e0 + t + 1];
+          part_next = p.plan.part[e0 + t + 1];
+        }
+        const bool masked = part >= 0 || (kt + 1) * kTile > wk.k_len;
+        uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        if (masked) row_mask_words(p, wk, qpos, row, kt, part, am);
 
-      const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
-      if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit
-      tc_fence_after();
-      // the whole S row in registers: four loads in flight, one wait
-      uint32_t sr[128];
-      tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      tmem_wait_ld();
-      reg_fence(sr);
-      float* s = reinterpret_cast<float*>(sr);
-      if (masked) {
+        const bool got = mbar_wait(barS, t & 1, cap, &abort_flag);
+        if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit
+        tc_fence_after();
+        // the whole S row in registers: four loads in flight, one wait
+        uint32_t sr[128];
+        tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_wait_ld();
+        reg_fence(sr);
+        float* s = reinterpret_cast<float*>(sr);
+        if (masked) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
-          if (!((am[j >> 5] >> (j & 31)) & 1u)) s[j] = -INFINITY;
-      }
-      // row max, 8 independent chains
-      float mx8[8];
+          for (int j = 0; j < 128; ++j)
+            if (!((am[j >> 5] >> (j & 31)) & 1u)) s[j] = -INFINITY;
+        }
+        // row max, 8 independent chains
+        float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-      for (int j = 8; j < 128; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mnew = fmaxf(m, mx * c);
-      // The reference max m only moves when some row of the warp grew by more
-      // than 2^8; then every row of the warp moves to its true running max (alpha
-      // is 1 for rows that did not grow).  The decision is warp-uniform because
-      // the O rescale uses whole-warp TMEM loads and stores.
-      if (__any_sync(0xffffffffu, mnew > m + kRescaleThreshold)) {
-        const float alpha = (mnew == m) ? 1.f : ex2_approx(m - mnew);  // 0 when m = -inf
-        l *= alpha;
-        if (u > 0) {
+        for (int j = 8; j < 128; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mnew = fmaxf(m, mx * c);
+        // The reference max m only moves when some row of the warp grew by more
+        // than 2^8; then every row of the warp moves to its true running max
+        // (alpha is 1 for rows that did not grow).  The decision is warp-uniform
+        // because the O rescale uses whole-warp TMEM loads and stores.
+        if (__any_sync(0xffffffffu, mnew > m + kRescaleThreshold)) {
+          const float alpha = (mnew == m) ? 1.f : ex2_approx(m - mnew);  // 0 when m = -inf
+          l *= alpha;
+          if (t > 0) {
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld_32x32b_x32(tO + cc * 32, o);
+              tmem_wait_ld();
+              reg_fence(o);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+              tmem_st_32x32b_x32(tO + cc * 32, o);
+            }
+          }
+          m = mnew;
+        }
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        // p = 2^(s*c - m), 4 independent row-sum chains; packed bf16 pairs go to
+        // the first 64 columns of S (the A operand of the P V product)
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float p0 = ex2_approx(fmaf(s[2 * j], c, -mref));
+          const float p1 = ex2_approx(fmaf(s[2 * j + 1], c, -mref));
+          rs[j & 3] += p0 + p1;
+          pk[j] = pack_bf16x2(p0, p1);
+        }
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(barP);
+      }
+      // ---------------------------------------------------------- epilogue
+      if (ok && n > 0) {
+        const bool got = mbar_wait(bar(BO), 0, cap, &abort_flag);
+        ok = !__any_sync(0xffffffffu, !got);
+      }
+      tc_fence_after();
+      const bool store = qpos < wk.q_len;  // TMEM loads below stay whole-warp; only stores are per row
+      if (ok) {
+        const int64_t tok = static_cast<int64_t>(wk.q_off) + qpos;
+        const int h = slot ? wk.h[1] : wk.h[0];
+        __nv_bfloat16* op =
+            p.out + static_cast<int64_t>(wk.b) * p.o_sb + tok * p.o_ss + static_cast<int64_t>(h) * p.o_sh;
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          if (n > 0) {
             tmem_ld_32x32b_x32(tO + cc * 32, o);
             tmem_wait_ld();
             reg_fence(o);
+          } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st_32x32b_x32(tO + cc * 32, o);
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            pkd[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(op + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pkd[4 * j], pkd[4 * j + 1], pkd[4 * j + 2], pkd[4 * j + 3]);
           }
         }
-        m = mnew;
-      }
-      const float mref = (m == -INFINITY) ? 0.f : m;
-      // p = 2^(s*c - m), 4 independent row-sum chains; packed bf16 pairs go to
-      // the first 64 columns of S (the A operand of the P V product)
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float p0 = ex2_approx(fmaf(s[2 * j], c, -mref));
-        const float p1 = ex2_approx(fmaf(s[2 * j + 1], c, -mref));
-        rs[j & 3] += p0 + p1;
-        pk[j] = pack_bf16x2(p0, p1);
-      }
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BP));
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok && wk.n > 0) {
-      const bool got = mbar_wait(bar(BO), 0, cap, &abort_flag);
-      ok = !__any_sync(0xffffffffu, !got);
-    }
-    tc_fence_after();
-    const int qpos = wk.qt * kTile + row;
-    const bool store = qpos < wk.q_len;  // TMEM loads below stay whole-warp; only stores are per row
-    if (ok) {
-      const int64_t tok = static_cast<int64_t>(wk.q_off) + qpos;
-      __nv_bfloat16* op = p.out + static_cast<int64_t>(wk.b) * p.o_sb + tok * p.o_ss + static_cast<int64_t>(wk.h) * p.o_sh;
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        if (wk.n > 0) {
-          tmem_ld_32x32b_x32(tO + cc * 32, o);
-          tmem_wait_ld();
-          reg_fence(o);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        if (p.lse && store) {
+          const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          const int64_t li = p.varlen ? static_cast<int64_t>(h) * p.Sq_lse + tok
+                                      : (static_cast<int64_t>(wk.b) * p.H + h) * p.Sq_lse + qpos;
+          p.lse[li] = lse;
         }
-        uint32_t pkd[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          pkd[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(op + cc * 32);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pkd[4 * j], pkd[4 * j + 1], pkd[4 * j + 2], pkd[4 * j + 3]);
-        }
-      }
-      if (p.lse && store) {
-        const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int64_t li = p.varlen ? static_cast<int64_t>(wk.h) * p.Sq_lse + tok
-                                    : (static_cast<int64_t>(wk.b) * p.H + wk.h) * p.Sq_lse + qpos;
-        p.lse[li] = lse;
       }
     }
   }
@@ -439,11 +583,12 @@ int fwd_smem_bytes(int D) { return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSm
 // The setmaxnreg split is only safe if every thread is launched with exactly
 // kRegsLaunch registers; refuse to launch otherwise.
 template <typename K>
-static cudaError_t check_regs(K kernel) {
+static cudaError_t prepare(K kernel, int smem) {
   cudaFuncAttributes a;
   cudaError_t e = cudaFuncGetAttributes(&a, kernel);
   if (e != cudaSuccess) return e;
-  return a.numRegs == kRegsLaunch ? cudaSuccess : cudaErrorInvalidKernelImage;
+  if (a.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -451,25 +596,12 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
   if (n_work <= 0) return cudaSuccess;
   if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (D == 64) {
-    static bool set = false;
-    if (!set) {
-      cudaError_t e = check_regs(bfa_fwd_kernel<64>);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(bfa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<64>::kSmemBytes);
-      if (e != cudaSuccess) return e;
-      set = true;
-    }
+    static cudaError_t ready = prepare(bfa_fwd_kernel<64>, Cfg<64>::kSmemBytes);
+    if (ready != cudaSuccess) return ready;
     bfa_fwd_kernel<64><<<static_cast<unsigned>(n_work), kThreads, Cfg<64>::kSmemBytes, s>>>(tq, tk, tv, p);
   } else {
-    static bool set = false;
-    if (!set) {
-      cudaError_t e = check_regs(bfa_fwd_kernel<128>);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(bfa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg<128>::kSmemBytes);
-      if (e != cudaSuccess) return e;
-      set = true;
-    }
+    static cudaError_t ready = prepare(bfa_fwd_kernel<128>, Cfg<128>::kSmemBytes);
+    if (ready != cudaSuccess) return ready;
     bfa_fwd_kernel<128><<<static_cast<unsigned>(n_work), kThreads, Cfg<128>::kSmemBytes, s>>>(tq, tk, tv, p);
   }
   return cudaGetLastError();

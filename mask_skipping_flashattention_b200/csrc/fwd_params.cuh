@@ -14,7 +14,8 @@ struct FwdParams {
   PlanDev plan;
   int32_t B, H, Hkv, D;
   int32_t rep;          // (batch, head) replicas that share one plan row
-  int32_t head_chunk;   // replicas kept together in the work order (K/V reuse in L2)
+  int32_t pair_heads;   // 1: a CTA runs two heads of one kv head on one row; 0: two rows of one head
+  int32_t head_chunk;   // replica units kept together in the work order (K/V reuse in L2)
   int32_t varlen;
   int32_t Sq_lse;       // batched: per-batch query length (lse row pitch); varlen: total_q
   float scale_log2;     // softmax scale * log2(e)

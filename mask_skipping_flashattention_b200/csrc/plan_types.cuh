@@ -49,12 +49,15 @@ struct PlanDev {
   const int32_t* part;       // [listed tiles]: -1 full, else the tile's class-grid index
   const uint32_t* fine;      // [grid_tiles * 512] (dense plans) indexed by grid index
   const int32_t* order;      // [n_rows] longest first
+  const int32_t* pair_row;   // [n_pairs] first row of each work pair (~row: single row)
+  const int32_t* pair_order; // [n_pairs] longest first
   const int32_t* qid;        // padded q block ids  (block-id plans)
   const uint8_t* qvalid;     // padded q validity   (block-id plans)
   const int32_t* kid;        // padded k block ids  (block-id plans)
   const uint32_t* kbits;     // padded k validity bits (block-id plans)
   uint32_t* err;             // device error word
   int32_t n_rows;
+  int32_t n_pairs;
   int32_t n_groups;
   int32_t mask_mode;
   int32_t causal;

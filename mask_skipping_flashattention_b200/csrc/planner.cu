@@ -213,41 +213,18 @@ __global__ void k_bsr_classify(const int32_t* __restrict__ indptr, const int32_t
 }
 
 // ----------------------------------------------------------------------------
-// classes -> CSR lists + longest-first order (one CTA of 1024 threads)
+// classes -> CSR lists + longest-first orders (one CTA of 1024 threads)
 // ----------------------------------------------------------------------------
-// Dynamic shared memory: (max_nkt + 1) ints of bucket counters.
-__global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ groups,
-                                               const int32_t* __restrict__ row_group,
-                                               const uint8_t* __restrict__ cls, int n_rows, int max_nkt,
-                                               int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_ptr,
-                                               int32_t* __restrict__ kv_tile, int32_t* __restrict__ part,
-                                               int32_t* __restrict__ order) {
-  extern __shared__ int32_t bucket[];  // [max_nkt + 1]
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t carry;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-
-  // 1. count the listed tiles of every row (warp per row, ballot + popc)
-  for (int r = warp; r < n_rows; r += nw) {
-    const GroupInfo g = groups[row_group[r]];
-    const uint8_t* c = cls + g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
-    int n = 0;
-    for (int k0 = 0; k0 < g.nkt; k0 += 32) {
-      const int kt = k0 + lane;
-      n += __popc(__ballot_sync(0xffffffffu, kt < g.nkt && c[kt] != 0));
-    }
-    if (lane == 0) row_cnt[r] = n;
-  }
-  for (int i = tid; i <= max_nkt; i += blockDim.x) bucket[i] = 0;
-  if (tid == 0) carry = 0;
+// Exclusive prefix sum over n values read through `get(i)`; out[i] = sum of the
+// values before i; returns the total.  All threads of the CTA call it.
+template <typename Get>
+__device__ int block_exclusive_scan(int n, Get get, int32_t* out, int32_t* warp_sums, int32_t* carry) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) *carry = 0;
   __syncthreads();
-
-  // 2. exclusive scan of the counts -> row_ptr; bucket histogram of the counts
-  for (int base = 0; base < n_rows; base += blockDim.x) {
-    const int r = base + tid;
-    const int v = r < n_rows ? row_cnt[r] : 0;
-    if (r < n_rows) atomicAdd(&bucket[v], 1);
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + tid;
+    const int v = i < n ? get(i) : 0;
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -266,13 +243,84 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
       warp_sums[lane] = w;
     }
     __syncthreads();
-    const int incl = x + (warp ? warp_sums[warp - 1] : 0) + carry;
-    if (r < n_rows) row_ptr[r] = incl - v;
+    const int incl = x + (warp ? warp_sums[warp - 1] : 0) + *carry;
+    if (i < n) out[i] = incl - v;
     __syncthreads();
-    if (tid == blockDim.x - 1) carry = incl;
+    if (tid == blockDim.x - 1) *carry = incl;
     __syncthreads();
   }
-  if (tid == 0) row_ptr[n_rows] = carry;
+  const int total = *carry;
+  __syncthreads();
+  return total;
+}
+
+// Stable sort of the indices 0..n-1 by descending key (keys in [0, max_key]):
+// a counting sort whose placement runs chunk by chunk and warp by warp, so equal
+// keys keep index order.  `bucket` is shared memory of max_key + 1 ints.
+__device__ void block_stable_order_desc(int n, const int32_t* keys, int max_key, int32_t* bucket,
+                                        int32_t* order) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int i = tid; i <= max_key; i += blockDim.x) bucket[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) atomicAdd(&bucket[keys[i]], 1);
+  __syncthreads();
+  if (tid == 0) {  // bucket[k] <- first output slot of key k
+    int acc = 0;
+    for (int k = max_key; k >= 0; --k) {
+      const int h = bucket[k];
+      bucket[k] = acc;
+      acc += h;
+    }
+  }
+  __syncthreads();
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + tid;
+    const int key = i < n ? keys[i] : -1;
+    const uint32_t same = __match_any_sync(0xffffffffu, key);
+    const int rank = __popc(same & lt_mask);
+    for (int w = 0; w < nw; ++w) {
+      if (warp == w && key >= 0) order[bucket[key] + rank] = i;
+      __syncthreads();
+      if (warp == w && key >= 0 && rank == 0) bucket[key] += __popc(same);
+      __syncthreads();
+    }
+  }
+}
+
+// Rows -> lists and row order; with pair outputs also the work pairs (two
+// consecutive query tiles of one group) and their longest-first order.
+// Dynamic shared memory: (2 * max_nkt + 1) ints.
+__global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ groups,
+                                               const int32_t* __restrict__ row_group,
+                                               const uint8_t* __restrict__ cls, int n_rows, int max_nkt,
+                                               int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_ptr,
+                                               int32_t* __restrict__ kv_tile, int32_t* __restrict__ part,
+                                               int32_t* __restrict__ order, int32_t* __restrict__ pair_row,
+                                               int32_t* __restrict__ pair_cost, int32_t* __restrict__ pair_order,
+                                               int32_t* __restrict__ pair_idx) {
+  extern __shared__ int32_t bucket[];
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  // 1. count the listed tiles of every row (warp per row, ballot + popc)
+  for (int r = warp; r < n_rows; r += nw) {
+    const GroupInfo g = groups[row_group[r]];
+    const uint8_t* c = cls + g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
+    int n = 0;
+    for (int k0 = 0; k0 < g.nkt; k0 += 32) {
+      const int kt = k0 + lane;
+      n += __popc(__ballot_sync(0xffffffffu, kt < g.nkt && c[kt] != 0));
+    }
+    if (lane == 0) row_cnt[r] = n;
+  }
+  __syncthreads();
+
+  // 2. exclusive scan of the counts -> row_ptr
+  const int total = block_exclusive_scan(n_rows, [&](int i) { return row_cnt[i]; }, row_ptr, warp_sums, &carry);
+  if (tid == 0) row_ptr[n_rows] = total;
   __syncthreads();
 
   // 3. write each row's ascending list (warp per row)
@@ -294,35 +342,28 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
     }
   }
 
-  // 4. longest-first stable order: counting sort over the counts.
-  //    bucket[k] <- first output slot of count k (descending counts)
+  // 4. longest-first stable row order
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    for (int k = max_nkt; k >= 0; --k) {
-      const int h = bucket[k];
-      bucket[k] = acc;
-      acc += h;
-    }
+  block_stable_order_desc(n_rows, row_cnt, max_nkt, bucket, order);
+  if (pair_row == nullptr) return;
+
+  // 5. pairs: a row opens a pair when its tile index inside its group is even;
+  //    pair_row = first row (bit-inverted when the pair has a single row)
+  auto opens = [&](int r) {
+    const GroupInfo g = groups[row_group[r]];
+    return ((r - g.row0) & 1) == 0 ? 1 : 0;
+  };
+  const int n_pairs = block_exclusive_scan(n_rows, opens, pair_idx, warp_sums, &carry);
+  for (int r = tid; r < n_rows; r += blockDim.x) {
+    const GroupInfo g = groups[row_group[r]];
+    if (((r - g.row0) & 1) != 0) continue;
+    const bool two = r + 1 < g.row0 + g.nqt;
+    const int pi = pair_idx[r];
+    pair_row[pi] = two ? r : ~r;
+    pair_cost[pi] = row_cnt[r] + (two ? row_cnt[r + 1] : 0);
   }
   __syncthreads();
-  //    rows are placed chunk by chunk, warp by warp, so equal counts keep row order
-  for (int base = 0; base < n_rows; base += blockDim.x) {
-    const int r = base + tid;
-    const int key = r < n_rows ? row_cnt[r] : -1;
-    const uint32_t same = __match_any_sync(0xffffffffu, key);
-    const int rank = __popc(same & lt_mask);
-    const bool leader = rank == 0;
-    for (int w = 0; w < nw; ++w) {
-      if (warp == w && key >= 0) {
-        const int slot = bucket[key] + rank;
-        order[slot] = r;
-      }
-      __syncthreads();
-      if (warp == w && key >= 0 && leader) bucket[key] += __popc(same);
-      __syncthreads();
-    }
-  }
+  block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
 }
 
 // ----------------------------------------------------------------------------
@@ -452,14 +493,16 @@ cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, i
 
 cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
-                        int32_t* order, cudaStream_t s) {
-  const size_t smem = sizeof(int32_t) * static_cast<size_t>(max_nkt + 1);
+                        int32_t* order, cudaStream_t s, int32_t* pair_row, int32_t* pair_cost,
+                        int32_t* pair_order, int32_t* pair_idx) {
+  const size_t smem = sizeof(int32_t) * static_cast<size_t>(2 * max_nkt + 1);
   if (smem > 48 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order);
+  k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order,
+                               pair_row, pair_cost, pair_order, pair_idx);
   return cudaGetLastError();
 }
 

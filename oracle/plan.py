@@ -17,6 +17,10 @@ Readings fixed here (the pages leave them open):
 * the key-tile list of a row is ascending;
 * the work order of rows is longest-first: a stable sort on (-count, row index),
   count = number of non-empty tiles of the row;
+* work pairs: inside each group, query tiles (2i, 2i+1) form one pair (the last
+  tile alone when the group has an odd number); pairs are listed group by group,
+  stored as their first row (bit-inverted, ~row, for a single-row pair), and
+  ordered longest-first by the pair's total listed tiles, ties by pair index;
 * a plan over several groups (batches, sequences, or BSR head groups) is the
   concatenation of the groups' rows in group order.
 
@@ -92,6 +96,15 @@ def plan_masks(masks, BM=128, BN=128):
         parts += rp
         fines += fn
     counts = np.array([len(x) for x in lists], dtype=np.int32)
+    pair_row, pair_cost = [], []
+    r0 = 0
+    for cls in cls_all:
+        nqt = cls.shape[0]
+        for i in range(0, nqt, 2):
+            two = i + 1 < nqt
+            pair_row.append(r0 + i if two else ~(r0 + i))
+            pair_cost.append(int(counts[r0 + i]) + (int(counts[r0 + i + 1]) if two else 0))
+        r0 += nqt
     row_ptr = np.zeros(len(lists) + 1, dtype=np.int32)
     row_ptr[1:] = np.cumsum(counts)
     kv_tile = np.concatenate(lists).astype(np.int32) if lists else np.zeros(0, np.int32)
@@ -106,6 +119,8 @@ def plan_masks(masks, BM=128, BN=128):
         "fine": fine,
         "counts": counts,
         "order": lpt_order(counts),
+        "pair_row": np.array(pair_row, dtype=np.int32),
+        "pair_order": lpt_order(pair_cost),
     }
 
 

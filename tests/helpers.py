@@ -30,6 +30,9 @@ def assert_plan_equal(got, ref):
     np.testing.assert_array_equal(got["classes"], ref_cls, err_msg="classes")
     if "fine" in got:
         np.testing.assert_array_equal(got["fine"], ref["fine"], err_msg="fine words")
+    if "pair_row" in got:
+        np.testing.assert_array_equal(got["pair_row"], ref["pair_row"], err_msg="pair rows")
+        np.testing.assert_array_equal(got["pair_order"], ref["pair_order"], err_msg="pair order")
 
 
 def compare_rows(O_gpu, L_gpu, O_ref, L_ref, where=""):
