@@ -10,7 +10,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     src = open(os.path.join(ROOT, "include", "bfa.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(bfa_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(bfa_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_north_star_calls():
