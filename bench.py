@@ -42,6 +42,24 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def _fwd_traffic():
+    """DRAM bytes per launch of the forward from the committed ncu record, or None
+    when the kernel sources have changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "bfa_fwd_kernel_causal_8192.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for name in rec["source_files"]:
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+    except Exception:
+        return None
+
+
 def _attended_flops(N, D, BH):
     nnz = N * (N + 1) // 2
     return 4.0 * D * nnz * BH, nnz
@@ -263,6 +281,8 @@ def run_bfa(args, rank, world, local_rank):
 
     peaks, src = _peaks()
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
+    # bytes the forward must move at least: read q, k, v once, write out and lse
+    algo_bytes = 3 * q.numel() * q.element_size() + out.numel() * out.element_size() + lse.numel() * 4
     peak = peaks["bf16_tflops"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -275,7 +295,8 @@ def run_bfa(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "bfa_fwd_kernel<128>", "achieved": fwd_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": fwd_tflops / peak, "peak_source": f"{src} bf16_tflops (burst)",
                      "frac_of_sustained": fwd_tflops / peaks.get("bf16_tflops_sustained", peak),
-                     "traffic": None},
+                     "traffic": _fwd_traffic(), "traffic_unit": "bytes per launch (ncu dram read + write)",
+                     "algorithmic_bytes": algo_bytes},
         "fwd_ms": fwd_ms, "plan_ms": plan_ms,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
