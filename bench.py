@@ -60,6 +60,21 @@ def _fwd_traffic():
         return None
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank timings (the job time is the slowest rank's)."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(flops_per_rank, world, ms_per_step):
+    """Weak scaling: every rank processes its own batch; value = all ranks' FLOPs / max time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def _attended_flops(N, D, BH):
     nnz = N * (N + 1) // 2
     return 4.0 * D * nnz * BH, nnz
@@ -234,12 +249,9 @@ def run_bfa(args, rank, world, local_rank):
     ms = t_start.elapsed_time(t_end)
     fwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     plan_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms, fwd_ms, plan_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, fwd_ms, plan_ms = t.tolist()
+    ms, fwd_ms, plan_ms = max_over_ranks([ms, fwd_ms, plan_ms], dist, dev)
     ms_per_step = ms / args.steps
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms_per_step)
 
     # end to end through the public API with host buffers: H2D of q/k/v/mask from
     # pinned memory, plan + forward, D2H of out and lse, every step
@@ -272,12 +284,8 @@ def run_bfa(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dist, dev)[0]
+    e2e_value = whole_job_tflops(flops, world, e2e_ms)
 
     peaks, src = _peaks()
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
