@@ -86,6 +86,7 @@ typedef struct bfa_plan_info {
   int32_t window_left;    /* -1: no window                                                        */
   int32_t causal;         /* positional / BSR plans: 1 if kv_idx <= q_idx is applied             */
   int32_t n_pairs;        /* work pairs: consecutive query tiles (2i, 2i+1) of one group          */
+  int32_t packed_fine;    /* 1: partial tiles carry packed fine masks (bfa_plan_export fills fine) */
 } bfa_plan_info;
 
 /* Library version string. */
@@ -149,21 +150,40 @@ bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const u
                              bfa_plan** out, void* stream);
 
 /*
- * Plan from BSR routing (flashinfer block_sparse_attention).
+ * Plan from BSR routing (flashinfer block_sparse_attention, sparse_format "bsr").
  *   indptr [B, Hkv, ceil(Sq/q_block)+1] i32: absolute offsets into indices, each
  *   (b, hkv) slice non-decreasing; indices [n_indices] i32: KV block ids, each
  *   row strictly increasing in [0, ceil(Skv/kv_block)).
- *   q_block == kv_block == 128 (BFA_TILE) in this build.
+ *   q_block >= 1 query tokens per BSR row; kv_block in {8, 16, 32} or a positive
+ *   multiple of 64 key tokens per block id (the page's allowed sizes).
  *   causal != 0 applies kv_idx <= q_idx on absolute positions inside the selected
- *   blocks (mask_type "causal"): blocks below the diagonal become full, blocks on
- *   it partial, blocks above it are dropped.
+ *   blocks (mask_type "causal"); otherwise every pair of a selected block attends.
+ *   kv_valid_bits [B, ceil(Skv/32)] u32 or NULL: bit j % 32 of word j / 32 of row b
+ *   marks key token j of batch b valid (kv_valid_bits); invalid keys never attend.
  * Query head h uses the routing of kv head h / (H / Hkv).
- * Validation runs on the device and is read back synchronously (one sync), like
- * the page's plan step; non-canonical rows give BFA_ERR_NONCANONICAL_BSR.
+ * 128 x 128 blocks without validity bits map BSR rows onto tile rows directly
+ * (blocks below the diagonal full, on it partial, above it dropped, masked by
+ * position in the kernel); any other shape is reduced to tile classes plus packed
+ * fine masks for the partial tiles.  Validation runs on the device and is read
+ * back synchronously, like the page's plan step (one or two syncs); non-canonical
+ * rows give BFA_ERR_NONCANONICAL_BSR.
  */
 bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
-                        int Sq, int Skv, int q_block, int kv_block, int causal, bfa_plan** out,
-                        void* stream);
+                        int Sq, int Skv, int q_block, int kv_block, int causal, const uint32_t* kv_valid_bits,
+                        bfa_plan** out, void* stream);
+
+/*
+ * Plan from an exact-block bitmap (flashinfer block_sparse_attention,
+ * sparse_format "bitmask", exact_block_bits).
+ *   block_bits [B, Hkv, ceil(Sq/q_block), ceil(nkb/32)] u32 with
+ *   nkb = ceil(Skv/kv_block): bit j % 32 of word j / 32 of row (b, hkv, i) selects
+ *   KV block j for query block i (LSB first).  q_block, kv_block, causal and
+ *   kv_valid_bits as for bfa_plan_bsr.  The structural KV-block count is the
+ *   capacity bound.  Reads the plan size back once (one sync).
+ */
+bfa_status bfa_plan_block_bits(const uint32_t* block_bits, int B, int Hkv, int Sq, int Skv, int q_block,
+                               int kv_block, int causal, const uint32_t* kv_valid_bits, bfa_plan** out,
+                               void* stream);
 
 /*
  * Fused masked attention forward with a prebuilt plan.
@@ -196,8 +216,8 @@ bfa_status bfa_plan_stats(const bfa_plan* plan, int64_t* n_full, int64_t* n_part
 /*
  * Copy a plan to HOST buffers (for parity checks); synchronises `stream`.
  * Sizes: row_ptr [n_rows + 1], kv_tile / partial [n_full + n_partial],
- * fine [n_partial * 512] uint32 (dense plans; partial tiles in list order, 128
- * rows x 4 words each) or NULL, order [n_rows] (longest row first, ties by row
+ * fine [n_partial * 512] uint32 (plans with packed_fine; partial tiles in list
+ * order, 128 rows x 4 words each) or NULL, order [n_rows] (longest row first, ties by row
  * index), classes [grid_tiles] (0 empty, 1 partial, 2 full; groups in order,
  * each group row-major over (query tile, key tile)).  Any pointer may be NULL.
  */

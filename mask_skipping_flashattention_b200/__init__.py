@@ -23,7 +23,8 @@ import torch
 from . import _lib
 from ._lib import BfaError, PlanInfo
 
-__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_bsr", "fwd", "make_att_block_ids",
+__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_bsr", "plan_block_bits", "fwd",
+           "make_att_block_ids",
            "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "library_path"]
 
 TILE = 128
@@ -112,14 +113,14 @@ class Plan:
         _lib.check(_L.bfa_plan_device_status(self.handle, _stream(stream)))
 
     def export(self, stream=None):
-        """Host copy: row_ptr, kv_tile, partial, fine (dense plans), order, classes."""
+        """Host copy: row_ptr, kv_tile, partial, fine (packed-mask plans), order, classes, pairs."""
         n_full, n_part, _ = self.stats(stream)
         R = self.info["n_rows"]
         nnz = n_full + n_part
         row_ptr = np.zeros(R + 1, np.int32)
         kv_tile = np.zeros(max(nnz, 1), np.int32)
         partial = np.zeros(max(nnz, 1), np.uint8)
-        fine = np.zeros((max(n_part, 1), TILE, 4), np.uint32) if self.kind == "dense" else None
+        fine = np.zeros((max(n_part, 1), TILE, 4), np.uint32) if self.info["packed_fine"] else None
         order = np.zeros(max(R, 1), np.int32)
         classes = np.zeros(max(self.info["grid_tiles"], 1), np.uint8)
         P = lambda a: a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
@@ -208,15 +209,33 @@ def plan_blockids(q_blk=None, k_blk=None, q_valid=None, k_valid=None, *, B=None,
 
 
 def plan_bsr(block_indptr, block_indices, Sq, Skv, q_block_size=TILE, kv_block_size=TILE, causal=False,
-             stream=None):
-    """Plan from BSR routing: indptr (B, Hkv, ceil(Sq/q_block)+1) int32, indices int32."""
+             kv_valid_bits=None, stream=None):
+    """Plan from BSR routing: indptr (B, Hkv, ceil(Sq/q_block)+1) int32, indices int32.
+
+    ``kv_valid_bits`` (B, ceil(Skv/32)) int32/uint32 marks valid key tokens, LSB first.
+    """
     ip = block_indptr.to(torch.int32).contiguous()
     ix = block_indices.to(torch.int32).contiguous()
+    kv = kv_valid_bits.contiguous() if kv_valid_bits is not None else None
     B, Hkv, _ = ip.shape
     h = ctypes.c_void_p()
     st = _stream(stream)
     _lib.check(_L.bfa_plan_bsr(_ptr(ip), _ptr(ix) if ix.numel() else None, ix.numel(), B, Hkv, int(Sq), int(Skv),
-                               int(q_block_size), int(kv_block_size), 1 if causal else 0, ctypes.byref(h), st))
+                               int(q_block_size), int(kv_block_size), 1 if causal else 0, _ptr(kv),
+                               ctypes.byref(h), st))
+    return Plan(h, st)
+
+
+def plan_block_bits(exact_block_bits, Sq, Skv, q_block_size=TILE, kv_block_size=TILE, causal=False,
+                    kv_valid_bits=None, stream=None):
+    """Plan from an exact-block bitmap (B, Hkv, ceil(Sq/q_block), ceil(nkb/32)), LSB first."""
+    bits = exact_block_bits.contiguous()
+    kv = kv_valid_bits.contiguous() if kv_valid_bits is not None else None
+    B, Hkv = bits.shape[:2]
+    h = ctypes.c_void_p()
+    st = _stream(stream)
+    _lib.check(_L.bfa_plan_block_bits(_ptr(bits), B, Hkv, int(Sq), int(Skv), int(q_block_size), int(kv_block_size),
+                                      1 if causal else 0, _ptr(kv), ctypes.byref(h), st))
     return Plan(h, st)
 
 

@@ -34,7 +34,16 @@ cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, i
 cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row = nullptr, int32_t* pair_cost = nullptr,
-                        int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr);
+                        int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr, int part_is_pos = 0);
+cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int n_groups,
+                               int nqb, int nkb, int wpr, uint32_t* bits, uint32_t* err, cudaStream_t s);
+cudaError_t launch_bits_classify(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
+                                 int q_block, int kv_block, int causal, const GroupInfo* groups, int n_groups,
+                                 int nqt, uint8_t* cls, cudaStream_t s);
+cudaError_t launch_bits_fine(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
+                             int q_block, int kv_block, int causal, const GroupInfo* groups, const int32_t* row_group,
+                             int n_rows, const int32_t* row_ptr, const int32_t* kv_tile, const int32_t* part,
+                             uint32_t* fine, cudaStream_t s);
 cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
                                   const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
                                   uint8_t* k_valid, cudaStream_t s);
@@ -53,6 +62,8 @@ struct bfa_plan {
   int kind = 0, varlen = 0, batch = 0, hkv = 0, sq = 0, sk = 0, window = -1, causal = 0;
   int n_groups = 0, n_rows = 0, n_pairs = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
   int64_t grid_tiles = 0;
+  int64_t fine_tiles = 0;       // tiles of packed fine words held in `fine`
+  void* fine_extra = nullptr;   // separately allocated fine words (generic block sparsity)
   bool regular = false;   // every group the same shape: the group table is built on the device
   int regular_hkv = 1;    // groups per batch of a regular layout (BSR: Hkv)
   bool copy_ids = false;
@@ -243,12 +254,13 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
 
 void free_plan(bfa_plan* P) {
   if (!P) return;
+  if (P->fine_extra) cudaFreeAsync(P->fine_extra, P->stream);
   if (P->slab) cudaFreeAsync(P->slab, P->stream);
   delete P;
 }
 
 // Finish the plan: groups laid out, classes written -> lists and order.
-bfa_status build_rows(bfa_plan* P) {
+bfa_status build_rows(bfa_plan* P, int part_is_pos = 0) {
   if (P->n_rows == 0) {
     cudaError_t e = cudaMemsetAsync(P->row_ptr, 0, sizeof(int32_t), P->stream);
     return e == cudaSuccess ? BFA_OK : cuda_fail(e, "empty plan");
@@ -256,7 +268,7 @@ bfa_status build_rows(bfa_plan* P) {
   if (P->max_nkt > kMaxKvTiles) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
   cudaError_t e = launch_rows(P->groups, P->row_group, P->cls, P->n_rows, P->max_nkt, P->row_cnt, P->row_ptr,
                               P->kv_tile, P->part, P->order, P->stream, P->pair_row, P->pair_cost,
-                              P->pair_order, P->pair_idx);
+                              P->pair_order, P->pair_idx, part_is_pos);
   return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
 }
 
@@ -371,6 +383,7 @@ BFA_API bfa_status bfa_plan_dense(const uint8_t* mask, int64_t ld, int Sq, int S
   finalize_layout(P);
   if ((s = check_capacity(P, true))) { cleanup(); return s; }
   if ((s = alloc_plan(P, true, 0, 0, 0))) { cleanup(); return s; }
+  P->fine_tiles = P->grid_tiles;
   BFA_CUDA(launch_dense_classify(mask, ld, Sq, Sk, P->cls, P->fine, P->stream), "dense classify kernel");
   if ((s = build_rows(P))) { cleanup(); return s; }
   *out = P;
@@ -463,21 +476,110 @@ BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk,
   return BFA_OK;
 }
 
+namespace {
+
+bool kv_block_ok(int kv_block) { return kv_block == 8 || kv_block == 16 || kv_block == 32 || (kv_block > 0 && kv_block % 64 == 0); }
+
+// Block sparsity of any block size (flashinfer block_sparse_attention: BSR rows or
+// an exact-block bitmap, key validity bits, dense or causal inside the blocks),
+// reduced to tile classes plus packed fine words for the partial tiles.
+bfa_status plan_block_sparse(const int32_t* indptr, const int32_t* indices, int64_t n_indices,
+                             const uint32_t* block_bits, const uint32_t* kv_valid, int B, int Hkv, int Sq, int Skv,
+                             int q_block, int kv_block, int causal, bfa_plan** out, cudaStream_t st) {
+  bfa_plan* P = new bfa_plan();
+  uint32_t* tmp_bits = nullptr;
+  auto cleanup = [&]() {
+    if (tmp_bits) cudaFreeAsync(tmp_bits, st);
+    free_plan(P);
+  };
+  bfa_status s;
+  P->kind = BFA_PLAN_BSR;
+  P->mask_mode = MASK_BITS;
+  P->causal = causal ? 1 : 0;
+  P->window = -1;
+  P->batch = B;
+  P->hkv = Hkv;
+  P->sq = Sq;
+  P->sk = Skv;
+  P->stream = st;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hkv; ++h) P->groups_h.push_back(make_group(0, Sq, 0, Skv, b, h));
+  P->regular = true;
+  P->regular_hkv = Hkv;
+  finalize_layout(P);
+  if ((s = check_capacity(P, false))) { cleanup(); return s; }
+  if ((s = alloc_plan(P, false, 0, 0, 0))) { cleanup(); return s; }
+  const int nqb = cdiv(Sq, q_block), nkb = cdiv(Skv, kv_block), wpr = cdiv(nkb, 32), kv_wpb = cdiv(Skv, 32);
+  const int G = B * Hkv;
+  const uint32_t* bits = block_bits;
+  if (!bits) {  // BSR rows -> bitmap, validated on the device and read back once
+    cudaMemPool_t pool;
+    BFA_CUDA(plan_pool(&pool), "plan memory pool");
+    const size_t nb = sizeof(uint32_t) * static_cast<size_t>(G) * nqb * wpr;
+    BFA_CUDA(cudaMallocFromPoolAsync(reinterpret_cast<void**>(&tmp_bits), std::max<size_t>(nb, 4), pool, st),
+             "block bitmap");
+    BFA_CUDA(cudaMemsetAsync(tmp_bits, 0, std::max<size_t>(nb, 4), st), "clear block bitmap");
+    BFA_CUDA(launch_bsr_to_bits(indptr, indices, n_indices, G, nqb, nkb, wpr, tmp_bits, P->err, st),
+             "BSR bitmap kernel");
+    uint32_t err = 0;
+    BFA_CUDA(cudaMemcpyAsync(&err, P->err, sizeof(err), cudaMemcpyDeviceToHost, st), "read BSR status");
+    BFA_CUDA(cudaStreamSynchronize(st), "BSR validation");
+    if (err) {
+      cleanup();
+      return fail(BFA_ERR_NONCANONICAL_BSR, "BSR routing is not canonical (%s)",
+                  (err & DEVERR_BSR_RANGE) ? "row offsets out of range or decreasing"
+                                            : "block ids unsorted, duplicated or out of range");
+    }
+    bits = tmp_bits;
+  }
+  BFA_CUDA(launch_bits_classify(bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, P->causal, P->groups,
+                                P->n_groups, P->max_nqt, P->cls, st),
+           "block-sparse classify kernel");
+  if ((s = build_rows(P, 1))) { cleanup(); return s; }
+  int32_t nnz = 0;
+  BFA_CUDA(cudaMemcpyAsync(&nnz, P->row_ptr + P->n_rows, sizeof(int32_t), cudaMemcpyDeviceToHost, st), "read size");
+  BFA_CUDA(cudaStreamSynchronize(st), "plan size");
+  cudaMemPool_t pool;
+  BFA_CUDA(plan_pool(&pool), "plan memory pool");
+  BFA_CUDA(cudaMallocFromPoolAsync(&P->fine_extra,
+                                   sizeof(uint32_t) * kFineWordsPerTile * static_cast<size_t>(std::max(nnz, 1)),
+                                   pool, st),
+           "fine-mask allocation");
+  P->fine = static_cast<uint32_t*>(P->fine_extra);
+  P->fine_tiles = nnz;
+  BFA_CUDA(launch_bits_fine(bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, P->causal, P->groups, P->row_group,
+                            P->n_rows, P->row_ptr, P->kv_tile, P->part, P->fine, st),
+           "block-sparse fine-mask kernel");
+  if (tmp_bits) {
+    cudaFreeAsync(tmp_bits, st);
+    tmp_bits = nullptr;
+  }
+  *out = P;
+  return BFA_OK;
+}
+
+}  // namespace
+
 BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
-                                int Sq, int Skv, int q_block, int kv_block, int causal, bfa_plan** out,
-                                void* stream) {
+                                int Sq, int Skv, int q_block, int kv_block, int causal, const uint32_t* kv_valid_bits,
+                                bfa_plan** out, void* stream) {
   if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (B <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || n_indices < 0)
     return fail(BFA_ERR_INVALID_ARG, "bad sizes B=%d Hkv=%d Sq=%d Skv=%d n_indices=%lld", B, Hkv, Sq, Skv,
                 (long long)n_indices);
-  if (q_block != kTile || kv_block != kTile)
-    return fail(BFA_ERR_UNSUPPORTED, "q_block=%d kv_block=%d: this build needs both equal to %d", q_block, kv_block,
-                kTile);
+  if (q_block <= 0) return fail(BFA_ERR_INVALID_ARG, "q_block=%d must be positive", q_block);
+  if (!kv_block_ok(kv_block))
+    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d must be 8, 16, 32 or a positive multiple of 64", kv_block);
   bfa_status s;
   if ((s = need_device(indptr, "block_indptr"))) return s;
   if (n_indices > 0 && (s = need_device(indices, "block_indices"))) return s;
+  if ((s = need_device(kv_valid_bits, "kv_valid_bits", true))) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (q_block != kTile || kv_block != kTile || kv_valid_bits != nullptr)
+    return plan_block_sparse(indptr, indices, n_indices, nullptr, kv_valid_bits, B, Hkv, Sq, Skv, q_block, kv_block,
+                             causal, out, st);
+  // 128 x 128 blocks: BSR rows are tile rows; causal blocks are classified by position
   bfa_plan* P = new bfa_plan();
   auto cleanup = [&]() { free_plan(P); };
   P->kind = BFA_PLAN_BSR;
@@ -512,6 +614,23 @@ BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, i
   if ((s = build_rows(P))) { cleanup(); return s; }
   *out = P;
   return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_block_bits(const uint32_t* block_bits, int B, int Hkv, int Sq, int Skv, int q_block,
+                                       int kv_block, int causal, const uint32_t* kv_valid_bits, bfa_plan** out,
+                                       void* stream) {
+  if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (B <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0)
+    return fail(BFA_ERR_INVALID_ARG, "bad sizes B=%d Hkv=%d Sq=%d Skv=%d", B, Hkv, Sq, Skv);
+  if (q_block <= 0) return fail(BFA_ERR_INVALID_ARG, "q_block=%d must be positive", q_block);
+  if (!kv_block_ok(kv_block))
+    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d must be 8, 16, 32 or a positive multiple of 64", kv_block);
+  bfa_status s;
+  if ((s = need_device(block_bits, "exact_block_bits")) || (s = need_device(kv_valid_bits, "kv_valid_bits", true)))
+    return s;
+  return plan_block_sparse(nullptr, nullptr, 0, block_bits, kv_valid_bits, B, Hkv, Sq, Skv, q_block, kv_block, causal,
+                           out, static_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------------
@@ -699,6 +818,7 @@ BFA_API bfa_status bfa_plan_get_info(const bfa_plan* P, bfa_plan_info* info) {
   info->window_left = P->window;
   info->causal = P->causal;
   info->n_pairs = P->n_pairs;
+  info->packed_fine = P->mask_mode == MASK_BITS ? 1 : 0;
   return BFA_OK;
 }
 
@@ -739,9 +859,9 @@ BFA_API bfa_status bfa_plan_export(const bfa_plan* P, int32_t* row_ptr, int32_t*
   if (classes && P->grid_tiles > 0)
     BFA_CUDA(cudaMemcpyAsync(classes, P->cls, static_cast<size_t>(P->grid_tiles), cudaMemcpyDeviceToHost, st), "read classes");
   std::vector<uint32_t> fine_all;
-  const bool want_fine = fine && P->mask_mode == MASK_BITS && P->grid_tiles > 0;
+  const bool want_fine = fine && P->mask_mode == MASK_BITS && P->fine_tiles > 0;
   if (want_fine) {
-    fine_all.resize(static_cast<size_t>(P->grid_tiles) * kFineWordsPerTile);
+    fine_all.resize(static_cast<size_t>(P->fine_tiles) * kFineWordsPerTile);
     BFA_CUDA(cudaMemcpyAsync(fine_all.data(), P->fine, fine_all.size() * sizeof(uint32_t), cudaMemcpyDeviceToHost, st),
              "read fine masks");
   }

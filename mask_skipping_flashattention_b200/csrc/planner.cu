@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
                                                int32_t* __restrict__ kv_tile, int32_t* __restrict__ part,
                                                int32_t* __restrict__ order, int32_t* __restrict__ pair_row,
                                                int32_t* __restrict__ pair_cost, int32_t* __restrict__ pair_order,
-                                               int32_t* __restrict__ pair_idx) {
+                                               int32_t* __restrict__ pair_idx, int part_is_pos) {
   extern __shared__ int32_t bucket[];
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
       if (klass != 0) {
         const int pos = out + __popc(bal & lt_mask);
         kv_tile[pos] = kt;
-        part[pos] = (klass == 1) ? static_cast<int32_t>(rowoff + kt) : -1;
+        part[pos] = (klass == 1) ? (part_is_pos ? pos : static_cast<int32_t>(rowoff + kt)) : -1;
       }
       out += __popc(bal);
     }
@@ -364,6 +364,134 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
   }
   __syncthreads();
   block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
+}
+
+// ----------------------------------------------------------------------------
+// generic block sparsity (any BSR block sizes, exact-block bitmaps, key validity)
+// ----------------------------------------------------------------------------
+// Block bitmap layout: [group][query block][wpr words], bit kb % 32 of word
+// kb / 32 selects KV block kb.
+
+// BSR rows -> block bitmap, validating canonical rows (one thread per row).
+__global__ void k_bsr_to_bits(const int32_t* __restrict__ indptr, const int32_t* __restrict__ indices,
+                              int64_t n_indices, int n_groups, int nqb, int nkb, int wpr, uint32_t* __restrict__ bits,
+                              uint32_t* err) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= static_cast<int64_t>(n_groups) * nqb) return;
+  const int grp = static_cast<int>(gid / nqb), qb = static_cast<int>(gid % nqb);
+  const int32_t* ip = indptr + static_cast<int64_t>(grp) * (nqb + 1);
+  const int32_t a = ip[qb], b = ip[qb + 1];
+  if (a < 0 || b < a || static_cast<int64_t>(b) > n_indices) {
+    atomicOr(err, DEVERR_BSR_RANGE);
+    return;
+  }
+  uint32_t* row = bits + gid * wpr;
+  int32_t prev = -1;
+  for (int32_t e = a; e < b; ++e) {
+    const int32_t kb = indices[e];
+    if (kb <= prev || kb >= nkb) {
+      atomicOr(err, DEVERR_BSR_ORDER);
+      return;
+    }
+    prev = kb;
+    row[kb >> 5] |= 1u << (kb & 31);
+  }
+}
+
+struct BlockSparseArgs {
+  const uint32_t* bits;      // block bitmap [group][nqb][wpr]
+  const uint32_t* kv_valid;  // [batch][kv_wpb] token validity bits, or null
+  int nqb, wpr, kv_wpb;
+  int q_block, kv_block, causal;
+};
+
+// attend-bits of query position i (row of query block qb) over the 32 columns
+// starting at c0 (a multiple of 32) of a group with k_len keys
+__device__ __forceinline__ uint32_t block_word(const BlockSparseArgs& a, const uint32_t* rowbits,
+                                               const uint32_t* kvrow, int i, int c0, int k_len) {
+  if (c0 >= k_len) return 0u;
+  uint32_t w;
+  if (a.kv_block % 32 == 0) {  // the 32 columns lie in one KV block
+    const int kb = c0 / a.kv_block;
+    w = ((rowbits[kb >> 5] >> (kb & 31)) & 1u) ? 0xffffffffu : 0u;
+  } else {                     // kv_block in {8, 16}: several blocks per word
+    w = 0u;
+    const uint32_t run = (1u << a.kv_block) - 1u;
+    for (int c = 0; c < 32 && c0 + c < k_len; c += a.kv_block) {  // blocks past the end are never read
+      const int kb = (c0 + c) / a.kv_block;
+      if ((rowbits[kb >> 5] >> (kb & 31)) & 1u) w |= run << c;
+    }
+  }
+  const int ncols = k_len - c0;
+  if (ncols < 32) w &= (1u << ncols) - 1u;
+  if (a.causal) {  // keep columns c0 + c <= i
+    const int z = i - c0;
+    w &= (z >= 31) ? 0xffffffffu : (z < 0 ? 0u : ((2u << z) - 1u));
+  }
+  if (kvrow) w &= kvrow[c0 >> 5];
+  return w;
+}
+
+// Tile classes from the block bitmap: CTA per (group, query tile), thread per row.
+__global__ void __launch_bounds__(128) k_bits_classify(BlockSparseArgs a, const GroupInfo* __restrict__ groups,
+                                                       uint8_t* __restrict__ cls) {
+  __shared__ int warp_cnt[4];
+  const GroupInfo g = groups[blockIdx.x];
+  const int qt = blockIdx.y;
+  if (qt >= g.nqt) return;
+  const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+  const int i = qt * kTile + r;
+  const bool in = i < g.q_len;
+  const uint32_t* rowbits = a.bits + (static_cast<int64_t>(blockIdx.x) * a.nqb + (in ? i / a.q_block : 0)) * a.wpr;
+  const uint32_t* kvrow = a.kv_valid ? a.kv_valid + static_cast<int64_t>(g.b) * a.kv_wpb : nullptr;
+  const int rows_in = min(kTile, g.q_len - qt * kTile);
+  for (int kt = 0; kt < g.nkt; ++kt) {
+    int cnt = 0;
+    if (in) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) cnt += __popc(block_word(a, rowbits, kvrow, i, kt * kTile + 32 * w, g.k_len));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) warp_cnt[warp] = cnt;
+    __syncthreads();
+    if (r == 0) {
+      const int c = warp_cnt[0] + warp_cnt[1] + warp_cnt[2] + warp_cnt[3];
+      const int n_in = rows_in * min(kTile, g.k_len - kt * kTile);
+      cls[g.cls_off + static_cast<int64_t>(qt) * g.nkt + kt] = static_cast<uint8_t>(c == 0 ? 0 : (c == n_in ? 2 : 1));
+    }
+    __syncthreads();
+  }
+}
+
+// Packed fine words of every partial listed tile, stored at its list position
+// (CTA per plan row, thread per tile row).
+__global__ void __launch_bounds__(128) k_bits_fine(BlockSparseArgs a, const GroupInfo* __restrict__ groups,
+                                                   const int32_t* __restrict__ row_group,
+                                                   const int32_t* __restrict__ row_ptr,
+                                                   const int32_t* __restrict__ kv_tile,
+                                                   const int32_t* __restrict__ part, uint32_t* __restrict__ fine) {
+  const int row = blockIdx.x;
+  const int grp = row_group[row];
+  const GroupInfo g = groups[grp];
+  const int qt = row - g.row0, r = threadIdx.x;
+  const int i = qt * kTile + r;
+  const bool in = i < g.q_len;
+  const uint32_t* rowbits = a.bits + (static_cast<int64_t>(grp) * a.nqb + (in ? i / a.q_block : 0)) * a.wpr;
+  const uint32_t* kvrow = a.kv_valid ? a.kv_valid + static_cast<int64_t>(g.b) * a.kv_wpb : nullptr;
+  for (int e = row_ptr[row]; e < row_ptr[row + 1]; ++e) {
+    const int slot = part[e];
+    if (slot < 0) continue;
+    const int kt = kv_tile[e];
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (in) {
+      w.x = block_word(a, rowbits, kvrow, i, kt * kTile + 0, g.k_len);
+      w.y = block_word(a, rowbits, kvrow, i, kt * kTile + 32, g.k_len);
+      w.z = block_word(a, rowbits, kvrow, i, kt * kTile + 64, g.k_len);
+      w.w = block_word(a, rowbits, kvrow, i, kt * kTile + 96, g.k_len);
+    }
+    reinterpret_cast<uint4*>(fine + static_cast<int64_t>(slot) * kFineWordsPerTile)[r] = w;
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -494,7 +622,7 @@ cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, i
 cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row, int32_t* pair_cost,
-                        int32_t* pair_order, int32_t* pair_idx) {
+                        int32_t* pair_order, int32_t* pair_idx, int part_is_pos) {
   const size_t smem = sizeof(int32_t) * static_cast<size_t>(2 * max_nkt + 1);
   if (smem > 48 * 1024) {
     cudaError_t e =
@@ -502,7 +630,35 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
     if (e != cudaSuccess) return e;
   }
   k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order,
-                               pair_row, pair_cost, pair_order, pair_idx);
+                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int n_groups,
+                               int nqb, int nkb, int wpr, uint32_t* bits, uint32_t* err, cudaStream_t s) {
+  const int64_t n = static_cast<int64_t>(n_groups) * nqb;
+  if (n <= 0) return cudaSuccess;
+  k_bsr_to_bits<<<static_cast<unsigned>((n + 127) / 128), 128, 0, s>>>(indptr, indices, n_indices, n_groups, nqb, nkb,
+                                                                        wpr, bits, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bits_classify(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
+                                 int q_block, int kv_block, int causal, const GroupInfo* groups, int n_groups,
+                                 int nqt, uint8_t* cls, cudaStream_t s) {
+  if (n_groups <= 0 || nqt <= 0) return cudaSuccess;
+  BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal};
+  k_bits_classify<<<dim3(n_groups, nqt), 128, 0, s>>>(a, groups, cls);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bits_fine(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
+                             int q_block, int kv_block, int causal, const GroupInfo* groups, const int32_t* row_group,
+                             int n_rows, const int32_t* row_ptr, const int32_t* kv_tile, const int32_t* part,
+                             uint32_t* fine, cudaStream_t s) {
+  if (n_rows <= 0) return cudaSuccess;
+  BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal};
+  k_bits_fine<<<n_rows, 128, 0, s>>>(a, groups, row_group, row_ptr, kv_tile, part, fine);
   return cudaGetLastError();
 }
 

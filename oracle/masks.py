@@ -164,6 +164,47 @@ def bsr_dense(block_indptr, block_indices, Sq, Skv, q_block_size, kv_block_size,
     return M
 
 
+def block_bits_dense(block_bits, Sq, Skv, q_block_size, kv_block_size, causal=False, kv_valid_bits=None):
+    """Expand an exact-block bitmap into (B, Hkv, Sq, Skv) bool (flashinfer
+    block_sparse_attention, ``sparse_format="bitmask"`` with ``exact_block_bits``).
+
+    Reading: ``block_bits`` is (B, Hkv, ceil(Sq/q_block_size), ceil(nkb/32)) uint32;
+    bit ``j`` of word ``w`` in row ``i`` selects KV block ``32 w + j`` for query block
+    ``i`` (least significant bit first).  ``kv_valid_bits`` (B, ceil(Skv/32)) uint32
+    marks valid key tokens the same way (``kv_valid_bits``); invalid keys are never
+    attended.  ``causal`` applies ``kv_idx <= q_idx`` (``mask_type``).
+    """
+    bits = np.asarray(block_bits, dtype=np.uint32)
+    B, H, nqb, _ = bits.shape
+    nkb = -(-Skv // kv_block_size)
+    sel = np.unpackbits(bits.view(np.uint8), axis=-1, bitorder="little").astype(bool)[..., :nkb]
+    rows = np.arange(Sq) // q_block_size
+    cols = np.arange(Skv) // kv_block_size
+    M = sel[:, :, rows][:, :, :, cols]
+    if causal:
+        M &= positional_dense(Sq, Skv, causal=True)[None, None]
+    if kv_valid_bits is not None:
+        kv = np.unpackbits(np.asarray(kv_valid_bits, dtype=np.uint32).view(np.uint8), axis=-1,
+                           bitorder="little").astype(bool)[:, :Skv]
+        M &= kv[:, None, None, :]
+    return M
+
+
+def bsr_to_block_bits(block_indptr, block_indices, n_kv_blocks):
+    """The exact-block bitmap of BSR routing (same selection, bitmask layout)."""
+    indptr = np.asarray(block_indptr, dtype=np.int64)
+    idx = np.asarray(block_indices, dtype=np.int64)
+    B, H, n1 = indptr.shape
+    words = -(-n_kv_blocks // 32)
+    out = np.zeros((B, H, n1 - 1, words), dtype=np.uint32)
+    for b in range(B):
+        for h in range(H):
+            for r in range(n1 - 1):
+                for kb in idx[indptr[b, h, r]:indptr[b, h, r + 1]]:
+                    out[b, h, r, kb // 32] |= np.uint32(1) << np.uint32(kb % 32)
+    return out
+
+
 def bsr_is_canonical(block_indptr, block_indices, n_kv_blocks):
     """Canonical BSR rows: offsets non-decreasing and inside the index array, and
     every row's ids strictly increasing inside [0, n_kv_blocks)

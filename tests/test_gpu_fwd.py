@@ -274,3 +274,21 @@ def test_bounded_wait_reports_timeout_and_context_survives():
         bfa.set_wait_timeout_ns(0)
     # the context is still usable
     test_default_scale_matches_explicit()
+
+
+@pytest.mark.parametrize("qb,kb,causal", [(64, 32, True), (100, 192, False)])
+def test_general_block_sparse_forward(qb, kb, causal):
+    from test_gpu_plan import _routing, _valid_bits
+    B, H, Hkv, Sq, Skv, D = 2, 4, 2, 300, 500, 128
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    indptr, indices = _routing(B, Hkv, nqb, nkb, 77 + qb)
+    kvb = _valid_bits(B, Skv, 5)
+    P = bfa.plan_bsr(_cuda(indptr), _cuda(indices), Sq, Skv, qb, kb, causal=causal,
+                     kv_valid_bits=_cuda(kvb.view(np.int32)))
+    q, k, v = _rand((B, Sq, H, D), 41), _rand((B, Skv, Hkv, D), 42), _rand((B, Skv, Hkv, D), 43)
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    M = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=causal,
+                            kv_valid_bits=kvb)
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M[b, h // (H // Hkv)], None, pairs, where="general bsr")

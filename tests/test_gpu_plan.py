@@ -2,7 +2,7 @@
 
 The oracle plan of any mask form is the plan of its dense mask (built by the
 oracle's own builders); the GPU planners get the compact forms (dense bytes,
-block ids, positions, BSR routing) through the C ABI.
+block ids, positions, BSR routing, exact-block bitmaps) through the C ABI.
 """
 
 import numpy as np
@@ -211,12 +211,67 @@ def test_bsr_noncanonical_rejected():
     with pytest.raises(bfa.BfaError) as e:
         bfa.plan_bsr(_cuda(np.array([[[0, 3, 2]]], np.int32)), _cuda(np.array([0, 1, 1], np.int32)), 256, 256)
     assert e.value.status == "BFA_ERR_NONCANONICAL_BSR"
-    with pytest.raises(bfa.BfaError) as e:
-        bfa.plan_bsr(_cuda(indptr), _cuda(np.array([0, 1, 1], np.int32)), 256, 256, q_block_size=64)
-    assert e.value.status == "BFA_ERR_UNSUPPORTED"
 
 
 def test_plan_rejects_host_memory():
     with pytest.raises(bfa.BfaError) as e:
         bfa.plan_dense(torch.ones(8, 8, dtype=torch.bool))
     assert e.value.status == "BFA_ERR_NOT_DEVICE"
+
+
+# ---------------------------------------------------------------- general block sparsity
+def _routing(B, H, nqb, nkb, seed, density=0.35):
+    rng = np.random.default_rng(seed)
+    indptr = np.zeros((B, H, nqb + 1), dtype=np.int32)
+    idx, pos = [], 0
+    for b in range(B):
+        for h in range(H):
+            indptr[b, h, 0] = pos
+            for r in range(nqb):
+                row = np.sort(rng.choice(nkb, size=int(rng.binomial(nkb, density)), replace=False))
+                idx.append(row)
+                pos += row.size
+                indptr[b, h, r + 1] = pos
+    return indptr, np.concatenate(idx).astype(np.int32)
+
+
+def _valid_bits(B, Skv, seed):
+    rng = np.random.default_rng(seed)
+    valid = rng.random((B, Skv)) < 0.9
+    words = -(-Skv // 32)
+    out = np.zeros((B, words), dtype=np.uint32)
+    for b in range(B):
+        for j in np.nonzero(valid[b])[0]:
+            out[b, j // 32] |= np.uint32(1) << np.uint32(j % 32)
+    return out
+
+
+@pytest.mark.parametrize("qb,kb,causal,valid", [
+    (64, 64, True, False), (32, 8, False, True), (100, 192, True, True), (128, 16, False, False),
+    (128, 128, True, True), (7, 32, True, False),
+])
+def test_general_block_sparse_plans(qb, kb, causal, valid):
+    B, H, Sq, Skv = 2, 2, 450, 600
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    indptr, indices = _routing(B, H, nqb, nkb, qb * 1000 + kb)
+    kvb = _valid_bits(B, Skv, kb) if valid else None
+    P = bfa.plan_bsr(_cuda(indptr), _cuda(indices), Sq, Skv, qb, kb, causal=causal,
+                     kv_valid_bits=_cuda(kvb.view(np.int32)) if valid else None)
+    assert P.info["packed_fine"] == 1
+    D = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=causal,
+                            kv_valid_bits=kvb)
+    ref = oracle_plan_for_groups([D[b, h] for b in range(B) for h in range(H)])
+    assert_plan_equal(P.export(), ref)
+    # the bitmask format selects the same mask
+    bits = om.bsr_to_block_bits(indptr, indices, nkb)
+    P2 = bfa.plan_block_bits(_cuda(bits.view(np.int32)), Sq, Skv, qb, kb, causal=causal,
+                             kv_valid_bits=_cuda(kvb.view(np.int32)) if valid else None)
+    assert_plan_equal(P2.export(), ref)
+
+
+def test_general_block_sparse_rejects_bad_blocks():
+    indptr, indices = _routing(1, 1, 4, 10, 3)
+    for kb in (0, 24, 48, 100):
+        with pytest.raises(bfa.BfaError) as e:
+            bfa.plan_bsr(_cuda(indptr), _cuda(indices), 256, 640, 64, kb)
+        assert e.value.status == "BFA_ERR_INVALID_ARG"

@@ -239,3 +239,41 @@ def test_bsr_canonical_checks():
     assert not om.bsr_is_canonical(indptr, np.array([0, 1, 2], np.int32), 2)       # out of range
     assert not om.bsr_is_canonical(np.array([[[0, 3, 2]]], np.int32), np.array([0, 1, 1], np.int32), 2)
     assert not om.bsr_is_canonical(np.array([[[0, 2, 4]]], np.int32), np.array([0, 1, 1], np.int32), 2)
+
+
+def _pack_bits(sel):
+    """bool (..., n) -> uint32 words LSB-first, written as an explicit loop."""
+    *lead, n = sel.shape
+    words = -(-n // 32)
+    out = np.zeros((*lead, words), dtype=np.uint32)
+    for idx in np.ndindex(*lead):
+        for j in range(n):
+            if sel[idx + (j,)]:
+                out[idx + (j // 32,)] |= np.uint32(1) << np.uint32(j % 32)
+    return out
+
+
+@pytest.mark.parametrize("qb,kb,causal", [(4, 8, False), (3, 5, True), (16, 16, True)])
+def test_block_bits_expand_matches_brute_force(qb, kb, causal):
+    rng = np.random.default_rng(qb * 10 + kb)
+    B, H, Sq, Skv = 2, 2, 37, 45
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    sel = rng.random((B, H, nqb, nkb)) < 0.4
+    valid = rng.random((B, Skv)) < 0.8
+    got = om.block_bits_dense(_pack_bits(sel), Sq, Skv, qb, kb, causal=causal, kv_valid_bits=_pack_bits(valid))
+    ref = np.zeros((B, H, Sq, Skv), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Sq):
+                for j in range(Skv):
+                    ref[b, h, i, j] = sel[b, h, i // qb, j // kb] and valid[b, j] and (not causal or j <= i)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_bsr_and_block_bits_select_the_same_mask():
+    from workloads import bsr_routing
+    indptr, indices = bsr_routing(1, 2, 6, 5)
+    bits = om.bsr_to_block_bits(indptr, indices, 6)
+    for causal in (False, True):
+        np.testing.assert_array_equal(om.bsr_dense(indptr, indices, 6 * 7, 6 * 9, 7, 9, causal=causal),
+                                      om.block_bits_dense(bits, 6 * 7, 6 * 9, 7, 9, causal=causal))
