@@ -137,6 +137,8 @@ bfa_status bfa_plan_dense(const uint8_t* mask, int64_t mask_row_stride, int Sq, 
  *     THD layout (tensorplay varlen), or NULL for the batched layout.  In varlen
  *     mode B is the number of sequences, Sq / Sk are ignored, and max_q / max_k
  *     must be >= every sequence length (under-stating is BFA_ERR_INVALID_ARG).
+ *   seqused_k: device i32 [B] or NULL: only the first seqused_k[b] keys of batch
+ *     entry / sequence b are usable (tensorplay varlen seqused_k); read back once.
  *   window_left: -1 = off; else keys with 0 <= q_pos - k_pos < window_left are
  *     kept (window of past keys including the query's own position).  Requires
  *     positional ids and no validity masks.
@@ -146,8 +148,8 @@ bfa_status bfa_plan_dense(const uint8_t* mask, int64_t mask_row_stride, int Sq, 
  */
 bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
                              const uint8_t* k_valid, int B, int Sq, int Sk, const int32_t* cu_seqlens_q,
-                             const int32_t* cu_seqlens_k, int max_q, int max_k, int window_left,
-                             bfa_plan** out, void* stream);
+                             const int32_t* cu_seqlens_k, const int32_t* seqused_k, int max_q, int max_k,
+                             int window_left, bfa_plan** out, void* stream);
 
 /*
  * Plan from BSR routing (flashinfer block_sparse_attention, sparse_format "bsr").
@@ -204,6 +206,24 @@ bfa_status bfa_fwd(const bfa_plan* plan, const void* q, const void* k, const voi
                    const int64_t q_strides[3], const int64_t k_strides[3], const int64_t v_strides[3],
                    int B, int H, int Hkv, int D, float scale, void* out, const int64_t o_strides[3],
                    float* lse, void* stream);
+
+/*
+ * bfa_fwd with keys and values in a paged cache (tensorplay varlen block_table):
+ * the cache need not be contiguous per sequence.
+ *   k_cache, v_cache: bf16 [num_pages, page_size, Hkv, D] with the same strides
+ *   cache_strides = {page, token, head} in elements (pages contiguous: page
+ *   stride = page_size * token stride; D contiguous).
+ *   block_table: device i32 [n_seq, pages_per_seq]; key token t of sequence s
+ *   (batch entry s of a batched or dense plan, sequence s of a varlen plan) is
+ *   row t % page_size of page block_table[s, t / page_size].  Entries past a
+ *   sequence's keys are not read.  page_size in {8, 16, 32, 64} or a multiple of
+ *   128; pages_per_seq * page_size must cover the plan's longest key range.
+ *   Everything else as for bfa_fwd (the plan's key lengths bound the keys).
+ */
+bfa_status bfa_fwd_paged(const bfa_plan* plan, const void* q, const int64_t q_strides[3], const void* k_cache,
+                         const void* v_cache, const int64_t cache_strides[3], int64_t num_pages, int page_size,
+                         const int32_t* block_table, int pages_per_seq, int B, int H, int Hkv, int D,
+                         float scale, void* out, const int64_t o_strides[3], float* lse, void* stream);
 
 /* Host-side plan description (no sync). */
 bfa_status bfa_plan_get_info(const bfa_plan* plan, bfa_plan_info* info);

@@ -23,7 +23,7 @@ import torch
 from . import _lib
 from ._lib import BfaError, PlanInfo
 
-__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_bsr", "plan_block_bits", "fwd",
+__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_bsr", "plan_block_bits", "fwd", "fwd_paged",
            "make_att_block_ids",
            "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "library_path"]
 
@@ -174,11 +174,13 @@ def plan_dense(mask, stream=None):
 
 
 def plan_blockids(q_blk=None, k_blk=None, q_valid=None, k_valid=None, *, B=None, Sq=None, Sk=None,
-                  cu_seqlens_q=None, cu_seqlens_k=None, max_q=0, max_k=0, window_left=-1, stream=None):
+                  cu_seqlens_q=None, cu_seqlens_k=None, seqused_k=None, max_q=0, max_k=0, window_left=-1,
+                  stream=None):
     """Plan from block ids / validity (opentau) or, with ids None, from causal positions.
 
     Batched: ids (B, Sq) / (B, Sk).  Varlen: ids over packed tokens, ``cu_seqlens_*``
     int32 (B + 1,) starting at 0, ``max_q`` / ``max_k`` >= every sequence length.
+    ``seqused_k`` int32 (B,) bounds the usable keys of each batch entry / sequence.
     ``window_left`` > 0 keeps keys with 0 <= q_pos - k_pos < window_left.
     """
     varlen = cu_seqlens_q is not None
@@ -202,8 +204,9 @@ def plan_blockids(q_blk=None, k_blk=None, q_valid=None, k_valid=None, *, B=None,
     ck = (cu_seqlens_k if cu_seqlens_k is not None else cu_seqlens_q).to(torch.int32).contiguous() if varlen else None
     h = ctypes.c_void_p()
     st = _stream(stream)
+    su = seqused_k.to(torch.int32).contiguous() if seqused_k is not None else None
     _lib.check(_L.bfa_plan_blockids(_ptr(qb), _ptr(kb), _ptr(qv), _ptr(kv), int(B), int(Sq or 0), int(Sk or 0),
-                                    _ptr(cq), _ptr(ck), int(max_q), int(max_k), int(window_left),
+                                    _ptr(cq), _ptr(ck), _ptr(su), int(max_q), int(max_k), int(window_left),
                                     ctypes.byref(h), st))
     return Plan(h, st)
 
@@ -278,4 +281,39 @@ def fwd(plan, q, k, v, scale=None, out=None, return_lse=True, lse=None, stream=N
     _lib.check(_L.bfa_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _strides3(q), _strides3(k), _strides3(v),
                           int(B), int(H), int(Hkv), int(D), ctypes.c_float(sc), _ptr(out), _strides3(out),
                           _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def fwd_paged(plan, q, k_cache, v_cache, block_table, scale=None, out=None, return_lse=True, lse=None, stream=None):
+    """Masked attention forward with keys / values in a paged cache.
+
+    k_cache / v_cache: (num_pages, page_size, Hkv, D) bf16; block_table: (n_seq,
+    pages_per_seq) int32 page ids (tensorplay varlen ``block_table``).  q and the
+    plan as for ``fwd``.
+    """
+    if q.dtype != torch.bfloat16 or k_cache.dtype != torch.bfloat16 or v_cache.dtype != torch.bfloat16:
+        raise TypeError("q and the caches must be bfloat16")
+    if k_cache.stride() != v_cache.stride() or k_cache.shape != v_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape and strides")
+    packed = q.dim() == 3
+    if packed:
+        B = plan.info["batch"]
+        _, H, D = q.shape
+        lse_shape = (H, q.shape[0])
+    else:
+        B, Sq, H, D = q.shape
+        lse_shape = (B, H, Sq)
+    num_pages, page_size, Hkv, _ = k_cache.shape
+    bt = block_table.to(torch.int32).contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    cs = (ctypes.c_int64 * 3)(k_cache.stride(0), k_cache.stride(1), k_cache.stride(2))
+    sc = float(scale) if scale is not None else 0.0
+    _lib.check(_L.bfa_fwd_paged(plan.handle, _ptr(q), _strides3(q), _ptr(k_cache), _ptr(v_cache), cs, num_pages,
+                                page_size, _ptr(bt), bt.shape[1], int(B), int(H), int(Hkv), int(D),
+                                ctypes.c_float(sc), _ptr(out), _strides3(out), _ptr(lse), _stream(stream)))
     return out, lse

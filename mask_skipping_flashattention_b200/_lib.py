@@ -32,8 +32,8 @@ SIGNATURES = {
     "bfa_plan_dense": (ctypes.c_int, [c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                       ctypes.POINTER(c_void), c_void]),
     "bfa_plan_blockids": (ctypes.c_int, [c_void, c_void, c_void, c_void, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_int, c_void, c_void, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                         ctypes.POINTER(c_void), c_void]),
+                                         ctypes.c_int, c_void, c_void, c_void, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.POINTER(c_void), c_void]),
     "bfa_plan_bsr": (ctypes.c_int, [c_void, c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, c_void,
                                     ctypes.POINTER(c_void), c_void]),
@@ -43,6 +43,9 @@ SIGNATURES = {
     "bfa_fwd": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_i64p, c_i64p, c_i64p, ctypes.c_int,
                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, c_void, c_i64p,
                                c_void, c_void]),
+    "bfa_fwd_paged": (ctypes.c_int, [c_void, c_void, c_i64p, c_void, c_void, c_i64p, ctypes.c_int64, ctypes.c_int,
+                                     c_void, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_float, c_void, c_i64p, c_void, c_void]),
     "bfa_plan_get_info": (ctypes.c_int, [c_void, c_void]),
     "bfa_plan_stats": (ctypes.c_int, [c_void, c_i64p, c_i64p, c_i64p, c_void]),
     "bfa_plan_export": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_void]),

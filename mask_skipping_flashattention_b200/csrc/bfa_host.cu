@@ -392,8 +392,8 @@ BFA_API bfa_status bfa_plan_dense(const uint8_t* mask, int64_t ld, int Sq, int S
 
 BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
                                      const uint8_t* k_valid, int B, int Sq, int Sk, const int32_t* cu_q,
-                                     const int32_t* cu_k, int max_q, int max_k, int window_left, bfa_plan** out,
-                                     void* stream) {
+                                     const int32_t* cu_k, const int32_t* seqused_k, int max_q, int max_k,
+                                     int window_left, bfa_plan** out, void* stream) {
   if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (B <= 0) return fail(BFA_ERR_INVALID_ARG, "B=%d must be positive", B);
@@ -409,7 +409,8 @@ BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk,
   bfa_status s;
   if ((s = need_device(q_blk, "q_blk", true)) || (s = need_device(k_blk, "k_blk", true)) ||
       (s = need_device(q_valid, "q_valid", true)) || (s = need_device(k_valid, "k_valid", true)) ||
-      (s = need_device(cu_q, "cu_seqlens_q", true)) || (s = need_device(cu_k, "cu_seqlens_k", true)))
+      (s = need_device(cu_q, "cu_seqlens_q", true)) || (s = need_device(cu_k, "cu_seqlens_k", true)) ||
+      (s = need_device(seqused_k, "seqused_k", true)))
     return s;
   const bool varlen = cu_q != nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -447,6 +448,18 @@ BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk,
     P->sk = Sk;
   }
   P->regular = !varlen;
+  if (seqused_k) {  // usable keys per batch entry / sequence (read back once)
+    std::vector<int32_t> used(B);
+    BFA_CUDA(cudaMemcpyAsync(used.data(), seqused_k, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, st), "read seqused_k");
+    BFA_CUDA(cudaStreamSynchronize(st), "read seqused_k");
+    for (int b = 0; b < B; ++b) {
+      GroupInfo& g = P->groups_h[b];
+      if (used[b] < 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "seqused_k[%d] = %d is negative", b, used[b]); }
+      g.k_len = std::min(g.k_len, used[b]);
+      g.nkt = cdiv(g.k_len, kTile);
+    }
+    P->regular = false;
+  }
   P->copy_ids = P->mask_mode == MASK_BLOCKID;
   finalize_layout(P);
   // padded per-group id copies (block-id mode only)
@@ -660,7 +673,7 @@ EncodeTiledFn encode_fn() {
 // 4-D map over (d, head, token, batch) of a bf16 tensor, box = 64 d x 1 head x
 // 128 tokens x 1 batch, 128-byte swizzle: one 16 KB panel of a 128 x D tile.
 bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int64_t tokens, int batch, int64_t s_head,
-               int64_t s_tok, int64_t s_batch, std::string* why) {
+               int64_t s_tok, int64_t s_batch, std::string* why, int box_rows = kTile) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
@@ -672,7 +685,7 @@ bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int64_t token
                         static_cast<cuuint64_t>(batch)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_head) * 2, static_cast<cuuint64_t>(s_tok) * 2,
                            static_cast<cuuint64_t>(s_batch) * 2};
-  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -698,16 +711,29 @@ int sm_count() {
   return n;
 }
 
+struct PagedKV {
+  const int32_t* block_table = nullptr;
+  int page_size = 0, pages_per_seq = 0;
+  int64_t cache_tokens = 0;  // num_pages * page_size
+};
+
 cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t* qs,
                                  const int64_t* ks, const int64_t* vs, int B, int H, int Hkv, int D, float scale,
                                  void* out, const int64_t* os, float* lse, uint64_t wait_ns, cudaStream_t st,
-                                 std::string* why) {
+                                 std::string* why, const PagedKV& pg = PagedKV()) {
   const int bq = P->varlen ? 1 : B;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why) ||
-      !make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], why) ||
-      !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], why))
-    return cudaErrorInvalidValue;
+  if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why)) return cudaErrorInvalidValue;
+  if (pg.page_size == 0) {
+    if (!make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], why) ||
+        !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], why))
+      return cudaErrorInvalidValue;
+  } else {  // the cache as one token axis; boxes of one page (at most one tile)
+    const int rows = std::min(pg.page_size, static_cast<int>(kTile));
+    if (!make_tmap(&tk, k, D, Hkv, pg.cache_tokens, 1, ks[2], ks[1], 0, why, rows) ||
+        !make_tmap(&tv, v, D, Hkv, pg.cache_tokens, 1, vs[2], vs[1], 0, why, rows))
+      return cudaErrorInvalidValue;
+  }
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
   p.plan.groups = P->groups;
@@ -761,6 +787,9 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.o_sh = os[2];
   p.lse = lse;
   p.wait_ns = wait_ns;
+  p.block_table = pg.block_table;
+  p.page_size = pg.page_size;
+  p.pages_per_seq = pg.pages_per_seq;
   const int64_t n_work = units * items;
   return launch_fwd(D, tq, tk, tv, p, n_work, st);
 }
@@ -796,6 +825,62 @@ BFA_API bfa_status bfa_fwd(const bfa_plan* P, const void* q, const void* k, cons
   std::string why;
   cudaError_t e = fwd_launch_from_host(P, q, k, v, qs, ks, vs, B, H, Hkv, D, scale, out, os, lse, g_wait_ns,
                                        static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) {
+    if (!why.empty()) return fail(BFA_ERR_INVALID_ARG, "%s", why.c_str());
+    return cuda_fail(e, "forward kernel");
+  }
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_fwd_paged(const bfa_plan* P, const void* q, const int64_t q_strides[3], const void* k_cache,
+                                 const void* v_cache, const int64_t cache_strides[3], int64_t num_pages, int page_size,
+                                 const int32_t* block_table, int pages_per_seq, int B, int H, int Hkv, int D,
+                                 float scale, void* out, const int64_t o_strides[3], float* lse, void* stream) {
+  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  if (!q_strides || !cache_strides || !o_strides) return fail(BFA_ERR_INVALID_ARG, "strides are NULL");
+  if (D != 64 && D != 128) return fail(BFA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", D);
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0) return fail(BFA_ERR_INVALID_ARG, "H=%d must be a positive multiple of Hkv=%d", H, Hkv);
+  if (B <= 0) return fail(BFA_ERR_INVALID_ARG, "B=%d must be positive", B);
+  if (P->kind != BFA_PLAN_DENSE && B != P->batch)
+    return fail(BFA_ERR_INVALID_ARG, "B=%d does not match the plan's %d", B, P->batch);
+  if (P->kind == BFA_PLAN_BSR && Hkv != P->hkv)
+    return fail(BFA_ERR_INVALID_ARG, "Hkv=%d does not match the BSR routing's %d", Hkv, P->hkv);
+  if (!(page_size == 8 || page_size == 16 || page_size == 32 || page_size == 64 ||
+        (page_size > 0 && page_size % kTile == 0)))
+    return fail(BFA_ERR_INVALID_ARG, "page_size=%d must be 8, 16, 32, 64 or a multiple of 128", page_size);
+  if (num_pages <= 0 || pages_per_seq <= 0) return fail(BFA_ERR_INVALID_ARG, "num_pages / pages_per_seq must be positive");
+  int max_k = 0;
+  for (const auto& g : P->groups_h) max_k = std::max(max_k, g.k_len);
+  if (static_cast<int64_t>(pages_per_seq) * page_size < max_k)
+    return fail(BFA_ERR_INVALID_ARG, "pages_per_seq * page_size = %lld is below the plan's %d keys",
+                (long long)pages_per_seq * page_size, max_k);
+  if (cache_strides[0] != static_cast<int64_t>(page_size) * cache_strides[1])
+    return fail(BFA_ERR_INVALID_ARG, "cache pages must be contiguous (page stride = page_size * token stride)");
+  if (num_pages * page_size >= (int64_t(1) << 31)) return fail(BFA_ERR_CAPACITY, "cache too large");
+  bfa_status s;
+  if ((s = need_device(q, "q")) || (s = need_device(k_cache, "k_cache")) || (s = need_device(v_cache, "v_cache")) ||
+      (s = need_device(block_table, "block_table")) || (s = need_device(out, "out")) ||
+      (s = need_device(lse, "lse", true)))
+    return s;
+  const int64_t* all[3] = {q_strides, cache_strides, o_strides};
+  for (int t = 0; t < 3; ++t)
+    for (int i = 0; i < 3; ++i) {
+      if ((P->varlen || t == 1) && i == 0) continue;
+      if (all[t][i] < 0 || all[t][i] % 8 != 0)
+        return fail(BFA_ERR_INVALID_ARG, "stride %lld is not a non-negative multiple of 8 elements", (long long)all[t][i]);
+    }
+  const void* ptrs[4] = {q, k_cache, v_cache, out};
+  for (int t = 0; t < 4; ++t)
+    if (reinterpret_cast<uintptr_t>(ptrs[t]) & 15u) return fail(BFA_ERR_INVALID_ARG, "tensor base is not 16-byte aligned");
+  PagedKV pg;
+  pg.block_table = block_table;
+  pg.page_size = page_size;
+  pg.pages_per_seq = pages_per_seq;
+  pg.cache_tokens = num_pages * page_size;
+  std::string why;
+  cudaError_t e = fwd_launch_from_host(P, q, k_cache, v_cache, q_strides, cache_strides, cache_strides, B, H, Hkv, D,
+                                       scale, out, o_strides, lse, g_wait_ns, static_cast<cudaStream_t>(stream), &why,
+                                       pg);
   if (e != cudaSuccess) {
     if (!why.empty()) return fail(BFA_ERR_INVALID_ARG, "%s", why.c_str());
     return cuda_fail(e, "forward kernel");

@@ -69,6 +69,7 @@ struct Work {
   int32_t qt[2];        // query tile inside the group
   int32_t h[2];         // query head of each slot
   int32_t b, hk;
+  int32_t seq;          // row of the page table (paged keys / values)
   int32_t same_row;     // both slots run the same row (so the same list)
   int32_t q_off, q_len, k_off, k_len;
   int32_t qid_off, kid_off, kbit_off;
@@ -105,7 +106,8 @@ __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk)
     r0 = pr >= 0 ? pr : ~pr;
     r1 = pr >= 0 ? r0 + 1 : -1;
   }
-  const GroupInfo g = p.plan.groups[p.plan.row_group[r0]];
+  const int grp = p.plan.row_group[r0];
+  const GroupInfo g = p.plan.groups[grp];
   wk.same_row = p.pair_heads;
   wk.row[0] = r0;
   wk.row[1] = r1;
@@ -124,6 +126,7 @@ __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk)
     h1 = h0;
   }
   wk.b = b;
+  wk.seq = p.varlen ? grp : b;
   wk.h[0] = h0;
   wk.h[1] = h1;
   wk.hk = h0 / (p.H / p.Hkv);
@@ -229,6 +232,40 @@ __device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& w
   }
 }
 
+// TMA of one 128-token K or V tile (all D/64 panels) into `dst`, completing on
+// `bar`.  Contiguous layouts take one box per panel at token row `ks`; paged
+// layouts look the pages up in the page table: pages of >= 128 tokens give one
+// box, smaller pages one box per page, each landing at its row offset of the
+// swizzled tile (a multiple of 8 rows, so the 128-byte swizzle pattern lines up).
+// Pages past the sequence's end re-read its last valid page: finite values that
+// the edge mask never lets into the result.
+template <int kPanels>
+__device__ __forceinline__ void load_kv_tile(const FwdParams& p, const Work& wk, const CUtensorMap* map, uint8_t* dst,
+                                             uint32_t bar, int kt, int ks) {
+  if (p.page_size == 0) {
+#pragma unroll
+    for (int pn = 0; pn < kPanels; ++pn) tma_load_4d(smem_u32(dst + pn * 16384), map, bar, pn * 64, wk.hk, ks, wk.b);
+    return;
+  }
+  const int32_t* bt = p.block_table + static_cast<int64_t>(wk.seq) * p.pages_per_seq;
+  const int t0 = kt * kTile;
+  if (p.page_size >= kTile) {
+    const int row = bt[t0 / p.page_size] * p.page_size + t0 % p.page_size;
+#pragma unroll
+    for (int pn = 0; pn < kPanels; ++pn) tma_load_4d(smem_u32(dst + pn * 16384), map, bar, pn * 64, wk.hk, row, 0);
+    return;
+  }
+  const int last = max(wk.k_len - 1, 0) / p.page_size;
+  for (int sub = 0; sub < kTile / p.page_size; ++sub) {
+    const int t = t0 + sub * p.page_size;
+    const int page = bt[min(t / p.page_size, last)];
+    const int row = page * p.page_size;
+#pragma unroll
+    for (int pn = 0; pn < kPanels; ++pn)
+      tma_load_4d(smem_u32(dst + pn * 16384 + sub * p.page_size * 128), map, bar, pn * 64, wk.hk, row, 0);
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t tS, uint8_t* sQ, uint8_t* sK) {
 #pragma unroll
@@ -317,15 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ks = wk.k_off + kt * kTile;
           if (u >= kStages && !mbar_wait(bar(BKE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
           mbar_expect_tx(bar(BKF + st), C::kTileBytes);
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_4d(smem_u32(sK(st) + pn * 16384), &tmK, bar(BKF + st), pn * 64, wk.hk, ks, wk.b);
+          load_kv_tile<C::kPanels>(p, wk, &tmK, sK(st), bar(BKF + st), kt, ks);
           last_k[st] = u;
           if (u >= kStages && !mbar_wait(bar(BVE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
           mbar_expect_tx(bar(BVF + st), C::kTileBytes);
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_4d(smem_u32(sV(st) + pn * 16384), &tmV, bar(BVF + st), pn * 64, wk.hk, ks, wk.b);
+          load_kv_tile<C::kPanels>(p, wk, &tmV, sV(st), bar(BVF + st), kt, ks);
           last_v[st] = u;
           ++u;
         }

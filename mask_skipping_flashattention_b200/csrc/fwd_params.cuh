@@ -23,6 +23,12 @@ struct FwdParams {
   int64_t o_sb, o_ss, o_sh;
   float* lse;
   uint64_t wait_ns;
+  // paged keys / values (0 = contiguous): key token t of sequence s lives at row
+  // block_table[s * pages_per_seq + t / page_size] * page_size + t % page_size of
+  // the cache viewed as one token axis
+  const int32_t* block_table;
+  int32_t page_size;
+  int32_t pages_per_seq;
 };
 
 int fwd_smem_bytes(int D);

@@ -292,3 +292,83 @@ def test_general_block_sparse_forward(qb, kb, causal):
                             kv_valid_bits=kvb)
     pairs = [(b, h) for b in range(B) for h in range(H)]
     check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M[b, h // (H // Hkv)], None, pairs, where="general bsr")
+
+
+# ---------------------------------------------------------------- paged keys / values, seqused_k
+def _paged_cache(lens, page_size, Hkv, D, seed):
+    """Scatter per-sequence K/V into randomly placed pages; returns caches, table, gathered K/V."""
+    rng = np.random.default_rng(seed)
+    n_pages_seq = [-(-L // page_size) for L in lens]
+    pages_per_seq = max(max(n_pages_seq), 1) + 1
+    num_pages = sum(n_pages_seq) + 5
+    perm = rng.permutation(num_pages)
+    kc = _rand((num_pages, page_size, Hkv, D), seed + 1)
+    vc = _rand((num_pages, page_size, Hkv, D), seed + 2)
+    table = np.full((len(lens), pages_per_seq), -1, dtype=np.int32)
+    ks, vs, pos = [], [], 0
+    for s, L in enumerate(lens):
+        pages = perm[pos:pos + n_pages_seq[s]]
+        pos += n_pages_seq[s]
+        table[s, :len(pages)] = pages
+        rows_k = torch.cat([kc[int(p_)] for p_ in pages], dim=0)[:L] if len(pages) else kc[:0, 0]
+        rows_v = torch.cat([vc[int(p_)] for p_ in pages], dim=0)[:L] if len(pages) else vc[:0, 0]
+        ks.append(rows_k)
+        vs.append(rows_v)
+    return kc, vc, table, ks, vs
+
+
+@pytest.mark.parametrize("page_size", [16, 64, 128, 256])
+def test_paged_kv_varlen(page_size):
+    lens = [100, 300, 129, 257, 1]
+    H, Hkv, D = 4, 2, 128
+    cu = np.zeros(len(lens) + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    T = int(cu[-1])
+    q = _rand((T, H, D), 61)
+    kc, vc, table, ks, vs = _paged_cache(lens, page_size, Hkv, D, 70 + page_size)
+    P = bfa.plan_blockids(cu_seqlens_q=_cuda(cu), cu_seqlens_k=_cuda(cu), max_q=max(lens), max_k=max(lens))
+    out, lse = bfa.fwd_paged(P, q.cuda(), kc.cuda(), vc.cuda(), _cuda(table))
+    torch.cuda.synchronize()
+    P.device_status()
+    for s, L in enumerate(lens):
+        a, b = int(cu[s]), int(cu[s + 1])
+        M = om.positional_dense(L, L, causal=True)
+        for h in range(H):
+            g = h // (H // Hkv)
+            O, Ls = oa.masked_attention(q[a:b, h], ks[s][:, g], vs[s][:, g], M)
+            compare_rows(out[a:b, h].cpu(), lse[h, a:b].cpu(), O, Ls, where=f"paged {page_size} seq {s} h {h}")
+
+
+def test_paged_kv_batched_dense_plan():
+    B, H, Hkv, S, D, page_size = 2, 2, 2, 300, 64, 32
+    q = _rand((B, S, H, D), 81)
+    kc, vc, table, ks, vs = _paged_cache([S] * B, page_size, Hkv, D, 90)
+    M = om.positional_dense(S, S, causal=True)
+    P = bfa.plan_dense(_cuda(M))
+    out, lse = bfa.fwd_paged(P, q.cuda(), kc.cuda(), vc.cuda(), _cuda(table))
+    torch.cuda.synchronize()
+    for b in range(B):
+        for h in range(H):
+            O, Ls = oa.masked_attention(q[b, :, h], ks[b][:, h], vs[b][:, h], M)
+            compare_rows(out[b, :, h].cpu(), lse[b, h].cpu(), O, Ls, where=f"paged dense b {b} h {h}")
+
+
+def test_seqused_k_bounds_the_keys():
+    lens = [300, 200, 129]
+    used = np.array([250, 0, 129], dtype=np.int32)       # a sequence with no usable key
+    H, Hkv, D = 2, 1, 64
+    cu = np.zeros(len(lens) + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    T = int(cu[-1])
+    q, k, v = _rand((T, H, D), 91), _rand((T, Hkv, D), 92), _rand((T, Hkv, D), 93)
+    P = bfa.plan_blockids(cu_seqlens_q=_cuda(cu), cu_seqlens_k=_cuda(cu), seqused_k=_cuda(used), max_q=300,
+                          max_k=300)
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    for s, L in enumerate(lens):
+        a, b = int(cu[s]), int(cu[s + 1])
+        M = om.positional_dense(L, L, causal=True)
+        M[:, used[s]:] = False
+        for h in range(H):
+            O, Ls = oa.masked_attention(q[a:b, h], k[a:b, 0], v[a:b, 0], M)
+            compare_rows(out[a:b, h].cpu(), lse[h, a:b].cpu(), O, Ls, where=f"seqused seq {s} h {h}")
