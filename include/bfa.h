@@ -68,8 +68,23 @@ typedef enum bfa_plan_kind {
   BFA_PLAN_DENSE = 1,      /* from a dense (Sq, Sk) bool mask, shared by every batch and head   */
   BFA_PLAN_BLOCKIDS = 2,   /* from per-token block ids and validity, per batch / sequence       */
   BFA_PLAN_POSITIONAL = 3, /* causal (+ window) on token positions, per batch / sequence        */
-  BFA_PLAN_BSR = 4         /* from BSR routing, per (batch, kv head)                            */
+  BFA_PLAN_BSR = 4,        /* from BSR routing or block bitmaps, per (batch, kv head)           */
+  BFA_PLAN_PREDICATE = 5   /* from position terms (OR of band / box constraints), per sequence  */
 } bfa_plan_kind;
+
+/* One conjunction of position constraints on (i, j) = (query, key) positions
+ * local to the sequence:  diag_lo <= i - j <= diag_hi  AND  q_lo <= i < q_hi
+ * AND  k_lo <= j < k_hi.  INT32_MIN / INT32_MAX leave a bound open.  Examples:
+ * causal {0, MAX, MIN, MAX, MIN, MAX}; past window of W keys {0, W-1, ...};
+ * G global query rows {MIN, MAX, MIN, G, MIN, MAX}; P prefix keys
+ * {MIN, MAX, MIN, MAX, MIN, P}. */
+typedef struct bfa_mask_term {
+  int32_t diag_lo, diag_hi;
+  int32_t q_lo, q_hi;
+  int32_t k_lo, k_hi;
+} bfa_mask_term;
+
+enum { BFA_MAX_MASK_TERMS = 16 };
 
 /* Host-side description of a plan (no synchronisation needed to read it). */
 typedef struct bfa_plan_info {
@@ -150,6 +165,20 @@ bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const u
                              const uint8_t* k_valid, int B, int Sq, int Sk, const int32_t* cu_seqlens_q,
                              const int32_t* cu_seqlens_k, const int32_t* seqused_k, int max_q, int max_k,
                              int window_left, bfa_plan** out, void* stream);
+
+/*
+ * Plan from a position predicate: attend(i, j) = OR over the n_terms terms of
+ * their constraints (tensorplay omni_attention mask_mod algebra: causal,
+ * window, and_masks inside a term, or_masks across terms; n_terms = 0 attends
+ * nothing, one open term is noop_mask).  terms: HOST array, copied.  Layout as
+ * for bfa_plan_blockids: batched (B, Sq, Sk) or varlen through cu_seqlens with
+ * max_q / max_k, and optional seqused_k.  Tiles are classified exactly from the
+ * terms; the kernel evaluates the terms on partial tiles only, so no mask is
+ * materialised.  Varlen and seqused_k read back once.
+ */
+bfa_status bfa_plan_predicate(const bfa_mask_term* terms, int n_terms, int B, int Sq, int Sk,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const int32_t* seqused_k,
+                              int max_q, int max_k, bfa_plan** out, void* stream);
 
 /*
  * Plan from BSR routing (flashinfer block_sparse_attention, sparse_format "bsr").

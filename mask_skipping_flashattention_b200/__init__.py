@@ -23,12 +23,14 @@ import torch
 from . import _lib
 from ._lib import BfaError, PlanInfo
 
-__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_bsr", "plan_block_bits", "fwd", "fwd_paged",
+__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_predicate", "plan_bsr", "plan_block_bits",
+           "fwd", "fwd_paged",
            "make_att_block_ids",
            "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "library_path"]
 
 TILE = 128
-KIND_NAMES = {1: "dense", 2: "blockids", 3: "positional", 4: "bsr"}
+KIND_NAMES = {1: "dense", 2: "blockids", 3: "positional", 4: "bsr", 5: "predicate"}
+_I32_MIN, _I32_MAX = -(2 ** 31), 2 ** 31 - 1
 
 library_path = _lib.LIB_PATH
 _L = _lib.load()
@@ -208,6 +210,34 @@ def plan_blockids(q_blk=None, k_blk=None, q_valid=None, k_valid=None, *, B=None,
     _lib.check(_L.bfa_plan_blockids(_ptr(qb), _ptr(kb), _ptr(qv), _ptr(kv), int(B), int(Sq or 0), int(Sk or 0),
                                     _ptr(cq), _ptr(ck), _ptr(su), int(max_q), int(max_k), int(window_left),
                                     ctypes.byref(h), st))
+    return Plan(h, st)
+
+
+def plan_predicate(terms, *, B=None, Sq=None, Sk=None, cu_seqlens_q=None, cu_seqlens_k=None, seqused_k=None,
+                   max_q=0, max_k=0, stream=None):
+    """Plan from position terms: attend(i, j) = OR over terms of
+    diag_lo <= i - j <= diag_hi AND q_lo <= i < q_hi AND k_lo <= j < k_hi.
+
+    ``terms``: list of dicts with those keys (missing / None = unbounded).  Layout
+    as for ``plan_blockids`` (batched B, Sq, Sk or varlen cu_seqlens).
+    """
+    arr = (_lib.MaskTerm * max(len(terms), 1))()
+    for n, t in enumerate(terms):
+        get = lambda key, dflt: dflt if t.get(key) is None else int(t[key])
+        arr[n] = _lib.MaskTerm(get("diag_lo", _I32_MIN), get("diag_hi", _I32_MAX), get("q_lo", _I32_MIN),
+                               get("q_hi", _I32_MAX), get("k_lo", _I32_MIN), get("k_hi", _I32_MAX))
+    varlen = cu_seqlens_q is not None
+    if varlen:
+        B = cu_seqlens_q.numel() - 1
+        Sq = Sk = 0
+    cq = cu_seqlens_q.to(torch.int32).contiguous() if varlen else None
+    ck = (cu_seqlens_k if cu_seqlens_k is not None else cu_seqlens_q).to(torch.int32).contiguous() if varlen else None
+    su = seqused_k.to(torch.int32).contiguous() if seqused_k is not None else None
+    h = ctypes.c_void_p()
+    st = _stream(stream)
+    _lib.check(_L.bfa_plan_predicate(ctypes.cast(arr, ctypes.c_void_p), len(terms), int(B), int(Sq or 0),
+                                     int(Sk or 0), _ptr(cq), _ptr(ck), _ptr(su), int(max_q), int(max_k),
+                                     ctypes.byref(h), st))
     return Plan(h, st)
 
 

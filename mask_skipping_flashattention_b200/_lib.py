@@ -34,6 +34,8 @@ SIGNATURES = {
     "bfa_plan_blockids": (ctypes.c_int, [c_void, c_void, c_void, c_void, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, c_void, c_void, c_void, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.POINTER(c_void), c_void]),
+    "bfa_plan_predicate": (ctypes.c_int, [c_void, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, c_void,
+                                          c_void, c_void, ctypes.c_int, ctypes.c_int, ctypes.POINTER(c_void), c_void]),
     "bfa_plan_bsr": (ctypes.c_int, [c_void, c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, c_void,
                                     ctypes.POINTER(c_void), c_void]),
@@ -65,6 +67,11 @@ class PlanInfo(ctypes.Structure):
                 ("hkv", ctypes.c_int32), ("sq", ctypes.c_int32), ("sk", ctypes.c_int32),
                 ("max_kv_tiles", ctypes.c_int32), ("window_left", ctypes.c_int32), ("causal", ctypes.c_int32),
                 ("n_pairs", ctypes.c_int32), ("packed_fine", ctypes.c_int32)]
+
+
+class MaskTerm(ctypes.Structure):
+    _fields_ = [("diag_lo", ctypes.c_int32), ("diag_hi", ctypes.c_int32), ("q_lo", ctypes.c_int32),
+                ("q_hi", ctypes.c_int32), ("k_lo", ctypes.c_int32), ("k_hi", ctypes.c_int32)]
 
 
 class BfaError(RuntimeError):

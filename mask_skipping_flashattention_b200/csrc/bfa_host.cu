@@ -47,6 +47,8 @@ cudaError_t launch_bits_fine(const uint32_t* bits, const uint32_t* kv_valid, int
 cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
                                   const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
                                   uint8_t* k_valid, cudaStream_t s);
+cudaError_t launch_pred_classify(const int32_t* terms, int n_terms, const GroupInfo* groups, int n_groups, int nqt,
+                                 uint8_t* cls, cudaStream_t s);
 cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
                                        GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s);
 
@@ -88,6 +90,8 @@ struct bfa_plan {
   uint8_t* qvalid = nullptr;
   int32_t* kid = nullptr;
   uint32_t* kbits = nullptr;
+  int32_t* terms = nullptr;
+  int n_terms = 0;
   uint32_t* err = nullptr;
   int32_t* max_width = nullptr;
 };
@@ -180,7 +184,8 @@ struct SlabLayout {
 };
 
 // Allocate and carve the plan slab; uploads groups and row_group.
-bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t kid_elems, int64_t kbit_words) {
+bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t kid_elems, int64_t kbit_words,
+                      int64_t term_ints = 0) {
   SlabLayout L;
   const int64_t cap_tiles = std::max<int64_t>(P->grid_tiles, 1);
   const size_t o_groups = L.take<GroupInfo>(std::max(P->n_groups, 1));
@@ -201,6 +206,7 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   const size_t o_qv = L.take<uint8_t>(std::max<int64_t>(qid_elems, 1));
   const size_t o_kid = L.take<int32_t>(std::max<int64_t>(kid_elems, 1));
   const size_t o_kb = L.take<uint32_t>(std::max<int64_t>(kbit_words, 1));
+  const size_t o_terms = L.take<int32_t>(std::max<int64_t>(term_ints, 1));
   const size_t o_fine = L.take<uint32_t>(with_fine ? static_cast<size_t>(cap_tiles) * kFineWordsPerTile : 1);
   cudaMemPool_t pool;
   cudaError_t e = plan_pool(&pool);
@@ -227,6 +233,7 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->qvalid = base + o_qv;
   P->kid = reinterpret_cast<int32_t*>(base + o_kid);
   P->kbits = reinterpret_cast<uint32_t*>(base + o_kb);
+  P->terms = reinterpret_cast<int32_t*>(base + o_terms);
   P->fine = reinterpret_cast<uint32_t*>(base + o_fine);
 
   if (P->regular) {
@@ -390,6 +397,56 @@ BFA_API bfa_status bfa_plan_dense(const uint8_t* mask, int64_t ld, int Sq, int S
   return BFA_OK;
 }
 
+namespace {
+
+// Row groups of a batched (B x Sq x Sk) or varlen (cu_seqlens) layout, with the
+// usable keys optionally bounded by seqused_k.  Varlen lengths and seqused_k are
+// read back to the host (one synchronisation) and validated against max_q / max_k.
+bfa_status setup_seq_groups(bfa_plan* P, int B, int Sq, int Sk, const int32_t* cu_q, const int32_t* cu_k,
+                            const int32_t* seqused_k, int max_q, int max_k, cudaStream_t st) {
+  auto cleanup = []() {};
+  const bool varlen = cu_q != nullptr;
+  if (varlen) {
+    std::vector<int32_t> cq(B + 1), ck(B + 1);
+    BFA_CUDA(cudaMemcpyAsync(cq.data(), cu_q, sizeof(int32_t) * (B + 1), cudaMemcpyDeviceToHost, st), "read cu_seqlens_q");
+    BFA_CUDA(cudaMemcpyAsync(ck.data(), cu_k, sizeof(int32_t) * (B + 1), cudaMemcpyDeviceToHost, st), "read cu_seqlens_k");
+    BFA_CUDA(cudaStreamSynchronize(st), "read cu_seqlens");
+    if (cq[0] != 0 || ck[0] != 0) { return fail(BFA_ERR_INVALID_ARG, "cu_seqlens must start at 0"); }
+    for (int i = 0; i < B; ++i) {
+      const int lq = cq[i + 1] - cq[i], lk = ck[i + 1] - ck[i];
+      if (lq < 0 || lk < 0) { return fail(BFA_ERR_INVALID_ARG, "cu_seqlens decreases at sequence %d", i); }
+      if (lq > max_q || lk > max_k) {
+        return fail(BFA_ERR_INVALID_ARG, "sequence %d has lengths (%d, %d) above max_q=%d / max_k=%d", i, lq, lk,
+                    max_q, max_k);
+      }
+      P->groups_h.push_back(make_group(cq[i], lq, ck[i], lk, 0, -1));
+    }
+    P->sq = cq[B];
+    P->sk = ck[B];
+  } else {
+    if (Sq <= 0 || Sk <= 0) { return fail(BFA_ERR_INVALID_ARG, "Sq=%d Sk=%d must be positive", Sq, Sk); }
+    for (int b = 0; b < B; ++b) P->groups_h.push_back(make_group(0, Sq, 0, Sk, b, -1));
+    P->sq = Sq;
+    P->sk = Sk;
+  }
+  P->regular = !varlen;
+  if (seqused_k) {  // usable keys per batch entry / sequence (read back once)
+    std::vector<int32_t> used(B);
+    BFA_CUDA(cudaMemcpyAsync(used.data(), seqused_k, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, st), "read seqused_k");
+    BFA_CUDA(cudaStreamSynchronize(st), "read seqused_k");
+    for (int b = 0; b < B; ++b) {
+      GroupInfo& g = P->groups_h[b];
+      if (used[b] < 0) { return fail(BFA_ERR_INVALID_ARG, "seqused_k[%d] = %d is negative", b, used[b]); }
+      g.k_len = std::min(g.k_len, used[b]);
+      g.nkt = cdiv(g.k_len, kTile);
+    }
+    P->regular = false;
+  }
+  return BFA_OK;
+}
+
+}  // namespace
+
 BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
                                      const uint8_t* k_valid, int B, int Sq, int Sk, const int32_t* cu_q,
                                      const int32_t* cu_k, const int32_t* seqused_k, int max_q, int max_k,
@@ -423,43 +480,7 @@ BFA_API bfa_status bfa_plan_blockids(const int32_t* q_blk, const int32_t* k_blk,
   P->varlen = varlen;
   P->batch = B;
   P->stream = st;
-  if (varlen) {
-    std::vector<int32_t> cq(B + 1), ck(B + 1);
-    BFA_CUDA(cudaMemcpyAsync(cq.data(), cu_q, sizeof(int32_t) * (B + 1), cudaMemcpyDeviceToHost, st), "read cu_seqlens_q");
-    BFA_CUDA(cudaMemcpyAsync(ck.data(), cu_k, sizeof(int32_t) * (B + 1), cudaMemcpyDeviceToHost, st), "read cu_seqlens_k");
-    BFA_CUDA(cudaStreamSynchronize(st), "read cu_seqlens");
-    if (cq[0] != 0 || ck[0] != 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "cu_seqlens must start at 0"); }
-    for (int i = 0; i < B; ++i) {
-      const int lq = cq[i + 1] - cq[i], lk = ck[i + 1] - ck[i];
-      if (lq < 0 || lk < 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "cu_seqlens decreases at sequence %d", i); }
-      if (lq > max_q || lk > max_k) {
-        cleanup();
-        return fail(BFA_ERR_INVALID_ARG, "sequence %d has lengths (%d, %d) above max_q=%d / max_k=%d", i, lq, lk,
-                    max_q, max_k);
-      }
-      P->groups_h.push_back(make_group(cq[i], lq, ck[i], lk, 0, -1));
-    }
-    P->sq = cq[B];
-    P->sk = ck[B];
-  } else {
-    if (Sq <= 0 || Sk <= 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "Sq=%d Sk=%d must be positive", Sq, Sk); }
-    for (int b = 0; b < B; ++b) P->groups_h.push_back(make_group(0, Sq, 0, Sk, b, -1));
-    P->sq = Sq;
-    P->sk = Sk;
-  }
-  P->regular = !varlen;
-  if (seqused_k) {  // usable keys per batch entry / sequence (read back once)
-    std::vector<int32_t> used(B);
-    BFA_CUDA(cudaMemcpyAsync(used.data(), seqused_k, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, st), "read seqused_k");
-    BFA_CUDA(cudaStreamSynchronize(st), "read seqused_k");
-    for (int b = 0; b < B; ++b) {
-      GroupInfo& g = P->groups_h[b];
-      if (used[b] < 0) { cleanup(); return fail(BFA_ERR_INVALID_ARG, "seqused_k[%d] = %d is negative", b, used[b]); }
-      g.k_len = std::min(g.k_len, used[b]);
-      g.nkt = cdiv(g.k_len, kTile);
-    }
-    P->regular = false;
-  }
+  if ((s = setup_seq_groups(P, B, Sq, Sk, cu_q, cu_k, seqused_k, max_q, max_k, st))) { cleanup(); return s; }
   P->copy_ids = P->mask_mode == MASK_BLOCKID;
   finalize_layout(P);
   // padded per-group id copies (block-id mode only)
@@ -572,6 +593,46 @@ bfa_status plan_block_sparse(const int32_t* indptr, const int32_t* indices, int6
 }
 
 }  // namespace
+
+BFA_API bfa_status bfa_plan_predicate(const bfa_mask_term* terms, int n_terms, int B, int Sq, int Sk,
+                                      const int32_t* cu_q, const int32_t* cu_k, const int32_t* seqused_k, int max_q,
+                                      int max_k, bfa_plan** out, void* stream) {
+  if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (B <= 0) return fail(BFA_ERR_INVALID_ARG, "B=%d must be positive", B);
+  if (n_terms < 0 || n_terms > BFA_MAX_MASK_TERMS)
+    return fail(BFA_ERR_INVALID_ARG, "n_terms=%d must be in [0, %d]", n_terms, BFA_MAX_MASK_TERMS);
+  if (n_terms > 0 && !terms) return fail(BFA_ERR_INVALID_ARG, "terms is NULL");
+  if ((cu_q == nullptr) != (cu_k == nullptr))
+    return fail(BFA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must both be given or both be NULL");
+  bfa_status s;
+  if ((s = need_device(cu_q, "cu_seqlens_q", true)) || (s = need_device(cu_k, "cu_seqlens_k", true)) ||
+      (s = need_device(seqused_k, "seqused_k", true)))
+    return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bfa_plan* P = new bfa_plan();
+  auto cleanup = [&]() { free_plan(P); };
+  P->kind = BFA_PLAN_PREDICATE;
+  P->mask_mode = MASK_PRED;
+  P->varlen = cu_q != nullptr;
+  P->batch = B;
+  P->stream = st;
+  P->n_terms = n_terms;
+  if ((s = setup_seq_groups(P, B, Sq, Sk, cu_q, cu_k, seqused_k, max_q, max_k, st))) { cleanup(); return s; }
+  finalize_layout(P);
+  if ((s = check_capacity(P, false))) { cleanup(); return s; }
+  if ((s = alloc_plan(P, false, 0, 0, 0, static_cast<int64_t>(n_terms) * 6))) { cleanup(); return s; }
+  if (n_terms > 0) {
+    // pageable upload of a few ints, completed before the call returns
+    BFA_CUDA(cudaMemcpyAsync(P->terms, terms, sizeof(bfa_mask_term) * n_terms, cudaMemcpyHostToDevice, st),
+             "upload mask terms");
+  }
+  BFA_CUDA(launch_pred_classify(P->terms, n_terms, P->groups, P->n_groups, P->max_nqt, P->cls, st),
+           "predicate classify kernel");
+  if ((s = build_rows(P))) { cleanup(); return s; }
+  *out = P;
+  return BFA_OK;
+}
 
 BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
                                 int Sq, int Skv, int q_block, int kv_block, int causal, const uint32_t* kv_valid_bits,
@@ -747,6 +808,8 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.plan.qvalid = P->qvalid;
   p.plan.kid = P->kid;
   p.plan.kbits = P->kbits;
+  p.plan.terms = P->terms;
+  p.plan.n_terms = P->n_terms;
   p.plan.err = P->err;
   p.plan.n_rows = P->n_rows;
   p.plan.n_groups = P->n_groups;

@@ -34,6 +34,7 @@
 
 #include "fwd_params.cuh"
 #include "plan_types.cuh"
+#include "pred.cuh"
 #include "ptx.cuh"
 
 namespace bfa {
@@ -206,6 +207,12 @@ __device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& w
         }
         am[w] = qv ? (bits & kvw[w]) : 0u;
       }
+    } else {
+      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
+    }
+  } else if (p.plan.mask_mode == MASK_PRED) {
+    if (part >= 0) {
+      pred_words(p.plan.terms, p.plan.n_terms, qpos, kt, wk.k_len, am);
     } else {
       am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
     }

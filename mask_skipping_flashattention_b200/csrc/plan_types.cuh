@@ -12,7 +12,8 @@ constexpr int kFineWordsPerTile = kTile * kWordsPerTileRow;  // 512 uint32 = 2 K
 enum MaskMode : int32_t {
   MASK_BITS = 0,     // partial tiles carry packed fine masks (dense plans)
   MASK_BLOCKID = 1,  // partial tiles evaluate q_valid & k_valid & (k_blk <= q_blk)
-  MASK_POS = 2       // partial tiles evaluate causal (+ window) on positions
+  MASK_POS = 2,      // partial tiles evaluate causal (+ window) on positions
+  MASK_PRED = 3      // partial tiles evaluate an OR of position terms (pred.cuh)
 };
 
 enum DevErr : uint32_t {
@@ -55,6 +56,7 @@ struct PlanDev {
   const uint8_t* qvalid;     // padded q validity   (block-id plans)
   const int32_t* kid;        // padded k block ids  (block-id plans)
   const uint32_t* kbits;     // padded k validity bits (block-id plans)
+  const int32_t* terms;      // position terms (predicate plans), 6 ints each
   uint32_t* err;             // device error word
   int32_t n_rows;
   int32_t n_pairs;
@@ -63,6 +65,7 @@ struct PlanDev {
   int32_t causal;
   int32_t window;            // -1 off
   int32_t kind;
+  int32_t n_terms;
 };
 
 }  // namespace bfa

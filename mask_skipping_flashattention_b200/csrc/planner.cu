@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include "plan_types.cuh"
+#include "pred.cuh"
 
 namespace bfa {
 
@@ -495,6 +496,39 @@ __global__ void __launch_bounds__(128) k_bits_fine(BlockSparseArgs a, const Grou
 }
 
 // ----------------------------------------------------------------------------
+// position-term predicates -> exact tile classes (CTA per (group, query tile))
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_pred_classify(const int32_t* __restrict__ terms, int n_terms,
+                                                       const GroupInfo* __restrict__ groups, uint8_t* __restrict__ cls) {
+  __shared__ int warp_cnt[4];
+  const GroupInfo g = groups[blockIdx.x];
+  const int qt = blockIdx.y;
+  if (qt >= g.nqt) return;
+  const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+  const int i = qt * kTile + r;
+  const bool in = i < g.q_len;
+  const int rows_in = min(kTile, g.q_len - qt * kTile);
+  for (int kt = 0; kt < g.nkt; ++kt) {
+    int cnt = 0;
+    if (in) {
+      uint32_t am[4];
+      pred_words(terms, n_terms, i, kt, g.k_len, am);
+      cnt = __popc(am[0]) + __popc(am[1]) + __popc(am[2]) + __popc(am[3]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) warp_cnt[warp] = cnt;
+    __syncthreads();
+    if (r == 0) {
+      const int c = warp_cnt[0] + warp_cnt[1] + warp_cnt[2] + warp_cnt[3];
+      const int n_in = rows_in * min(kTile, g.k_len - kt * kTile);
+      cls[g.cls_off + static_cast<int64_t>(qt) * g.nkt + kt] = static_cast<uint8_t>(c == 0 ? 0 : (c == n_in ? 2 : 1));
+    }
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------
 // make_att_block_ids: inclusive running count of block openings (CTA per batch)
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) k_make_block_ids(const uint8_t* __restrict__ pad,
@@ -659,6 +693,13 @@ cudaError_t launch_bits_fine(const uint32_t* bits, const uint32_t* kv_valid, int
   if (n_rows <= 0) return cudaSuccess;
   BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal};
   k_bits_fine<<<n_rows, 128, 0, s>>>(a, groups, row_group, row_ptr, kv_tile, part, fine);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pred_classify(const int32_t* terms, int n_terms, const GroupInfo* groups, int n_groups, int nqt,
+                                 uint8_t* cls, cudaStream_t s) {
+  if (n_groups <= 0 || nqt <= 0) return cudaSuccess;
+  k_pred_classify<<<dim3(n_groups, nqt), 128, 0, s>>>(terms, n_terms, groups, cls);
   return cudaGetLastError();
 }
 

@@ -224,6 +224,41 @@ def bsr_is_canonical(block_indptr, block_indices, n_kv_blocks):
 
 
 # --------------------------------------------------------------------------
+# position-term predicates: OR of ANDs of band and box constraints
+# --------------------------------------------------------------------------
+
+def term(diag_lo=None, diag_hi=None, q_lo=None, q_hi=None, k_lo=None, k_hi=None):
+    """One conjunction: diag_lo <= i - j <= diag_hi, q_lo <= i < q_hi, k_lo <= j < k_hi
+    (None = unbounded).  ``causal`` is term(diag_lo=0); a past window of W keys is
+    term(diag_lo=0, diag_hi=W - 1); global query rows are term(q_hi=G)."""
+    return dict(diag_lo=diag_lo, diag_hi=diag_hi, q_lo=q_lo, q_hi=q_hi, k_lo=k_lo, k_hi=k_hi)
+
+
+def predicate_dense(terms, Sq, Sk):
+    """attend(i, j) = OR over ``terms`` of their constraints, positions local to the
+    sequence; an empty list attends nothing.  Returns (Sq, Sk) bool."""
+    i = np.arange(Sq)[:, None]
+    j = np.arange(Sk)[None, :]
+    M = np.zeros((Sq, Sk), dtype=bool)
+    for t in terms:
+        m = np.ones((Sq, Sk), dtype=bool)
+        if t.get("diag_lo") is not None:
+            m &= (i - j) >= t["diag_lo"]
+        if t.get("diag_hi") is not None:
+            m &= (i - j) <= t["diag_hi"]
+        if t.get("q_lo") is not None:
+            m &= i >= t["q_lo"]
+        if t.get("q_hi") is not None:
+            m &= i < t["q_hi"]
+        if t.get("k_lo") is not None:
+            m &= j >= t["k_lo"]
+        if t.get("k_hi") is not None:
+            m &= j < t["k_hi"]
+        M |= m
+    return M
+
+
+# --------------------------------------------------------------------------
 # predicate algebra (tensorplay.nn.attention.omni_attention, "Block masks")
 # --------------------------------------------------------------------------
 

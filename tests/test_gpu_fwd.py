@@ -372,3 +372,30 @@ def test_seqused_k_bounds_the_keys():
         for h in range(H):
             O, Ls = oa.masked_attention(q[a:b, h], k[a:b, 0], v[a:b, 0], M)
             compare_rows(out[a:b, h].cpu(), lse[h, a:b].cpu(), O, Ls, where=f"seqused seq {s} h {h}")
+
+
+@pytest.mark.parametrize("name", ["prefix_lm", "global64_window256", "two_bands"])
+def test_predicate_forward(name):
+    from test_gpu_plan import PRED_CASES
+    terms = PRED_CASES[name]
+    B, H, Hkv, Sq, Sk, D = 2, 4, 2, 700, 650, 128
+    q, k, v = _rand((B, Sq, H, D), 51), _rand((B, Sk, Hkv, D), 52), _rand((B, Sk, Hkv, D), 53)
+    P = bfa.plan_predicate(terms, B=B, Sq=Sq, Sk=Sk)
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    M = om.predicate_dense(terms, Sq, Sk)
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M, None, pairs, where=name)
+
+
+def test_predicate_union_workload_sampled():
+    """The union workload's window and global tokens as terms (no dense mask), N=16384."""
+    terms = [om.term(diag_lo=0, diag_hi=2047), om.term(q_hi=64), om.term(k_hi=64)]
+    w = workloads.union_16384(with_qkv=True)
+    P = bfa.plan_predicate(terms, B=w["B"], Sq=w["S"], Sk=w["S"])
+    out, lse = bfa.fwd(P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda())
+    torch.cuda.synchronize()
+    rows = sample_rows(w["S"], 32, 8, must=(0, 63, 64, 2047, 2048, 16383))
+    M = om.predicate_dense(terms, w["S"], w["S"])
+    check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: M, None, [(0, 3), (1, 17)], rows=rows,
+               where="union terms")

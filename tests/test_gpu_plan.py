@@ -275,3 +275,38 @@ def test_general_block_sparse_rejects_bad_blocks():
         with pytest.raises(bfa.BfaError) as e:
             bfa.plan_bsr(_cuda(indptr), _cuda(indices), 256, 640, 64, kb)
         assert e.value.status == "BFA_ERR_INVALID_ARG"
+
+
+# ---------------------------------------------------------------- position-term predicates
+PRED_CASES = {
+    "causal": [om.term(diag_lo=0)],
+    "window100": [om.term(diag_lo=0, diag_hi=99)],
+    "prefix_lm": [om.term(diag_lo=0), om.term(k_hi=300)],
+    "global64_window256": [om.term(diag_lo=0, diag_hi=255), om.term(q_hi=64), om.term(k_hi=64)],
+    "two_bands": [om.term(diag_lo=-20, diag_hi=20), om.term(diag_lo=400, diag_hi=412, q_lo=450, q_hi=700)],
+    "noop": [om.term()],
+    "none": [],
+}
+
+
+@pytest.mark.parametrize("name", sorted(PRED_CASES))
+def test_predicate_plan_batched(name):
+    terms = PRED_CASES[name]
+    P = bfa.plan_predicate(terms, B=2, Sq=700, Sk=650)
+    assert P.kind == "predicate"
+    M = om.predicate_dense(terms, 700, 650)
+    assert_plan_equal(P.export(), oracle_plan_for_groups([M, M]))
+
+
+def test_predicate_plan_varlen_seqused():
+    terms = PRED_CASES["prefix_lm"]
+    cq = np.array([0, 500, 501, 1300], dtype=np.int32)
+    ck = np.array([0, 400, 900, 1700], dtype=np.int32)
+    used = np.array([400, 350, 790], dtype=np.int32)
+    P = bfa.plan_predicate(terms, cu_seqlens_q=_cuda(cq), cu_seqlens_k=_cuda(ck), seqused_k=_cuda(used),
+                           max_q=800, max_k=800)
+    masks = []
+    for s in range(3):
+        lq, lk = int(cq[s + 1] - cq[s]), int(min(ck[s + 1] - ck[s], used[s]))
+        masks.append(om.predicate_dense(terms, lq, lk))
+    assert_plan_equal(P.export(), oracle_plan_for_groups(masks))

@@ -277,3 +277,48 @@ def test_bsr_and_block_bits_select_the_same_mask():
     for causal in (False, True):
         np.testing.assert_array_equal(om.bsr_dense(indptr, indices, 6 * 7, 6 * 9, 7, 9, causal=causal),
                                       om.block_bits_dense(bits, 6 * 7, 6 * 9, 7, 9, causal=causal))
+
+
+def _brute_terms(terms, Sq, Sk):
+    M = np.zeros((Sq, Sk), dtype=bool)
+    for i in range(Sq):
+        for j in range(Sk):
+            for t in terms:
+                ok = True
+                for key, test in (("diag_lo", lambda v: i - j >= v), ("diag_hi", lambda v: i - j <= v),
+                                  ("q_lo", lambda v: i >= v), ("q_hi", lambda v: i < v),
+                                  ("k_lo", lambda v: j >= v), ("k_hi", lambda v: j < v)):
+                    if t.get(key) is not None and not test(t[key]):
+                        ok = False
+                if ok:
+                    M[i, j] = True
+                    break
+    return M
+
+
+PREDICATES = {
+    "causal": [om.term(diag_lo=0)],
+    "window5": [om.term(diag_lo=0, diag_hi=4)],
+    "prefix_lm7": [om.term(diag_lo=0), om.term(k_hi=7)],
+    "global3_window4": [om.term(diag_lo=0, diag_hi=3), om.term(q_hi=3), om.term(k_hi=3)],
+    "two_bands": [om.term(diag_lo=-2, diag_hi=2), om.term(diag_lo=10, diag_hi=12, q_lo=5, q_hi=20)],
+    "noop": [om.term()],
+    "none": [],
+}
+
+
+@pytest.mark.parametrize("name", sorted(PREDICATES))
+def test_predicate_terms_match_brute_force(name):
+    terms = PREDICATES[name]
+    np.testing.assert_array_equal(om.predicate_dense(terms, 23, 29), _brute_terms(terms, 23, 29))
+
+
+def test_predicate_terms_match_the_page_algebra():
+    """causal / window terms equal the omni_attention predicates built with and_masks / or_masks."""
+    np.testing.assert_array_equal(om.predicate_dense([om.term(diag_lo=0, diag_hi=3)], 16, 16),
+                                  om.create_mask(om.and_masks(om.causal, om.window(4)), 1, 1, 16, 16)[0, 0])
+    glob = lambda b, h, qi, ki: (qi < 3) | (ki < 3)
+    alg = om.create_mask(om.or_masks(om.and_masks(om.causal, om.window(4)), glob), 1, 1, 20, 20)[0, 0]
+    np.testing.assert_array_equal(om.predicate_dense(PREDICATES["global3_window4"], 20, 20), alg)
+    assert om.predicate_dense(PREDICATES["noop"], 4, 6).all()
+    assert not om.predicate_dense([], 4, 6).any()
