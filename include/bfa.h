@@ -237,6 +237,24 @@ bfa_status bfa_fwd(const bfa_plan* plan, const void* q, const void* k, const voi
                    float* lse, void* stream);
 
 /*
+ * bfa_fwd with content-based block skipping (BinFlash approximate_softmax +
+ * softmax_threshold, "BLASST-style"): once a query tile's scores are computed,
+ * a key tile is dropped -- no exponentials, no P V product -- when every query
+ * row of the tile has all its scores in that key tile more than
+ * softmax_threshold (natural-log units, > 0) below the row's running maximum.
+ * Each dropped weight is then below exp(-softmax_threshold) relative to the
+ * row's final maximum weight, so per row the output moves by at most
+ * 2 * n_dropped * exp(-softmax_threshold) * max|v| and the LSE by at most
+ * n_dropped * exp(-softmax_threshold).  The first tile of a row is never dropped.
+ * Everything else as for bfa_fwd.  An approximation: the result differs from
+ * bfa_fwd whenever a tile is dropped.
+ */
+bfa_status bfa_fwd_approx(const bfa_plan* plan, const void* q, const void* k, const void* v,
+                          const int64_t q_strides[3], const int64_t k_strides[3], const int64_t v_strides[3],
+                          int B, int H, int Hkv, int D, float scale, float softmax_threshold, void* out,
+                          const int64_t o_strides[3], float* lse, void* stream);
+
+/*
  * bfa_fwd with keys and values in a paged cache (tensorplay varlen block_table):
  * the cache need not be contiguous per sequence.
  *   k_cache, v_cache: bf16 [num_pages, page_size, Hkv, D] with the same strides

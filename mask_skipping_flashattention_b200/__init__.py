@@ -280,11 +280,12 @@ def _strides3(t):
     raise ValueError("expected a 4-D (B, S, H, D) or 3-D (T, H, D) tensor")
 
 
-def fwd(plan, q, k, v, scale=None, out=None, return_lse=True, lse=None, stream=None):
+def fwd(plan, q, k, v, scale=None, out=None, return_lse=True, lse=None, stream=None, softmax_threshold=None):
     """Masked attention forward; returns (out, lse or None).
 
     Batched q (B, Sq, H, D), k/v (B, Sk, Hkv, D); packed (varlen plans) q (Tq, H, D),
-    k/v (Tk, Hkv, D).  bf16, last dim contiguous, D in {64, 128}.
+    k/v (Tk, Hkv, D).  bf16, last dim contiguous, D in {64, 128}.  A positive
+    ``softmax_threshold`` turns on content-based block skipping (approximate).
     """
     for t in (q, k, v):
         if t.dtype != torch.bfloat16:
@@ -308,9 +309,15 @@ def fwd(plan, q, k, v, scale=None, out=None, return_lse=True, lse=None, stream=N
     if not return_lse:
         lse = None
     sc = float(scale) if scale is not None else 0.0
-    _lib.check(_L.bfa_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _strides3(q), _strides3(k), _strides3(v),
-                          int(B), int(H), int(Hkv), int(D), ctypes.c_float(sc), _ptr(out), _strides3(out),
-                          _ptr(lse), _stream(stream)))
+    if softmax_threshold is None:
+        _lib.check(_L.bfa_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _strides3(q), _strides3(k), _strides3(v),
+                              int(B), int(H), int(Hkv), int(D), ctypes.c_float(sc), _ptr(out), _strides3(out),
+                              _ptr(lse), _stream(stream)))
+    else:  # content-based block skipping (an approximation)
+        _lib.check(_L.bfa_fwd_approx(plan.handle, _ptr(q), _ptr(k), _ptr(v), _strides3(q), _strides3(k),
+                                     _strides3(v), int(B), int(H), int(Hkv), int(D), ctypes.c_float(sc),
+                                     ctypes.c_float(float(softmax_threshold)), _ptr(out), _strides3(out), _ptr(lse),
+                                     _stream(stream)))
     return out, lse
 
 

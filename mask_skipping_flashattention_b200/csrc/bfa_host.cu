@@ -781,7 +781,7 @@ struct PagedKV {
 cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t* qs,
                                  const int64_t* ks, const int64_t* vs, int B, int H, int Hkv, int D, float scale,
                                  void* out, const int64_t* os, float* lse, uint64_t wait_ns, cudaStream_t st,
-                                 std::string* why, const PagedKV& pg = PagedKV()) {
+                                 std::string* why, const PagedKV& pg = PagedKV(), float skip_log2 = 0.f) {
   const int bq = P->varlen ? 1 : B;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why)) return cudaErrorInvalidValue;
@@ -853,15 +853,18 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.block_table = pg.block_table;
   p.page_size = pg.page_size;
   p.pages_per_seq = pg.pages_per_seq;
+  p.skip_log2 = skip_log2;
   const int64_t n_work = units * items;
   return launch_fwd(D, tq, tk, tv, p, n_work, st);
 }
 
 }  // namespace
 
-BFA_API bfa_status bfa_fwd(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t qs[3],
-                           const int64_t ks[3], const int64_t vs[3], int B, int H, int Hkv, int D, float scale,
-                           void* out, const int64_t os[3], float* lse, void* stream) {
+namespace {
+
+bfa_status fwd_checked(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t qs[3],
+                       const int64_t ks[3], const int64_t vs[3], int B, int H, int Hkv, int D, float scale, void* out,
+                       const int64_t os[3], float* lse, void* stream, float skip_log2) {
   if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
   if (!qs || !ks || !vs || !os) return fail(BFA_ERR_INVALID_ARG, "strides are NULL");
   if (D != 64 && D != 128) return fail(BFA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", D);
@@ -887,12 +890,30 @@ BFA_API bfa_status bfa_fwd(const bfa_plan* P, const void* q, const void* k, cons
     if (reinterpret_cast<uintptr_t>(ptrs[t]) & 15u) return fail(BFA_ERR_INVALID_ARG, "tensor base is not 16-byte aligned");
   std::string why;
   cudaError_t e = fwd_launch_from_host(P, q, k, v, qs, ks, vs, B, H, Hkv, D, scale, out, os, lse, g_wait_ns,
-                                       static_cast<cudaStream_t>(stream), &why);
+                                       static_cast<cudaStream_t>(stream), &why, PagedKV(), skip_log2);
   if (e != cudaSuccess) {
     if (!why.empty()) return fail(BFA_ERR_INVALID_ARG, "%s", why.c_str());
     return cuda_fail(e, "forward kernel");
   }
   return BFA_OK;
+}
+
+}  // namespace
+
+BFA_API bfa_status bfa_fwd(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t qs[3],
+                           const int64_t ks[3], const int64_t vs[3], int B, int H, int Hkv, int D, float scale,
+                           void* out, const int64_t os[3], float* lse, void* stream) {
+  return fwd_checked(P, q, k, v, qs, ks, vs, B, H, Hkv, D, scale, out, os, lse, stream, 0.f);
+}
+
+BFA_API bfa_status bfa_fwd_approx(const bfa_plan* P, const void* q, const void* k, const void* v,
+                                  const int64_t qs[3], const int64_t ks[3], const int64_t vs[3], int B, int H,
+                                  int Hkv, int D, float scale, float softmax_threshold, void* out,
+                                  const int64_t os[3], float* lse, void* stream) {
+  if (!(softmax_threshold > 0.f))
+    return fail(BFA_ERR_INVALID_ARG, "softmax_threshold must be positive (use bfa_fwd for the exact result)");
+  return fwd_checked(P, q, k, v, qs, ks, vs, B, H, Hkv, D, scale, out, os, lse, stream,
+                     softmax_threshold * 1.4426950408889634f);
 }
 
 BFA_API bfa_status bfa_fwd_paged(const bfa_plan* P, const void* q, const int64_t q_strides[3], const void* k_cache,

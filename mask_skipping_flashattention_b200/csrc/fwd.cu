@@ -273,6 +273,14 @@ __device__ __forceinline__ void load_kv_tile(const FwdParams& p, const Work& wk,
   }
 }
 
+// approximate mode: whether the softmax warps of a slot dropped its tile t
+// (their votes were written before they arrived on the P barrier)
+__device__ __forceinline__ bool tile_skipped(const FwdParams& p, const int (&votes)[2][4], int t) {
+  if (!(p.skip_log2 > 0.f) || t == 0) return false;
+  const volatile int* v = votes[t & 1];
+  return (v[0] & v[1] & v[2] & v[3]) != 0;
+}
+
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t tS, uint8_t* sQ, uint8_t* sK) {
 #pragma unroll
@@ -308,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ Work wk_s;
+  __shared__ int skip_votes[2][2][4];  // approximate mode: [slot][tile parity][warp] "tile negligible"
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -407,12 +416,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // slot 0: O0 += P0(u) V(u), then S0 = Q0 K(u+1)^T over the consumed P0
           if (a) {
             if (!mbar_wait(bar(BP + 0), cnt0 & 1, cap, &abort_flag)) { ok = false; break; }
+            const bool skip0 = tile_skipped(p, skip_votes[0], cnt0);
             ++cnt0;
             if (!mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
             v_ready = true;
-            tc_fence_after();
-            issue_pv<D>(tO0, tS0, sV(st), started0);
-            started0 = true;
+            if (!skip0) {
+              tc_fence_after();
+              issue_pv<D>(tO0, tS0, sV(st), started0);
+              started0 = true;
+            }
           }
           if (have_next && na_) {
             if (!mbar_wait(bar(BKF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
@@ -424,11 +436,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // slot 1: O1 += P1(u) V(u), then S1 = Q1 K(u+1)^T
           if (b) {
             if (!mbar_wait(bar(BP + 1), cnt1 & 1, cap, &abort_flag)) { ok = false; break; }
+            const bool skip1 = tile_skipped(p, skip_votes[1], cnt1);
             ++cnt1;
             if (!v_ready && !mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv<D>(tO1, tS1, sV(st), started1);
-            started1 = true;
+            v_ready = true;
+            if (!skip1) {
+              tc_fence_after();
+              issue_pv<D>(tO1, tS1, sV(st), started1);
+              started1 = true;
+            }
           }
           if (have_next && nb_) {
             if (!k_ready && !mbar_wait(bar(BKF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
@@ -503,7 +519,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 8; j < 128; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float mnew = fmaxf(m, mx * c);
+        // Approximate mode (content-based block skipping): the tile is dropped when
+        // every row of the slot has its tile max more than the threshold below its
+        // running reference max (rows past the sequence count as negligible).  The
+        // four warps of the slot vote through shared memory; the MMA thread reads
+        // the same votes after the P barrier and then issues no P V for the tile.
+        bool skip = false;
+        if (p.skip_log2 > 0.f && t > 0) {
+          const bool neg = qpos >= wk.q_len || mx * c < m - p.skip_log2;
+          const bool wall = __all_sync(0xffffffffu, neg);
+          if (lane == 0) skip_votes[slot][t & 1][quarter] = wall ? 1 : 0;
+          named_bar_sync(1 + slot, 128);
+          const volatile int* v = skip_votes[slot][t & 1];
+          skip = (v[0] & v[1] & v[2] & v[3]) != 0;
+        }
+        const float mnew = skip ? m : fmaxf(m, mx * c);
         // The reference max m only moves when some row of the warp grew by more
         // than 2^8; then every row of the warp moves to its true running max
         // (alpha is 1 for rows that did not grow).  The decision is warp-uniform
@@ -525,22 +555,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           m = mnew;
         }
-        const float mref = (m == -INFINITY) ? 0.f : m;
-        // p = 2^(s*c - m), 4 independent row-sum chains; packed bf16 pairs go to
-        // the first 64 columns of S (the A operand of the P V product)
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[64];
+        if (!skip) {
+          const float mref = (m == -INFINITY) ? 0.f : m;
+          // p = 2^(s*c - m), 4 independent row-sum chains; packed bf16 pairs go to
+          // the first 64 columns of S (the A operand of the P V product)
+          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t pk[64];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float p0 = ex2_approx(fmaf(s[2 * j], c, -mref));
-          const float p1 = ex2_approx(fmaf(s[2 * j + 1], c, -mref));
-          rs[j & 3] += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
+          for (int j = 0; j < 64; ++j) {
+            const float p0 = ex2_approx(fmaf(s[2 * j], c, -mref));
+            const float p1 = ex2_approx(fmaf(s[2 * j + 1], c, -mref));
+            rs[j & 3] += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
+          }
+          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+          tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+          tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+          tmem_wait_st();
         }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(barP);

@@ -29,6 +29,9 @@ struct FwdParams {
   const int32_t* block_table;
   int32_t page_size;
   int32_t pages_per_seq;
+  // approximate mode: a tile whose scores all lie more than skip_log2 (log2 units)
+  // below the rows' running maxima is dropped; <= 0 keeps the exact computation
+  float skip_log2;
 };
 
 int fwd_smem_bytes(int D);

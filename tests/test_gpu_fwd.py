@@ -399,3 +399,52 @@ def test_predicate_union_workload_sampled():
     M = om.predicate_dense(terms, w["S"], w["S"])
     check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: M, None, [(0, 3), (1, 17)], rows=rows,
                where="union terms")
+
+
+def _near_far_inputs(B, S, H, Hkv, D, seed):
+    """Even key tiles score about +6, odd ones about -6 (natural units) for every
+    query; odd tiles carry values of 1e4, so their e^-12 weights still move the
+    exact output by ~0.06 while the approximation drops them."""
+    g = torch.Generator().manual_seed(seed)
+    u = (torch.randint(0, 2, (D,), generator=g) * 2 - 1).float() * 0.73
+    q = (u + 0.1 * torch.randn(B, S, H, D, generator=g)).to(torch.bfloat16)
+    sign = torch.ones(S)
+    for t in range(S // 128):
+        if t % 2:
+            sign[t * 128:(t + 1) * 128] = -1.0
+    k = (sign[None, :, None, None] * u + 0.1 * torch.randn(B, S, Hkv, D, generator=g)).to(torch.bfloat16)
+    v = torch.randn(B, S, Hkv, D, generator=g)
+    v[:, sign < 0] = 1e4
+    return q, k, v.to(torch.bfloat16), sign > 0
+
+
+@pytest.mark.parametrize("H,Hkv", [(2, 2), (4, 2)])
+def test_block_skipping_drops_far_tiles(H, Hkv):
+    B, S, D = 1, 1024, 128
+    q, k, v, near = _near_far_inputs(B, S, H, Hkv, D, 7)
+    P = bfa.plan_dense(_cuda(np.ones((S, S), bool)))
+    exact, lse_e = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    approx, lse_a = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda(), softmax_threshold=8.0)
+    torch.cuda.synchronize()
+    full = np.ones((S, S), bool)
+    near_only = np.broadcast_to(near.numpy()[None, :], (S, S))
+    pairs = [(0, h) for h in range(H)]
+    Of, _ = oa.attention_bshd(q, k, v, lambda b, h: full, None, heads=pairs)
+    On, _ = oa.attention_bshd(q, k, v, lambda b, h: near_only, None, heads=pairs)
+    assert max(np.abs(Of[p] - On[p]).max() for p in pairs) > 0.03   # the far tiles matter exactly
+    check_bshd(exact.cpu(), lse_e.cpu(), q, k, v, lambda b, h: full, None, pairs, where="exact")
+    check_bshd(approx.cpu(), None, q, k, v, lambda b, h: near_only, None, pairs, where="approx = near keys")
+    # LSE moves by at most n_dropped * exp(-threshold)
+    assert float((lse_a - lse_e).abs().max()) <= 512 * math.exp(-8.0) + 1e-3
+
+
+def test_block_skipping_with_huge_threshold_is_exact():
+    B, S, H, D = 1, 512, 2, 64
+    q, k, v = _rand((B, S, H, D), 5), _rand((B, S, H, D), 6), _rand((B, S, H, D), 7)
+    P = bfa.plan_dense(_cuda(om.positional_dense(S, S)))
+    o1, l1 = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    o2, l2 = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda(), softmax_threshold=1e9)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    with pytest.raises(bfa.BfaError):
+        bfa.fwd(P, q.cuda(), k.cuda(), v.cuda(), softmax_threshold=-1.0)
