@@ -28,6 +28,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+# kernels of one step: k_init_regular_groups, k_dense_classify, k_rows (the plan)
+# and bfa_fwd_kernel<128> (the forward)
+LAUNCHES_PER_STEP = 4
 METRIC = "masked attn fwd TFLOP/s on attended pairs (bf16), % of B200 tensor peak"
 WORKLOAD = dict(workload="causal_8192", B=4, H=32, Hkv=32, N=8192, D=128, mask="dense causal (N,N) bool",
                 plan="bfa_plan_dense per step", layout="BSHD")
@@ -308,7 +311,7 @@ def run_bfa(args, rank, world, local_rank):
         "fwd_ms": fwd_ms, "plan_ms": plan_ms,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
