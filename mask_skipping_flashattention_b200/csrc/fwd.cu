@@ -275,8 +275,9 @@ __device__ __forceinline__ void load_kv_tile(const FwdParams& p, const Work& wk,
 
 // approximate mode: whether the softmax warps of a slot dropped its tile t
 // (their votes were written before they arrived on the P barrier)
-__device__ __forceinline__ bool tile_skipped(const FwdParams& p, const int (&votes)[2][4], int t) {
-  if (!(p.skip_log2 > 0.f) || t == 0) return false;
+template <bool kSkip>
+__device__ __forceinline__ bool tile_skipped(const int (&votes)[2][4], int t) {
+  if (!kSkip || t == 0) return false;
   const volatile int* v = votes[t & 1];
   return (v[0] & v[1] & v[2] & v[3]) != 0;
 }
@@ -299,7 +300,9 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint8_t* sV, 
             (acc || kk > 0) ? 1u : 0u);
 }
 
-template <int D>
+// kSkip: approximate mode (content-based block skipping); the exact kernel is
+// compiled without any of its code.
+template <int D, bool kSkip>
 __global__ void __launch_bounds__(kThreads, 1)
     bfa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  const Work wk = wk_s;
+  const Work& wk = wk_s;  // read from shared memory where used: keeps warpgroup 0 within its registers
   const uint64_t cap = p.wait_ns;
   const bool any_tiles = wk.n[0] + wk.n[1] > 0;
 
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // slot 0: O0 += P0(u) V(u), then S0 = Q0 K(u+1)^T over the consumed P0
           if (a) {
             if (!mbar_wait(bar(BP + 0), cnt0 & 1, cap, &abort_flag)) { ok = false; break; }
-            const bool skip0 = tile_skipped(p, skip_votes[0], cnt0);
+            const bool skip0 = tile_skipped<kSkip>(skip_votes[0], cnt0);
             ++cnt0;
             if (!mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
             v_ready = true;
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // slot 1: O1 += P1(u) V(u), then S1 = Q1 K(u+1)^T
           if (b) {
             if (!mbar_wait(bar(BP + 1), cnt1 & 1, cap, &abort_flag)) { ok = false; break; }
-            const bool skip1 = tile_skipped(p, skip_votes[1], cnt1);
+            const bool skip1 = tile_skipped<kSkip>(skip_votes[1], cnt1);
             ++cnt1;
             if (!v_ready && !mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
             v_ready = true;
@@ -525,13 +528,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // four warps of the slot vote through shared memory; the MMA thread reads
         // the same votes after the P barrier and then issues no P V for the tile.
         bool skip = false;
-        if (p.skip_log2 > 0.f && t > 0) {
-          const bool neg = qpos >= wk.q_len || mx * c < m - p.skip_log2;
-          const bool wall = __all_sync(0xffffffffu, neg);
-          if (lane == 0) skip_votes[slot][t & 1][quarter] = wall ? 1 : 0;
-          named_bar_sync(1 + slot, 128);
-          const volatile int* v = skip_votes[slot][t & 1];
-          skip = (v[0] & v[1] & v[2] & v[3]) != 0;
+        if constexpr (kSkip) {
+          if (t > 0) {
+            const bool neg = qpos >= wk.q_len || mx * c < m - p.skip_log2;
+            const bool wall = __all_sync(0xffffffffu, neg);
+            if (lane == 0) skip_votes[slot][t & 1][quarter] = wall ? 1 : 0;
+            named_bar_sync(1 + slot, 128);
+            const volatile int* v = skip_votes[slot][t & 1];
+            skip = (v[0] & v[1] & v[2] & v[3]) != 0;
+          }
         }
         const float mnew = skip ? m : fmaxf(m, mx * c);
         // The reference max m only moves when some row of the warp grew by more
@@ -663,20 +668,22 @@ static cudaError_t prepare(K kernel, int smem) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
+template <int D, bool kSkip>
+static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const FwdParams& p, int64_t n_work, cudaStream_t s) {
+  static cudaError_t ready = prepare(bfa_fwd_kernel<D, kSkip>, Cfg<D>::kSmemBytes);
+  if (ready != cudaSuccess) return ready;
+  bfa_fwd_kernel<D, kSkip><<<static_cast<unsigned>(n_work), kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int64_t n_work, cudaStream_t s) {
   if (n_work <= 0) return cudaSuccess;
   if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  if (D == 64) {
-    static cudaError_t ready = prepare(bfa_fwd_kernel<64>, Cfg<64>::kSmemBytes);
-    if (ready != cudaSuccess) return ready;
-    bfa_fwd_kernel<64><<<static_cast<unsigned>(n_work), kThreads, Cfg<64>::kSmemBytes, s>>>(tq, tk, tv, p);
-  } else {
-    static cudaError_t ready = prepare(bfa_fwd_kernel<128>, Cfg<128>::kSmemBytes);
-    if (ready != cudaSuccess) return ready;
-    bfa_fwd_kernel<128><<<static_cast<unsigned>(n_work), kThreads, Cfg<128>::kSmemBytes, s>>>(tq, tk, tv, p);
-  }
-  return cudaGetLastError();
+  const bool approx = p.skip_log2 > 0.f;
+  if (D == 64) return approx ? launch_one<64, true>(tq, tk, tv, p, n_work, s) : launch_one<64, false>(tq, tk, tv, p, n_work, s);
+  return approx ? launch_one<128, true>(tq, tk, tv, p, n_work, s) : launch_one<128, false>(tq, tk, tv, p, n_work, s);
 }
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s) {
@@ -686,8 +693,10 @@ cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s) {
 
 cudaError_t probe_fwd_kernels() {
   cudaFuncAttributes a;
-  cudaError_t e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128>);
-  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64>);
+  cudaError_t e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, true>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, true>);
   return e;
 }
 
