@@ -140,10 +140,14 @@ __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk)
   wk.kbit_off = g.kbit_off;
 }
 
-// Walk the union of the two slots' ascending key-tile lists.
+// Walk the union of the two slots' ascending key-tile lists.  The entry after
+// each list's head is loaded one step early, so a step only moves registers and
+// issues the load for a later step: no global-memory latency on the caller.
 struct UnionWalk {
+  static constexpr int kEnd = 0x7fffffff;
   const int32_t* kv;
   int ea, na, eb, nb, ia, ib;
+  int ka, kb, ka2, kb2;  // heads of both lists and the entries after them
   bool same;
   __device__ __forceinline__ void init(const FwdParams& p, const Work& wk) {
     kv = p.plan.kv_tile;
@@ -153,23 +157,27 @@ struct UnionWalk {
     nb = wk.n[1];
     ia = ib = 0;
     same = wk.same_row != 0;
+    ka = na > 0 ? kv[ea] : kEnd;
+    ka2 = na > 1 ? kv[ea + 1] : kEnd;
+    kb = (!same && nb > 0) ? kv[eb] : kEnd;
+    kb2 = (!same && nb > 1) ? kv[eb + 1] : kEnd;
   }
   // next tile: kt, and whether slot 0 / slot 1 have it; false at the end
   __device__ __forceinline__ bool next(int& kt, bool& a, bool& b) {
-    if (same) {
-      if (ia >= na) return false;
-      kt = kv[ea + ia++];
-      a = b = true;
-      return true;
-    }
-    const int ka = ia < na ? kv[ea + ia] : 0x7fffffff;
-    const int kb = ib < nb ? kv[eb + ib] : 0x7fffffff;
-    if (ka == 0x7fffffff && kb == 0x7fffffff) return false;
     kt = min(ka, kb);
-    a = ka == kt;
-    b = kb == kt;
-    ia += a;
-    ib += b;
+    if (kt == kEnd) return false;
+    a = same || ka == kt;
+    b = same || kb == kt;
+    if (ka == kt) {
+      ++ia;
+      ka = ka2;
+      ka2 = ia + 1 < na ? kv[ea + ia + 1] : kEnd;
+    }
+    if (!same && kb == kt) {
+      ++ib;
+      kb = kb2;
+      kb2 = ib + 1 < nb ? kv[eb + ib + 1] : kEnd;
+    }
     return true;
   }
 };
@@ -314,7 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const sK0 = smem + 2 * C::kTileBytes;
   uint8_t* const sV0 = smem + (2 + kStages) * C::kTileBytes;
 
-  enum { BQ = 0, BKF = 1, BKE = 3, BVF = 5, BVE = 7, BS = 9, BP = 11, BO = 13, BDONE = 14, NBAR = 15 };
+  // BQ: Q0, Q1 and the first K.  BF[2]: V(j) and K(j + 1).  BE[2]: stages free.
+  // BS[2] / BP[2]: S ready / P ready per slot.  BO: all products done.
+  enum { BQ = 0, BF = 1, BE = 3, BS = 5, BP = 7, BO = 9, BDONE = 10, NBAR = 11 };
   __shared__ __align__(8) uint64_t bars[NBAR];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -349,11 +359,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsWG0>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
+      // Q of both slots and K of the first union tile on BQ; then at step j, V of
+      // union tile j and K of tile j + 1 together on F[j & 1], once the MMAs of
+      // commit j - 1 (which read the previous occupants of both stages) are done.
       if (lane == 0 && any_tiles) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        mbar_expect_tx(bar(BQ), ((wk.n[0] > 0 ? 1 : 0) + (wk.n[1] > 0 ? 1 : 0)) * C::kTileBytes);
+        UnionWalk walk;
+        walk.init(p, wk);
+        int kt, kt_n;
+        bool ha, hb;
+        walk.next(kt, ha, hb);  // any_tiles: the union has a first tile
+        mbar_expect_tx(bar(BQ), ((wk.n[0] > 0 ? 1 : 0) + (wk.n[1] > 0 ? 1 : 0) + 1) * C::kTileBytes);
         for (int s = 0; s < 2; ++s) {
           if (wk.n[s] == 0) continue;
           const int qs = wk.q_off + wk.qt[s] * kTile;
@@ -362,67 +380,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h[s], qs, wk.b);
         }
-        UnionWalk walk;
-        walk.init(p, wk);
-        int kt;
-        bool ha, hb;
-        int u = 0;
-        int last_k[kStages] = {-1, -1}, last_v[kStages] = {-1, -1};  // last fill of each stage
-        while (walk.next(kt, ha, hb)) {
-          const int st = u & 1;
-          const int ks = wk.k_off + kt * kTile;
-          if (u >= kStages && !mbar_wait(bar(BKE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
-          mbar_expect_tx(bar(BKF + st), C::kTileBytes);
-          load_kv_tile<C::kPanels>(p, wk, &tmK, sK(st), bar(BKF + st), kt, ks);
-          last_k[st] = u;
-          if (u >= kStages && !mbar_wait(bar(BVE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
-          mbar_expect_tx(bar(BVF + st), C::kTileBytes);
-          load_kv_tile<C::kPanels>(p, wk, &tmV, sV(st), bar(BVF + st), kt, ks);
-          last_v[st] = u;
-          ++u;
+        load_kv_tile<C::kPanels>(p, wk, &tmK, sK(0), bar(BQ), kt, wk.k_off + kt * kTile);
+        int last_f[2] = {-1, -1};  // last step that filled F[0] / F[1]
+        for (int j = 0;; ++j) {
+          const bool have_next = walk.next(kt_n, ha, hb);
+          if (j >= 1 && !mbar_wait_fast(bar(BE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, cap, &abort_flag)) break;
+          const uint32_t f = bar(BF + (j & 1));
+          mbar_expect_tx(f, (have_next ? 2 : 1) * C::kTileBytes);
+          load_kv_tile<C::kPanels>(p, wk, &tmV, sV(j & 1), f, kt, wk.k_off + kt * kTile);
+          if (have_next) load_kv_tile<C::kPanels>(p, wk, &tmK, sK((j + 1) & 1), f, kt_n, wk.k_off + kt_n * kTile);
+          last_f[j & 1] = j;
+          if (!have_next) break;
+          kt = kt_n;
         }
         // every copy this CTA issued must land before it can exit (bounded; on the
         // normal path these phases completed long ago)
         volatile int no_abort = 0;
-        mbar_wait(bar(BQ), 0, cap, &no_abort);
-        for (int st = 0; st < kStages; ++st) {
-          if (last_k[st] >= 0) mbar_wait(bar(BKF + st), (last_k[st] >> 1) & 1, cap, &no_abort);
-          if (last_v[st] >= 0) mbar_wait(bar(BVF + st), (last_v[st] >> 1) & 1, cap, &no_abort);
-        }
+        mbar_wait_fast(bar(BQ), 0, cap, &no_abort);
+        for (int b = 0; b < 2; ++b)
+          if (last_f[b] >= 0) mbar_wait_fast(bar(BF + b), (last_f[b] >> 1) & 1, cap, &no_abort);
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
+      // Commit c = 0 follows the first S products, commit c = u + 1 the products of
+      // iteration u; E[c & 1] tells the producer that K(c) and V(c - 1) are free.
       if (lane == 0 && any_tiles) {
         const uint32_t tS0 = tmem + C::kColS0, tS1 = tmem + C::kColS1;
         const uint32_t tO0 = tmem + C::kColO0, tO1 = tmem + C::kColO1;
         UnionWalk walk;
         walk.init(p, wk);
-        bool ok = mbar_wait(bar(BQ), 0, cap, &abort_flag);
-        int cnt0 = 0, cnt1 = 0;           // P phases consumed per slot
+        bool ok = mbar_wait_fast(bar(BQ), 0, cap, &abort_flag);
+        int cnt0 = 0, cnt1 = 0;  // P phases consumed per slot
         bool started0 = false, started1 = false;
         int kt;
         bool a, b, na_, nb_;
         bool have = ok && walk.next(kt, a, b);
         if (have) {
-          ok = mbar_wait(bar(BKF + 0), 0, cap, &abort_flag);
-          if (ok) {
-            tc_fence_after();
-            if (a) { issue_s<D>(tS0, sQ0, sK(0)); umma_commit(bar(BS + 0)); }
-            if (b) { issue_s<D>(tS1, sQ1, sK(0)); umma_commit(bar(BS + 1)); }
-            umma_commit(bar(BKE + 0));
-          }
+          tc_fence_after();
+          if (a) { issue_s<D>(tS0, sQ0, sK(0)); umma_commit(bar(BS + 0)); }
+          if (b) { issue_s<D>(tS1, sQ1, sK(0)); umma_commit(bar(BS + 1)); }
+          umma_commit(bar(BE + 0));
         }
         for (int u = 0; ok && have; ++u) {
           const int st = u & 1, st1 = (u + 1) & 1;
           const bool have_next = walk.next(kt, na_, nb_);
-          bool v_ready = false, k_ready = false;
+          // V(u) and K(u + 1)
+          if (!mbar_wait_fast(bar(BF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
           // slot 0: O0 += P0(u) V(u), then S0 = Q0 K(u+1)^T over the consumed P0
           if (a) {
-            if (!mbar_wait(bar(BP + 0), cnt0 & 1, cap, &abort_flag)) { ok = false; break; }
+            if (!mbar_wait_fast(bar(BP + 0), cnt0 & 1, cap, &abort_flag)) { ok = false; break; }
             const bool skip0 = tile_skipped<kSkip>(skip_votes[0], cnt0);
             ++cnt0;
-            if (!mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
-            v_ready = true;
             if (!skip0) {
               tc_fence_after();
               issue_pv<D>(tO0, tS0, sV(st), started0);
@@ -430,19 +438,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (have_next && na_) {
-            if (!mbar_wait(bar(BKF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
-            k_ready = true;
             tc_fence_after();
             issue_s<D>(tS0, sQ0, sK(st1));
             umma_commit(bar(BS + 0));
           }
           // slot 1: O1 += P1(u) V(u), then S1 = Q1 K(u+1)^T
           if (b) {
-            if (!mbar_wait(bar(BP + 1), cnt1 & 1, cap, &abort_flag)) { ok = false; break; }
+            if (!mbar_wait_fast(bar(BP + 1), cnt1 & 1, cap, &abort_flag)) { ok = false; break; }
             const bool skip1 = tile_skipped<kSkip>(skip_votes[1], cnt1);
             ++cnt1;
-            if (!v_ready && !mbar_wait(bar(BVF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
-            v_ready = true;
             if (!skip1) {
               tc_fence_after();
               issue_pv<D>(tO1, tS1, sV(st), started1);
@@ -450,13 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (have_next && nb_) {
-            if (!k_ready && !mbar_wait(bar(BKF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
             tc_fence_after();
             issue_s<D>(tS1, sQ1, sK(st1));
             umma_commit(bar(BS + 1));
           }
-          if (have_next) umma_commit(bar(BKE + st1));
-          umma_commit(bar(BVE + st));
+          umma_commit(bar(BE + st1));
           a = na_;
           b = nb_;
           have = have_next;
@@ -465,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // every MMA issued must be finished before TMEM is released (bounded)
         umma_commit(bar(BDONE));
         volatile int no_abort = 0;
-        mbar_wait(bar(BDONE), 0, cap, &no_abort);
+        mbar_wait_fast(bar(BDONE), 0, cap, &no_abort);
       }
     }
   } else {

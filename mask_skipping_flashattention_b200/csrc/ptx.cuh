@@ -49,12 +49,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on the phase with the given parity.  Gives up after `cap_ns`
 // nanoseconds of wall time, or as soon as `*abort` is set by another thread of
 // the block; returns false in both cases.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t cap_ns,
                                           volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -64,6 +77,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
       return false;
     }
   }
+}
+
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t cap_ns,
+                                                   volatile int* abort) {
+  return mbar_wait(bar, parity, cap_ns, abort);
+}
+
+// The same wait with its polling loop out of line, so that the common case of a
+// single thread finding the phase already complete costs one test and one
+// branch (the TMA producer and the MMA issuer, which hold few registers).
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, uint64_t cap_ns,
+                                               volatile int* abort) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, cap_ns, abort);
 }
 
 // ---------------------------------------------------------------- fences
