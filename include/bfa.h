@@ -317,6 +317,14 @@ void bfa_set_wait_timeout_ns(uint64_t ns);
  * stays usable), BFA_OK never.  Exercises the failure path without a fault. */
 bfa_status bfa_selftest_wait_timeout(void* stream);
 
+/* Evaluate, on the device, the FMA-pipe 2^x that the forward's softmax uses for
+ * part of its exponentials (range reduction to n + f, f in [-1/2, 1/2], and a
+ * degree-3 polynomial for 2^f): y[i] = 2^x[i] for i < n.  x and y are device
+ * pointers to n floats (n >= 0), owned by the caller; arguments at or below
+ * -127 give +0.  Returns BFA_ERR_INVALID_ARG for NULL pointers with n > 0 or
+ * n < 0, BFA_ERR_CUDA for a launch error.  Enqueued on `stream`; no sync. */
+bfa_status bfa_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
+
 /*
  * Dense-mask planner that allocates nothing.  The source pages have no
  * counterpart: this entry point exists for callers that cannot let a library

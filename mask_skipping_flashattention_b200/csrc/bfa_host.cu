@@ -1098,6 +1098,13 @@ BFA_API bfa_status bfa_selftest_wait_timeout(void* stream) {
   return BFA_OK;
 }
 
+BFA_API bfa_status bfa_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return fail(BFA_ERR_INVALID_ARG, "n = %lld < 0", static_cast<long long>(n));
+  if (n > 0 && (!x || !y)) return fail(BFA_ERR_INVALID_ARG, "x or y is NULL");
+  auto cleanup = []() {};
+  BFA_CUDA(launch_exp2_selftest(x, y, n, static_cast<cudaStream_t>(stream)), "exp2 selftest kernel");
+  return BFA_OK;
+}
 
 // ----------------------------------------------------------------------------
 // Dense planner that allocates nothing

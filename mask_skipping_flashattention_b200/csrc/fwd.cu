@@ -51,6 +51,13 @@ constexpr uint32_t kRegsSoftmax = 216;
 static_assert(128 * kRegsWG0 + 256 * kRegsSoftmax == kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
 constexpr int kStages = 2;
+// Of every 8 column pairs of a row, this many take 2^x on the FMA pipe
+// (ex2_poly) and the rest on the MUFU (ex2.approx): the exponentials are the
+// softmax's longest phase, and the two pipes run side by side.
+#ifndef BFA_POLY_PAIRS
+#define BFA_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = BFA_POLY_PAIRS;
 
 template <int D>
 struct Cfg {
@@ -516,12 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 128; ++j)
             if (!((am[j >> 5] >> (j & 31)) & 1u)) s[j] = -INFINITY;
         }
-        // row max, 8 independent chains
+        // row max, 8 independent chains of three-input max
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-        for (int j = 8; j < 128; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], s[j]);
+        for (int j = 8; j < 128; j += 2) mx8[(j >> 1) & 7] = fmax3(mx8[(j >> 1) & 7], s[j], s[j + 1]);
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         // Approximate mode (content-based block skipping): the tile is dropped when
@@ -566,16 +573,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float mref = (m == -INFINITY) ? 0.f : m;
           // p = 2^(s*c - m), 4 independent row-sum chains; packed bf16 pairs go to
           // the first 64 columns of S (the A operand of the P V product)
-          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+          // (pairs of columns go through the packed fp32x2 fma and add: half the
+          // FMA-pipe instructions of the scalar form)
+          uint64_t rs2[4] = {0, 0, 0, 0};
+          const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-mref, -mref);
           uint32_t pk[64];
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            const float p0 = ex2_approx(fmaf(s[2 * j], c, -mref));
-            const float p1 = ex2_approx(fmaf(s[2 * j + 1], c, -mref));
-            rs[j & 3] += p0 + p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, nm2), x0, x1);
+            const bool fma_pipe = (j & 7) < kPolyPairs;
+            const float p0 = fma_pipe ? ex2_poly(x0) : ex2_approx(x0);
+            const float p1 = fma_pipe ? ex2_poly(x1) : ex2_approx(x1);
+            rs2[j & 3] = f2_add(rs2[j & 3], f2_pack(p0, p1));
             pk[j] = pack_bf16x2(p0, p1);
           }
-          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+          float r[8];
+          f2_unpack(f2_add(rs2[0], rs2[1]), r[0], r[1]);
+          f2_unpack(f2_add(rs2[2], rs2[3]), r[2], r[3]);
+          l += (r[0] + r[2]) + (r[1] + r[3]);
           tmem_st_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
           tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
           tmem_wait_st();
@@ -655,6 +671,14 @@ __global__ void k_wait_selftest(uint32_t* err, uint64_t cap) {
 }
 
 // ----------------------------------------------------------------------------
+// FMA-pipe exp2 self test: y[i] = ex2_poly(x[i])
+// ----------------------------------------------------------------------------
+__global__ void k_exp2_selftest(const float* x, float* y, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = ex2_poly(x[i]);
+}
+
+// ----------------------------------------------------------------------------
 // launchers (host)
 // ----------------------------------------------------------------------------
 int fwd_smem_bytes(int D) { return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes; }
@@ -686,6 +710,12 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
   const bool approx = p.skip_log2 > 0.f;
   if (D == 64) return approx ? launch_one<64, true>(tq, tk, tv, p, n_work, s) : launch_one<64, false>(tq, tk, tv, p, n_work, s);
   return approx ? launch_one<128, true>(tq, tk, tv, p, n_work, s) : launch_one<128, false>(tq, tk, tv, p, n_work, s);
+}
+
+cudaError_t launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  k_exp2_selftest<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s) {
