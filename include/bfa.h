@@ -102,6 +102,8 @@ typedef struct bfa_plan_info {
   int32_t causal;         /* positional / BSR plans: 1 if kv_idx <= q_idx is applied             */
   int32_t n_pairs;        /* work pairs: consecutive query tiles (2i, 2i+1) of one group          */
   int32_t packed_fine;    /* 1: partial tiles carry packed fine masks (bfa_plan_export fills fine) */
+  int32_t n_cols;         /* key-tile columns (sum over groups of their key tiles): the backward's
+                             dK/dV work units, see bfa_plan_export_cols                         */
 } bfa_plan_info;
 
 /* Library version string. */
@@ -298,6 +300,19 @@ bfa_status bfa_plan_export(const bfa_plan* plan, int32_t* row_ptr, int32_t* kv_t
  * longest first (by their total listed tiles), ties by pair index.  Either pointer
  * may be NULL. */
 bfa_status bfa_plan_export_pairs(const bfa_plan* plan, int32_t* pair_row, int32_t* pair_order, void* stream);
+
+/* Copy the plan's transposed lists to HOST buffers (built on first use, on
+ * `stream`; synchronises it).  For the backward's key-tile pass (BinFlash:
+ * "dKdV over K-blocks"): column c (group g, key tile kt; groups in order, key
+ * tiles ascending) lists the query tiles whose tile (qt, kt) is not empty,
+ * ascending, in q_tile[col_ptr[c] .. col_ptr[c+1]); tpart holds -1 for full tiles
+ * and, for partial ones, the index of their packed fine words (the same index the
+ * row lists' partial entries use); col_order [n_cols] lists the columns longest
+ * first, ties by column index.  Sizes: col_ptr n_cols + 1, q_tile and tpart
+ * col_ptr[n_cols], col_order n_cols (bfa_plan_info.n_cols).  Any pointer may be
+ * NULL. */
+bfa_status bfa_plan_export_cols(const bfa_plan* plan, int32_t* col_ptr, int32_t* q_tile, int32_t* tpart,
+                                int32_t* col_order, void* stream);
 
 /* Synchronise `stream` and report BFA_ERR_TIMEOUT if a kernel that used the plan
  * hit its wait bound since the last call (the flag is then cleared). */

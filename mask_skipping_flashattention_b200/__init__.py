@@ -127,6 +127,21 @@ class Plan:
         """Raise BfaError(BFA_ERR_TIMEOUT) if a kernel using this plan hit its wait bound."""
         _lib.check(_L.bfa_plan_device_status(self.handle, _stream(stream)))
 
+    def export_cols(self, stream=None):
+        """Host copy of the transposed lists of the backward's key-tile pass:
+        col_ptr, q_tile, tpart (-1 full, else the fine-word index), col_order."""
+        n_full, n_part, _ = self.stats(stream)
+        C = self.info["n_cols"]
+        nnz = n_full + n_part
+        col_ptr = np.zeros(C + 1, np.int32)
+        q_tile = np.zeros(max(nnz, 1), np.int32)
+        tpart = np.zeros(max(nnz, 1), np.int32)
+        col_order = np.zeros(max(C, 1), np.int32)
+        P = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+        _lib.check(_L.bfa_plan_export_cols(self.handle, P(col_ptr), P(q_tile), P(tpart), P(col_order),
+                                           _stream(stream)))
+        return dict(col_ptr=col_ptr, q_tile=q_tile[:nnz], tpart=tpart[:nnz], col_order=col_order[:C])
+
     def export(self, stream=None):
         """Host copy: row_ptr, kv_tile, partial, fine (packed-mask plans), order, classes, pairs."""
         n_full, n_part, _ = self.stats(stream)

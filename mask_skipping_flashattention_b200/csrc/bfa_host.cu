@@ -37,6 +37,10 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
                         int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr, int part_is_pos = 0);
 cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int n_groups,
                                int nqb, int nkb, int wpr, uint32_t* bits, uint32_t* err, cudaStream_t s);
+cudaError_t launch_cols(const GroupInfo* groups, int n_groups, const uint8_t* cls, const int32_t* row_ptr,
+                        const int32_t* kv_tile, int part_is_pos, int max_nqt, int n_cols, int32_t* col0,
+                        int32_t* col_group, int32_t* col_cnt, int32_t* col_ptr, int32_t* q_tile, int32_t* tpart,
+                        int32_t* col_order, cudaStream_t s);
 cudaError_t launch_bits_classify(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
                                  int q_block, int kv_block, int causal, const GroupInfo* groups, int n_groups,
                                  int nqt, uint8_t* cls, cudaStream_t s);
@@ -94,6 +98,16 @@ struct bfa_plan {
   int n_terms = 0;
   uint32_t* err = nullptr;
   int32_t* max_width = nullptr;
+  int part_is_pos = 0;    // partial entries index the fine words by list position (else by grid index)
+  // transposed lists (built on first use by the backward or an export)
+  void* cols_slab = nullptr;
+  int32_t* col0 = nullptr;       // [n_groups + 1] first column of each group
+  int32_t* col_group = nullptr;  // [n_cols]
+  int32_t* col_cnt = nullptr;    // [n_cols]
+  int32_t* col_ptr = nullptr;    // [n_cols + 1]
+  int32_t* q_tile = nullptr;     // [listed tiles]
+  int32_t* tpart = nullptr;      // [listed tiles]
+  int32_t* col_order = nullptr;  // [n_cols]
 };
 
 namespace {
@@ -261,6 +275,7 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
 
 void free_plan(bfa_plan* P) {
   if (!P) return;
+  if (P->cols_slab) cudaFreeAsync(P->cols_slab, P->stream);
   if (P->fine_extra) cudaFreeAsync(P->fine_extra, P->stream);
   if (P->slab) cudaFreeAsync(P->slab, P->stream);
   delete P;
@@ -268,6 +283,7 @@ void free_plan(bfa_plan* P) {
 
 // Finish the plan: groups laid out, classes written -> lists and order.
 bfa_status build_rows(bfa_plan* P, int part_is_pos = 0) {
+  P->part_is_pos = part_is_pos;
   if (P->n_rows == 0) {
     cudaError_t e = cudaMemsetAsync(P->row_ptr, 0, sizeof(int32_t), P->stream);
     return e == cudaSuccess ? BFA_OK : cuda_fail(e, "empty plan");
@@ -277,6 +293,53 @@ bfa_status build_rows(bfa_plan* P, int part_is_pos = 0) {
                               P->kv_tile, P->part, P->order, P->stream, P->pair_row, P->pair_cost,
                               P->pair_order, P->pair_idx, part_is_pos);
   return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
+}
+
+// Key-tile columns of the plan: every group's key tiles, groups in order.
+int plan_n_cols(const bfa_plan* P) {
+  if (P->regular) return P->groups_h.empty() ? 0 : P->n_groups * P->groups_h[0].nkt;
+  int n = 0;
+  for (const auto& g : P->groups_h) n += g.nkt;
+  return n;
+}
+
+// Build the transposed lists on `st` unless they exist.
+bfa_status ensure_cols(bfa_plan* P, cudaStream_t st) {
+  if (P->cols_slab) return BFA_OK;
+  const int n_cols = plan_n_cols(P);
+  SlabLayout L;
+  const int64_t cap = std::max<int64_t>(P->grid_tiles, 1);
+  const size_t o_c0 = L.take<int32_t>(P->n_groups + 1);
+  const size_t o_cg = L.take<int32_t>(std::max(n_cols, 1));
+  const size_t o_cc = L.take<int32_t>(std::max(n_cols, 1));
+  const size_t o_cp = L.take<int32_t>(n_cols + 1);
+  const size_t o_qt = L.take<int32_t>(cap);
+  const size_t o_tp = L.take<int32_t>(cap);
+  const size_t o_co = L.take<int32_t>(std::max(n_cols, 1));
+  cudaMemPool_t pool;
+  cudaError_t e = plan_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "plan memory pool");
+  e = cudaMallocFromPoolAsync(&P->cols_slab, L.off, pool, st);
+  if (e != cudaSuccess) {
+    P->cols_slab = nullptr;
+    return fail(BFA_ERR_CAPACITY, "transposed plan allocation of %zu bytes failed: %s", L.off, cudaGetErrorString(e));
+  }
+  uint8_t* base = static_cast<uint8_t*>(P->cols_slab);
+  P->col0 = reinterpret_cast<int32_t*>(base + o_c0);
+  P->col_group = reinterpret_cast<int32_t*>(base + o_cg);
+  P->col_cnt = reinterpret_cast<int32_t*>(base + o_cc);
+  P->col_ptr = reinterpret_cast<int32_t*>(base + o_cp);
+  P->q_tile = reinterpret_cast<int32_t*>(base + o_qt);
+  P->tpart = reinterpret_cast<int32_t*>(base + o_tp);
+  P->col_order = reinterpret_cast<int32_t*>(base + o_co);
+  if (n_cols == 0 || P->n_groups == 0) {
+    e = cudaMemsetAsync(P->col_ptr, 0, sizeof(int32_t), st);
+    return e == cudaSuccess ? BFA_OK : cuda_fail(e, "empty transposed plan");
+  }
+  if (P->max_nqt > kMaxKvTiles) return fail(BFA_ERR_CAPACITY, "too many query tiles per column (%d)", P->max_nqt);
+  e = launch_cols(P->groups, P->n_groups, P->cls, P->row_ptr, P->kv_tile, P->part_is_pos, std::max(P->max_nqt, 1),
+                  n_cols, P->col0, P->col_group, P->col_cnt, P->col_ptr, P->q_tile, P->tpart, P->col_order, st);
+  return e == cudaSuccess ? BFA_OK : cuda_fail(e, "transposed plan kernel");
 }
 
 void finalize_layout(bfa_plan* P) {
@@ -988,6 +1051,7 @@ BFA_API bfa_status bfa_plan_get_info(const bfa_plan* P, bfa_plan_info* info) {
   info->causal = P->causal;
   info->n_pairs = P->n_pairs;
   info->packed_fine = P->mask_mode == MASK_BITS ? 1 : 0;
+  info->n_cols = plan_n_cols(P);
   return BFA_OK;
 }
 
@@ -1061,6 +1125,33 @@ BFA_API bfa_status bfa_plan_export_pairs(const bfa_plan* P, int32_t* pair_row, i
                "read pair order");
   }
   BFA_CUDA(cudaStreamSynchronize(st), "export pairs");
+  return BFA_OK;
+}
+
+BFA_API bfa_status bfa_plan_export_cols(const bfa_plan* Pc, int32_t* col_ptr, int32_t* q_tile, int32_t* tpart,
+                                        int32_t* col_order, void* stream) {
+  if (!Pc) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  bfa_plan* P = const_cast<bfa_plan*>(Pc);  // the transposed lists are a cache of the plan
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto cleanup = []() {};
+  bfa_status s = ensure_cols(P, st);
+  if (s != BFA_OK) return s;
+  const int n_cols = plan_n_cols(P);
+  int32_t n_listed = 0;
+  BFA_CUDA(cudaMemcpyAsync(&n_listed, P->col_ptr + n_cols, sizeof(int32_t), cudaMemcpyDeviceToHost, st),
+           "read column count");
+  BFA_CUDA(cudaStreamSynchronize(st), "export columns");
+  if (col_ptr)
+    BFA_CUDA(cudaMemcpyAsync(col_ptr, P->col_ptr, sizeof(int32_t) * (n_cols + 1), cudaMemcpyDeviceToHost, st),
+             "read col_ptr");
+  if (n_listed > 0 && q_tile)
+    BFA_CUDA(cudaMemcpyAsync(q_tile, P->q_tile, sizeof(int32_t) * n_listed, cudaMemcpyDeviceToHost, st), "read q_tile");
+  if (n_listed > 0 && tpart)
+    BFA_CUDA(cudaMemcpyAsync(tpart, P->tpart, sizeof(int32_t) * n_listed, cudaMemcpyDeviceToHost, st), "read tpart");
+  if (n_cols > 0 && col_order)
+    BFA_CUDA(cudaMemcpyAsync(col_order, P->col_order, sizeof(int32_t) * n_cols, cudaMemcpyDeviceToHost, st),
+             "read col_order");
+  BFA_CUDA(cudaStreamSynchronize(st), "export columns");
   return BFA_OK;
 }
 

@@ -367,6 +367,98 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
   block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
 }
 
+// Transposed lists for the backward's key-tile pass (BinFlash: "dKdV over
+// K-blocks"): for every key-tile column (group g, key tile kt), the ascending
+// query tiles whose class is not empty, each with its fine-word index when the
+// tile is partial (-1 when full), and the columns in longest-first order.
+// One CTA of 1024 threads; dynamic shared memory: max_nqt + 1 ints.
+__global__ void __launch_bounds__(1024) k_cols(const GroupInfo* __restrict__ groups, int n_groups,
+                                               const uint8_t* __restrict__ cls, const int32_t* __restrict__ row_ptr,
+                                               const int32_t* __restrict__ kv_tile, int part_is_pos, int max_nqt,
+                                               int n_cols, int32_t* __restrict__ col0, int32_t* __restrict__ col_group,
+                                               int32_t* __restrict__ col_cnt, int32_t* __restrict__ col_ptr,
+                                               int32_t* __restrict__ q_tile, int32_t* __restrict__ tpart,
+                                               int32_t* __restrict__ col_order) {
+  extern __shared__ int32_t bucket[];
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  // 1. first column of every group, and the group of every column
+  const int total_cols = block_exclusive_scan(n_groups, [&](int g) { return groups[g].nkt; }, col0, warp_sums, &carry);
+  if (tid == 0) col0[n_groups] = total_cols;
+  __syncthreads();
+  for (int c = tid; c < n_cols; c += blockDim.x) {
+    int lo = 0, hi = n_groups - 1;  // last group whose first column is <= c
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (col0[mid] <= c) lo = mid;
+      else hi = mid - 1;
+    }
+    col_group[c] = lo;
+  }
+  __syncthreads();
+
+  // 2. listed query tiles per column (warp per column, ballot + popc)
+  for (int c = warp; c < n_cols; c += nw) {
+    const GroupInfo g = groups[col_group[c]];
+    const int kt = c - col0[col_group[c]];
+    const uint8_t* cc = cls + g.cls_off + kt;
+    int n = 0;
+    for (int q0 = 0; q0 < g.nqt; q0 += 32) {
+      const int qt = q0 + lane;
+      n += __popc(__ballot_sync(0xffffffffu, qt < g.nqt && cc[static_cast<int64_t>(qt) * g.nkt] != 0));
+    }
+    if (lane == 0) col_cnt[c] = n;
+  }
+  __syncthreads();
+
+  // 3. exclusive scan -> col_ptr
+  const int total = block_exclusive_scan(n_cols, [&](int i) { return col_cnt[i]; }, col_ptr, warp_sums, &carry);
+  if (tid == 0) col_ptr[n_cols] = total;
+  __syncthreads();
+
+  // 4. ascending lists with the fine-word index of partial tiles
+  for (int c = warp; c < n_cols; c += nw) {
+    const int grp = col_group[c];
+    const GroupInfo g = groups[grp];
+    const int kt = c - col0[grp];
+    int out = col_ptr[c];
+    for (int q0 = 0; q0 < g.nqt; q0 += 32) {
+      const int qt = q0 + lane;
+      const int64_t cell = g.cls_off + static_cast<int64_t>(qt) * g.nkt + kt;
+      const int klass = qt < g.nqt ? cls[cell] : 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, klass != 0);
+      if (klass != 0) {
+        const int pos = out + __popc(bal & lt_mask);
+        q_tile[pos] = qt;
+        int32_t pi = -1;
+        if (klass == 1) {
+          if (part_is_pos) {  // fine words stored by list position: find kt in row (row0 + qt)
+            const int r = g.row0 + qt;
+            int lo = row_ptr[r], hi = row_ptr[r + 1] - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (kv_tile[mid] < kt) lo = mid + 1;
+              else hi = mid;
+            }
+            pi = lo;
+          } else {
+            pi = static_cast<int32_t>(cell);
+          }
+        }
+        tpart[pos] = pi;
+      }
+      out += __popc(bal);
+    }
+  }
+
+  // 5. longest-first stable column order
+  __syncthreads();
+  block_stable_order_desc(n_cols, col_cnt, max_nqt, bucket, col_order);
+}
+
 // ----------------------------------------------------------------------------
 // generic block sparsity (any BSR block sizes, exact-block bitmaps, key validity)
 // ----------------------------------------------------------------------------
@@ -665,6 +757,21 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
   }
   k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order,
                                pair_row, pair_cost, pair_order, pair_idx, part_is_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cols(const GroupInfo* groups, int n_groups, const uint8_t* cls, const int32_t* row_ptr,
+                        const int32_t* kv_tile, int part_is_pos, int max_nqt, int n_cols, int32_t* col0,
+                        int32_t* col_group, int32_t* col_cnt, int32_t* col_ptr, int32_t* q_tile, int32_t* tpart,
+                        int32_t* col_order, cudaStream_t s) {
+  const size_t smem = sizeof(int32_t) * static_cast<size_t>(max_nqt + 1);
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k_cols<<<1, 1024, smem, s>>>(groups, n_groups, cls, row_ptr, kv_tile, part_is_pos, max_nqt, n_cols, col0,
+                               col_group, col_cnt, col_ptr, q_tile, tpart, col_order);
   return cudaGetLastError();
 }
 

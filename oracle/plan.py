@@ -124,6 +124,40 @@ def plan_masks(masks, BM=128, BN=128):
     }
 
 
+def transpose_plan(cls_groups):
+    """Key-tile columns of a plan: the work lists of the backward's key-tile pass.
+
+    BinFlash ("Backward uses two passes (dKdV over K-blocks, dQ over Q-blocks)
+    with the same gathered-dispatch machinery"): the dK/dV pass visits, for every
+    key tile, the query tiles whose tile is not empty.  Column c enumerates the
+    groups in order and, inside a group, the key tiles ascending; its list holds
+    the query tiles qt with class(qt, kt) != empty, ascending, with a partial flag;
+    columns are ordered longest first, ties by column index (the row order's rule).
+    """
+    q_tile, partial, counts, col_group, col_kt = [], [], [], [], []
+    for g, cls in enumerate(cls_groups):
+        nqt, nkt = cls.shape
+        for kt in range(nkt):
+            qs = [qt for qt in range(nqt) if cls[qt, kt] != EMPTY]
+            q_tile += qs
+            partial += [1 if cls[qt, kt] == PARTIAL else 0 for qt in qs]
+            counts.append(len(qs))
+            col_group.append(g)
+            col_kt.append(kt)
+    counts = np.array(counts, dtype=np.int32)
+    col_ptr = np.zeros(len(counts) + 1, dtype=np.int32)
+    col_ptr[1:] = np.cumsum(counts)
+    return {
+        "col_ptr": col_ptr,
+        "q_tile": np.array(q_tile, dtype=np.int32),
+        "partial": np.array(partial, dtype=np.uint8),
+        "counts": counts,
+        "order": lpt_order(counts),
+        "col_group": np.array(col_group, dtype=np.int32),
+        "col_kt": np.array(col_kt, dtype=np.int32),
+    }
+
+
 def expand_plan(plan, shapes, BM=128, BN=128):
     """Inverse check: rebuild every group's dense mask from a plan.
 

@@ -310,3 +310,42 @@ def test_predicate_plan_varlen_seqused():
         lq, lk = int(cq[s + 1] - cq[s]), int(min(ck[s + 1] - ck[s], used[s]))
         masks.append(om.predicate_dense(terms, lq, lk))
     assert_plan_equal(P.export(), oracle_plan_for_groups(masks))
+
+
+# ---------------------------------------------------------------- transposed lists (backward)
+def _assert_cols_equal(P, masks):
+    from oracle import plan as op
+    ref = op.transpose_plan(op.plan_masks(masks)["cls"])
+    got = P.export_cols()
+    np.testing.assert_array_equal(got["col_ptr"], ref["col_ptr"], err_msg="col_ptr")
+    np.testing.assert_array_equal(got["q_tile"], ref["q_tile"], err_msg="q_tile")
+    np.testing.assert_array_equal((got["tpart"] >= 0).astype(np.uint8), ref["partial"], err_msg="partial flags")
+    np.testing.assert_array_equal(got["col_order"], ref["order"], err_msg="column order")
+
+
+@pytest.mark.parametrize("shape,density", [((1, 1), 1.0), ((300, 420), 0.01), ((1000, 700), 0.3), ((513, 129), 1.0)])
+def test_transposed_lists_dense(shape, density):
+    rng = np.random.default_rng(shape[0] + shape[1])
+    M = rng.random(shape) < density
+    _assert_cols_equal(bfa.plan_dense(_cuda(M)), [M])
+
+
+def test_transposed_lists_causal_8192_and_blockids():
+    M = np.tril(np.ones((8192, 8192), dtype=bool))
+    _assert_cols_equal(bfa.plan_dense(_cuda(M)), [M])
+    P = bfa.plan_blockids(B=2, Sq=700, Sk=650, window_left=100)
+    M2 = om.positional_dense(700, 650, True, 100)
+    _assert_cols_equal(P, [M2, M2])
+
+
+def test_transposed_lists_block_bits_and_predicates():
+    B, H, Sq, Skv, qb, kb = 2, 2, 450, 600, 32, 8
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    indptr, indices = _routing(B, H, nqb, nkb, 77)
+    P = bfa.plan_bsr(_cuda(indptr), _cuda(indices), Sq, Skv, qb, kb, causal=True)
+    D = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=True)
+    _assert_cols_equal(P, [D[b, h] for b in range(B) for h in range(H)])
+    terms = PRED_CASES["global64_window256"]
+    Pp = bfa.plan_predicate(terms, B=2, Sq=700, Sk=650)
+    Mp = om.predicate_dense(terms, 700, 650)
+    _assert_cols_equal(Pp, [Mp, Mp])

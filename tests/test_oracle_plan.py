@@ -131,3 +131,32 @@ def test_plan_stats_cover_grid():
     P = op.plan_masks(masks)
     assert sum(op.plan_stats(P)) == 3 * 3 + 1
     assert P["counts"][-1] == 0 and P["row_ptr"][-1] == P["kv_tile"].size
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_transposed_plan_lists_the_same_tiles_as_the_rows(seed):
+    rng = np.random.default_rng(seed)
+    masks = [rng.random((300, 420)) < 0.002, np.tril(np.ones((260, 260), dtype=bool)), rng.random((129, 77)) < 0.5]
+    plan = op.plan_masks(masks)
+    tp = op.transpose_plan(plan["cls"])
+    # brute force: column c of group g lists every query tile holding an attended pair of key tile kt
+    c = 0
+    r0 = 0
+    rows_pairs, cols_pairs = set(), set()
+    for g, M in enumerate(masks):
+        nqt, nkt = -(-M.shape[0] // 128), -(-M.shape[1] // 128)
+        for kt in range(nkt):
+            want = [qt for qt in range(nqt) if M[qt * 128:(qt + 1) * 128, kt * 128:(kt + 1) * 128].any()]
+            got = tp["q_tile"][tp["col_ptr"][c]:tp["col_ptr"][c + 1]].tolist()
+            assert got == want and tp["col_group"][c] == g and tp["col_kt"][c] == kt
+            for e, qt in enumerate(got):
+                blk = M[qt * 128:(qt + 1) * 128, kt * 128:(kt + 1) * 128]
+                assert tp["partial"][tp["col_ptr"][c] + e] == (0 if blk.all() else 1)
+                cols_pairs.add((g, qt, kt))
+            c += 1
+        for qt in range(nqt):
+            for e in range(plan["row_ptr"][r0 + qt], plan["row_ptr"][r0 + qt + 1]):
+                rows_pairs.add((g, qt, int(plan["kv_tile"][e])))
+        r0 += nqt
+    assert rows_pairs == cols_pairs
+    assert np.array_equal(tp["order"], np.lexsort((np.arange(len(tp["counts"])), -tp["counts"])))
