@@ -239,6 +239,29 @@ bfa_status bfa_fwd(const bfa_plan* plan, const void* q, const void* k, const voi
                    float* lse, void* stream);
 
 /*
+ * Backward of bfa_fwd (BinFlash: "Backward uses two passes (dKdV over K-blocks,
+ * dQ over Q-blocks)"; the LSE is the forward's auxiliary output that the
+ * backward reuses, tensorplay varlen): for an upstream gradient dout of `out`,
+ *   dV = P^T dO,  dS = P * (dO V^T - D),  D_i = dO_i . O_i,
+ *   dQ = scale dS K,  dK = scale dS^T Q,  P = exp(scale Q K^T - LSE) on attended pairs.
+ *   q, k, v, out, lse, scale, B, H, Hkv, D and the plan: exactly as given to (and
+ *   produced by) bfa_fwd.  dout: bf16, the layout of q (do_strides); dq, dk, dv:
+ *   caller-owned bf16 outputs shaped like q, k, v (their own strides), fully
+ *   written (rows that attend nothing, or keys nothing attends, get 0).  Under
+ *   GQA dk and dv sum over the query heads of each kv head.  All strides
+ *   {batch, token, head} in elements, multiples of 8; bases 16-byte aligned.
+ * The first call on a plan builds its transposed lists (bfa_plan_export_cols) on
+ * `stream`; a per-call workspace of 8 bytes per (replica, query-tile row) comes
+ * from the plan's stream-ordered pool.  Asynchronous; a device-side timeout is
+ * reported by bfa_plan_device_status().  Paged caches are not accepted here.
+ */
+bfa_status bfa_bwd(const bfa_plan* plan, const void* q, const void* k, const void* v, const void* out,
+                   const void* dout, const float* lse, const int64_t q_strides[3], const int64_t k_strides[3],
+                   const int64_t v_strides[3], const int64_t o_strides[3], const int64_t do_strides[3], int B, int H,
+                   int Hkv, int D, float scale, void* dq, void* dk, void* dv, const int64_t dq_strides[3],
+                   const int64_t dk_strides[3], const int64_t dv_strides[3], void* stream);
+
+/*
  * bfa_fwd with content-based block skipping (BinFlash approximate_softmax +
  * softmax_threshold, "BLASST-style"): once a query tile's scores are computed,
  * a key tile is dropped -- no exponentials, no P V product -- when every query

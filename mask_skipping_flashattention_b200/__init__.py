@@ -24,7 +24,7 @@ from . import _lib
 from ._lib import BfaError, PlanInfo
 
 __all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_predicate", "plan_bsr", "plan_block_bits",
-           "fwd", "fwd_paged",
+           "fwd", "bwd", "fwd_paged",
            "make_att_block_ids",
            "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "selftest_exp2", "library_path"]
 
@@ -347,6 +347,41 @@ def fwd(plan, q, k, v, scale=None, out=None, return_lse=True, lse=None, stream=N
                                      ctypes.c_float(float(softmax_threshold)), _ptr(out), _strides3(out), _ptr(lse),
                                      _stream(stream)))
     return out, lse
+
+
+def bwd(plan, q, k, v, out, dout, lse, scale=None, dq=None, dk=None, dv=None, stream=None):
+    """Gradients (dq, dk, dv) of ``fwd`` for an upstream gradient ``dout`` of ``out``.
+
+    q, k, v, the plan and scale exactly as given to ``fwd``; out and lse as it
+    returned them; dout shaped like q.  bf16 outputs shaped like q, k, v (dk and
+    dv sum over the query heads of each kv head under GQA).
+    """
+    for t in (q, k, v, out, dout):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("q, k, v, out, dout must be bfloat16")
+        if t.stride(-1) != 1:
+            raise ValueError("the head dim of q, k, v, out, dout must be contiguous")
+    if lse is None or lse.dtype != torch.float32:
+        raise TypeError("lse (float32, from fwd) is required")
+    if dout.shape != q.shape or out.shape != q.shape:
+        raise ValueError("out and dout must have the shape of q")
+    packed = q.dim() == 3
+    if packed:
+        B = plan.info["batch"]
+        _, H, D = q.shape
+        Hkv = k.shape[1]
+    else:
+        B, _, H, D = q.shape
+        Hkv = k.shape[2]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    sc = float(scale) if scale is not None else 0.0
+    _lib.check(_L.bfa_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse.contiguous()),
+                          _strides3(q), _strides3(k), _strides3(v), _strides3(out), _strides3(dout), int(B), int(H),
+                          int(Hkv), int(D), ctypes.c_float(sc), _ptr(dq), _ptr(dk), _ptr(dv), _strides3(dq),
+                          _strides3(dk), _strides3(dv), _stream(stream)))
+    return dq, dk, dv
 
 
 def fwd_paged(plan, q, k_cache, v_cache, block_table, scale=None, out=None, return_lse=True, lse=None, stream=None):

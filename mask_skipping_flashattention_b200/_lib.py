@@ -45,6 +45,9 @@ SIGNATURES = {
     "bfa_fwd": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_i64p, c_i64p, c_i64p, ctypes.c_int,
                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, c_void, c_i64p,
                                c_void, c_void]),
+    "bfa_bwd": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_i64p, c_i64p, c_i64p,
+                               c_i64p, c_i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                               c_void, c_void, c_void, c_i64p, c_i64p, c_i64p, c_void]),
     "bfa_fwd_approx": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_i64p, c_i64p, c_i64p, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_float,
                                       c_void, c_i64p, c_void, c_void]),

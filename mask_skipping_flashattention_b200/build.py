@@ -19,8 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbfa.so")
-SOURCES = ["planner.cu", "fwd.cu", "bfa_host.cu"]
-HEADERS = ["ptx.cuh", "plan_types.cuh", "fwd_params.cuh", "pred.cuh"]
+SOURCES = ["planner.cu", "fwd.cu", "bwd.cu", "bfa_host.cu"]
+HEADERS = ["ptx.cuh", "plan_types.cuh", "fwd_params.cuh", "pred.cuh", "tile_mask.cuh", "bwd_params.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-Xptxas", "-v",
          f"-I{os.path.join(ROOT, 'include')}"]

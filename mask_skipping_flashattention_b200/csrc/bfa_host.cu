@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/bfa.h"
+#include "bwd_params.cuh"
 #include "fwd_params.cuh"
 #include "plan_types.cuh"
 
@@ -962,6 +963,156 @@ bfa_status fwd_checked(const bfa_plan* P, const void* q, const void* k, const vo
 }
 
 }  // namespace
+
+namespace {
+
+// Backward: preprocess (D, LSE * log2 e) -> dQ pass over the plan's rows -> dK/dV
+// pass over its key-tile columns.  The workspace comes from the plan pool in
+// stream order and is returned after the kernels.
+bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const void* v, const void* out,
+                                const void* dout, const float* lse, const int64_t* qs, const int64_t* ks,
+                                const int64_t* vs, const int64_t* os, const int64_t* dos, int B, int H, int Hkv,
+                                int D, float scale, void* dq, void* dk, void* dv, const int64_t* dqs,
+                                const int64_t* dks, const int64_t* dvs, cudaStream_t st) {
+  std::string why;
+  const int bq = P->varlen ? 1 : B;
+  CUtensorMap tq, tdo, tk, tv;
+  if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], &why) ||
+      !make_tmap(&tdo, dout, D, H, P->sq, bq, dos[2], dos[1], dos[0], &why) ||
+      !make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], &why) ||
+      !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], &why))
+    return fail(BFA_ERR_INVALID_ARG, "%s", why.c_str());
+  bfa_status s = ensure_cols(P, st);
+  if (s != BFA_OK) return s;
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.plan.groups = P->groups;
+  p.plan.row_group = P->row_group;
+  p.plan.row_ptr = P->row_ptr;
+  p.plan.kv_tile = P->kv_tile;
+  p.plan.part = P->part;
+  p.plan.fine = P->fine;
+  p.plan.order = P->order;
+  p.plan.qid = P->qid;
+  p.plan.qvalid = P->qvalid;
+  p.plan.kid = P->kid;
+  p.plan.kbits = P->kbits;
+  p.plan.terms = P->terms;
+  p.plan.n_terms = P->n_terms;
+  p.plan.err = P->err;
+  p.plan.n_rows = P->n_rows;
+  p.plan.n_groups = P->n_groups;
+  p.plan.mask_mode = P->mask_mode;
+  p.plan.causal = P->causal;
+  p.plan.window = P->window;
+  p.plan.kind = P->kind;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? H / Hkv : H);
+  p.rep_kv = P->kind == BFA_PLAN_DENSE ? B * Hkv : (P->kind == BFA_PLAN_BSR ? 1 : Hkv);
+  const int n_cols = plan_n_cols(P);
+  const int64_t waves = 2LL * sm_count();
+  auto chunk_for = [&](int64_t units, int64_t items) {
+    return std::min<int64_t>(items, std::max<int64_t>(1, (waves + units - 1) / std::max<int64_t>(units, 1)));
+  };
+  p.head_chunk = static_cast<int>(chunk_for(P->n_rows, p.rep));
+  p.kv_chunk = static_cast<int>(chunk_for(n_cols, p.rep_kv));
+  p.varlen = P->varlen;
+  p.Sq_lse = P->sq;
+  const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.out = static_cast<const __nv_bfloat16*>(out);
+  p.o_sb = P->varlen ? 0 : os[0];
+  p.o_ss = os[1];
+  p.o_sh = os[2];
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.do_sb = P->varlen ? 0 : dos[0];
+  p.do_ss = dos[1];
+  p.do_sh = dos[2];
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dq_sb = P->varlen ? 0 : dqs[0];
+  p.dq_ss = dqs[1];
+  p.dq_sh = dqs[2];
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dk_sb = P->varlen ? 0 : dks[0];
+  p.dk_ss = dks[1];
+  p.dk_sh = dks[2];
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dv_sb = P->varlen ? 0 : dvs[0];
+  p.dv_ss = dvs[1];
+  p.dv_sh = dvs[2];
+  p.col0 = P->col0;
+  p.col_group = P->col_group;
+  p.col_ptr = P->col_ptr;
+  p.q_tile = P->q_tile;
+  p.tpart = P->tpart;
+  p.col_order = P->col_order;
+  p.n_cols = n_cols;
+  p.wait_ns = g_wait_ns;
+  const int64_t ws_rows = static_cast<int64_t>(p.rep) * P->n_rows * kTile;
+  void* ws = nullptr;
+  auto cleanup = [&]() {
+    if (ws) cudaFreeAsync(ws, st);
+  };
+  if (ws_rows > 0) {
+    cudaMemPool_t pool;
+    BFA_CUDA(plan_pool(&pool), "plan memory pool");
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(ws_rows) * 2 * sizeof(float), pool, st);
+    if (e != cudaSuccess) {
+      ws = nullptr;
+      return fail(BFA_ERR_CAPACITY, "backward workspace of %lld bytes: %s", (long long)(ws_rows * 8),
+                  cudaGetErrorString(e));
+    }
+    p.ws_lse2 = static_cast<float*>(ws);
+    p.ws_d = p.ws_lse2 + ws_rows;
+  }
+  BFA_CUDA(launch_bwd_prep(p, st), "backward preprocess kernel");
+  BFA_CUDA(launch_bwd_dq(D, tq, tdo, tk, tv, p, static_cast<int64_t>(P->n_rows) * p.rep, st), "dQ kernel");
+  BFA_CUDA(launch_bwd_dkdv(D, tk, tv, tq, tdo, p, static_cast<int64_t>(n_cols) * p.rep_kv, st), "dK/dV kernel");
+  cleanup();
+  return BFA_OK;
+}
+
+}  // namespace
+
+BFA_API bfa_status bfa_bwd(const bfa_plan* Pc, const void* q, const void* k, const void* v, const void* out,
+                           const void* dout, const float* lse, const int64_t qs[3], const int64_t ks[3],
+                           const int64_t vs[3], const int64_t os[3], const int64_t dos[3], int B, int H, int Hkv,
+                           int D, float scale, void* dq, void* dk, void* dv, const int64_t dqs[3],
+                           const int64_t dks[3], const int64_t dvs[3], void* stream) {
+  if (!Pc) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
+  bfa_plan* P = const_cast<bfa_plan*>(Pc);  // the transposed lists are a cache of the plan
+  if (!qs || !ks || !vs || !os || !dos || !dqs || !dks || !dvs) return fail(BFA_ERR_INVALID_ARG, "strides are NULL");
+  if (D != 64 && D != 128) return fail(BFA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", D);
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0) return fail(BFA_ERR_INVALID_ARG, "H=%d must be a positive multiple of Hkv=%d", H, Hkv);
+  if (B <= 0) return fail(BFA_ERR_INVALID_ARG, "B=%d must be positive", B);
+  if (P->kind != BFA_PLAN_DENSE && B != P->batch)
+    return fail(BFA_ERR_INVALID_ARG, "B=%d does not match the plan's %d", B, P->batch);
+  if (P->kind == BFA_PLAN_BSR && Hkv != P->hkv)
+    return fail(BFA_ERR_INVALID_ARG, "Hkv=%d does not match the BSR routing's %d", Hkv, P->hkv);
+  if (!lse) return fail(BFA_ERR_INVALID_ARG, "lse is required by the backward");
+  bfa_status s;
+  if ((s = need_device(q, "q")) || (s = need_device(k, "k")) || (s = need_device(v, "v")) ||
+      (s = need_device(out, "out")) || (s = need_device(dout, "dout")) || (s = need_device(lse, "lse")) ||
+      (s = need_device(dq, "dq")) || (s = need_device(dk, "dk")) || (s = need_device(dv, "dv")))
+    return s;
+  const int64_t* all[8] = {qs, ks, vs, os, dos, dqs, dks, dvs};
+  for (int t = 0; t < 8; ++t)
+    for (int i = 0; i < 3; ++i) {
+      if (P->varlen && i == 0) continue;
+      if (all[t][i] < 0 || all[t][i] % 8 != 0)
+        return fail(BFA_ERR_INVALID_ARG, "stride %lld is not a non-negative multiple of 8 elements", (long long)all[t][i]);
+    }
+  const void* ptrs[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (int t = 0; t < 8; ++t)
+    if (reinterpret_cast<uintptr_t>(ptrs[t]) & 15u) return fail(BFA_ERR_INVALID_ARG, "tensor base is not 16-byte aligned");
+  return bwd_launch_from_host(P, q, k, v, out, dout, lse, qs, ks, vs, os, dos, B, H, Hkv, D, scale, dq, dk, dv, dqs,
+                              dks, dvs, static_cast<cudaStream_t>(stream));
+}
 
 BFA_API bfa_status bfa_fwd(const bfa_plan* P, const void* q, const void* k, const void* v, const int64_t qs[3],
                            const int64_t ks[3], const int64_t vs[3], int B, int H, int Hkv, int D, float scale,

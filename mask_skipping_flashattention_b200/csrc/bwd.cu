@@ -1,0 +1,666 @@
+// Backward of the mask-aware attention for sm_100a: gradients of
+//   O = softmax(scale Q K^T + mask) V
+// with respect to Q, K and V for an upstream gradient dO, reusing the forward's
+// plan and LSE (BinFlash: "Backward uses two passes (dKdV over K-blocks, dQ over
+// Q-blocks) with the same gathered-dispatch machinery"; tensorplay varlen: the
+// log-sum-exp is the auxiliary output "that the backward pass reuses").
+//
+// With P = exp(scale S - LSE) (S = Q K^T, masked pairs 0), dP = dO V^T and
+// D_i = dO_i . O_i, the score gradient is dS = P * (dP - D), and
+//   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Three kernels:
+//   k_bwd_prep  per query row: D = dO . O and LSE * log2(e) into a workspace
+//               padded to whole tiles (HBM-bound, one pass over O and dO);
+//   k_bwd_dq    one CTA per (plan row, replica), walking the row's key-tile list:
+//               S = Q K^T and dP = dO V^T (SS), dS into TMEM as bf16, dQ += dS K
+//               (TS); the mask on partial and edge tiles only;
+//   k_bwd_dkdv  one CTA per (key-tile column, kv replica), walking the column's
+//               query-tile list for every query head of the kv head (GQA sums in
+//               TMEM, no atomics): S^T = K Q^T and dP^T = V dO^T (SS), P^T and dS^T
+//               into TMEM as bf16, dV += P^T dO and dK += dS^T Q (TS).
+// Warp roles of the two tile kernels (256 threads): warp 0 TMA producer, warp 1
+// TMEM owner and single-thread tcgen05.mma issuer, warps 4..7 one tile row per
+// thread (query rows in k_bwd_dq, key rows in k_bwd_dkdv).  Every wait is
+// bounded.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bwd_params.cuh"
+#include "plan_types.cuh"
+#include "ptx.cuh"
+#include "tile_mask.cuh"
+
+namespace bfa {
+
+using namespace ptx;
+
+namespace {
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdStages = 2;
+
+template <int D>
+struct BCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kVecBytes = 2 * kTile * 4;  // LSE * log2(e) and D of one query tile
+  // two resident tiles, then kBwdStages stages of two tiles (+ the vectors in k_bwd_dkdv)
+  static constexpr int kSmemBytes = (2 + 2 * kBwdStages) * kTileBytes + kBwdStages * kVecBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdescNN = idesc_bf16_f32(128, 128, 0);  // both operands K-major, N = 128
+  static constexpr uint32_t kIdescD = idesc_bf16_f32(128, D, 1);     // B MN-major, N = D
+};
+
+// Context of one group's tile for the mask functions of tile_mask.cuh.
+struct GroupCtx {
+  int32_t q_len, k_len, qid_off, kid_off, kbit_off;
+};
+
+__device__ __forceinline__ GroupCtx group_ctx(const GroupInfo& g) {
+  GroupCtx c;
+  c.q_len = g.q_len;
+  c.k_len = g.k_len;
+  c.qid_off = g.qid_off;
+  c.kid_off = g.kid_off;
+  c.kbit_off = g.kbit_off;
+  return c;
+}
+
+// replica index -> (batch, head) of a plan row (as in the forward)
+__device__ __forceinline__ void replica_bh(const BwdParams& p, const GroupInfo& g, int j, int& b, int& h) {
+  if (p.plan.kind == 1 /*BFA_PLAN_DENSE*/) {
+    b = j / p.H;
+    h = j % p.H;
+  } else if (p.plan.kind == 4 /*BFA_PLAN_BSR*/) {
+    b = g.b;
+    h = g.hkv * (p.H / p.Hkv) + j;
+  } else {
+    b = p.varlen ? 0 : g.b;
+    h = j;
+  }
+}
+
+// (batch, head) -> replica index of the workspace
+__device__ __forceinline__ int replica_of(const BwdParams& p, const GroupInfo& g, int b, int h) {
+  if (p.plan.kind == 1) return b * p.H + h;
+  if (p.plan.kind == 4) return h - g.hkv * (p.H / p.Hkv);
+  return h;
+}
+
+// kv replica index -> (batch, kv head) of a key-tile column
+__device__ __forceinline__ void kv_replica_bh(const BwdParams& p, const GroupInfo& g, int j, int& b, int& hk) {
+  if (p.plan.kind == 1) {
+    b = j / p.Hkv;
+    hk = j % p.Hkv;
+  } else if (p.plan.kind == 4) {
+    b = g.b;
+    hk = g.hkv;
+  } else {
+    b = p.varlen ? 0 : g.b;
+    hk = j;
+  }
+}
+
+// work item -> (unit in longest-first order, replica), chunked so a chunk's
+// replicas of consecutive units run together (keys / values or queries in L2)
+__device__ __forceinline__ void chunked_decode(int64_t w, int64_t units, int64_t items, int64_t chunk, int& i, int& j) {
+  const int64_t hg = w / (units * chunk);
+  const int64_t rem = w - hg * units * chunk;
+  const int64_t gs = min(chunk, items - hg * chunk);
+  i = static_cast<int>(rem / gs);
+  j = static_cast<int>(hg * chunk + rem % gs);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_nn(uint32_t tD, const uint8_t* sA, const uint8_t* sB) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    umma_ss(tD, smem_desc(smem_u32(sA + off), 16, 1024), smem_desc(smem_u32(sB + off), 16, 1024), BCfg<D>::kIdescNN,
+            kk > 0);
+  }
+}
+
+// D (tmem, N = D columns) (+)= A (tmem, bf16 128 x 128) * B (smem tile, rows = the K axis)
+template <int D>
+__device__ __forceinline__ void issue_td(uint32_t tD, uint32_t tA, const uint8_t* sB, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    umma_ts(tD, tA + kk * 8, smem_desc(smem_u32(sB + kk * 2048), 16384, 1024), BCfg<D>::kIdescD,
+            (acc || kk > 0) ? 1u : 0u);
+}
+
+// fp32 accumulator row (TMEM, D columns) * scale -> bf16 row in global memory
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t tAcc, bool have, float scale, __nv_bfloat16* dst, bool store) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    if (have) {
+      tmem_ld_32x32b_x32(tAcc + cc * 32, o);
+      tmem_wait_ld();
+      reg_fence(o);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) o[j] = 0u;
+    }
+    uint32_t pkd[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      pkd[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * scale, __uint_as_float(o[2 * j + 1]) * scale);
+    if (store) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d4[j] = make_uint4(pkd[4 * j], pkd[4 * j + 1], pkd[4 * j + 2], pkd[4 * j + 3]);
+    }
+  }
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------------------
+// preprocess: D = dO . O and LSE * log2(e), per (replica, plan row, tile row)
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) k_bwd_prep(const BwdParams p) {
+  const int64_t blk = blockIdx.x;
+  const int r = static_cast<int>(blk % p.plan.n_rows);
+  const int j = static_cast<int>(blk / p.plan.n_rows);
+  const GroupInfo g = p.plan.groups[p.plan.row_group[r]];
+  int b, h;
+  replica_bh(p, g, j, b, h);
+  const int qpos = (r - g.row0) * kTile + threadIdx.x;
+  float dval = 0.f, lse2 = 0.f;
+  if (qpos < g.q_len) {
+    const int64_t tok = static_cast<int64_t>(g.q_off) + qpos;
+    const uint4* o4 = reinterpret_cast<const uint4*>(p.out + static_cast<int64_t>(b) * p.o_sb + tok * p.o_ss +
+                                                     static_cast<int64_t>(h) * p.o_sh);
+    const uint4* d4 = reinterpret_cast<const uint4*>(p.dout + static_cast<int64_t>(b) * p.do_sb + tok * p.do_ss +
+                                                     static_cast<int64_t>(h) * p.do_sh);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 a = __ldg(o4 + c), z = __ldg(d4 + c);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, zv[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+        const float2 fz = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zv[e]));
+        acc[e] = fmaf(fa.x, fz.x, acc[e]);
+        acc[e] = fmaf(fa.y, fz.y, acc[e]);
+      }
+    }
+    dval = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    const int64_t li = p.varlen ? static_cast<int64_t>(h) * p.Sq_lse + tok
+                                : (static_cast<int64_t>(b) * p.H + h) * p.Sq_lse + qpos;
+    const float L = p.lse[li];
+    lse2 = (L == -INFINITY) ? 0.f : L * 1.4426950408889634f;  // a row that attends nothing has no listed pair
+  }
+  const int64_t wi = (static_cast<int64_t>(j) * p.plan.n_rows + r) * kTile + threadIdx.x;
+  p.ws_lse2[wi] = lse2;
+  p.ws_d[wi] = dval;
+}
+
+// ----------------------------------------------------------------------------
+// dQ pass: one CTA per (plan row, replica), over the row's key-tile list
+// ----------------------------------------------------------------------------
+struct DqWork {
+  GroupInfo g;
+  int32_t r, e0, n, qt, b, h, hk, j;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+             const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const BwdParams p) {
+  using C = BCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* const sQ = smem;
+  uint8_t* const sdO = smem + C::kTileBytes;
+  uint8_t* const sK0 = smem + 2 * C::kTileBytes;
+  uint8_t* const sV0 = smem + (2 + kBwdStages) * C::kTileBytes;
+  // BQ: Q and dO.  BF / BE [2]: K, V stage full / free.  BS: S and dP of the
+  // current tile ready.  BP: dS written (4 warps).  BO: every product done.
+  enum { BQ = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 7, BDONE = 8, NBAR = 9 };
+  __shared__ __align__(8) uint64_t bars[NBAR];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ DqWork wk_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto sK = [&](int st) { return sK0 + st * C::kTileBytes; };
+  auto sV = [&](int st) { return sV0 + st * C::kTileBytes; };
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), i == BP ? 4 : 1);
+    fence_barrier_init();
+    int i, j;
+    chunked_decode(blockIdx.x, p.plan.n_rows, p.rep, p.head_chunk, i, j);
+    const int r = p.plan.order[i];
+    DqWork w;
+    w.g = p.plan.groups[p.plan.row_group[r]];
+    w.r = r;
+    w.e0 = p.plan.row_ptr[r];
+    w.n = p.plan.row_ptr[r + 1] - w.e0;
+    w.qt = r - w.g.row0;
+    w.j = j;
+    replica_bh(p, w.g, j, w.b, w.h);
+    w.hk = w.h / (p.H / p.Hkv);
+    wk_s = w;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const DqWork& wk = wk_s;
+  const uint64_t cap = p.wait_ns;
+  const int n = wk.n;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmdO);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int qs = wk.g.q_off + wk.qt * kTile;
+      mbar_expect_tx(bar(BQ), 2 * C::kTileBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_4d(smem_u32(sQ + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h, qs, wk.b);
+        tma_load_4d(smem_u32(sdO + pn * 16384), &tmdO, bar(BQ), pn * 64, wk.h, qs, wk.b);
+      }
+      const int32_t* kv = p.plan.kv_tile + wk.e0;
+      int last[kBwdStages] = {-1, -1};
+      int kt_next = kv[0];
+      for (int u = 0; u < n; ++u) {
+        const int kt = kt_next;
+        if (u + 1 < n) kt_next = kv[u + 1];
+        const int st = u & 1;
+        if (u >= kBwdStages && !mbar_wait_fast(bar(BE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
+        const uint32_t f = bar(BF + st);
+        mbar_expect_tx(f, 2 * C::kTileBytes);
+        const int ks = wk.g.k_off + kt * kTile;
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_4d(smem_u32(sK(st) + pn * 16384), &tmK, f, pn * 64, wk.hk, ks, wk.b);
+          tma_load_4d(smem_u32(sV(st) + pn * 16384), &tmV, f, pn * 64, wk.hk, ks, wk.b);
+        }
+        last[st] = u;
+      }
+      volatile int no_abort = 0;
+      mbar_wait_fast(bar(BQ), 0, cap, &no_abort);
+      for (int st = 0; st < kBwdStages; ++st)
+        if (last[st] >= 0) mbar_wait_fast(bar(BF + st), (last[st] >> 1) & 1, cap, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+      bool ok = mbar_wait_fast(bar(BQ), 0, cap, &abort_flag);
+      bool started = false;
+      for (int u = 0; ok && u < n; ++u) {
+        const int st = u & 1;
+        if (!mbar_wait_fast(bar(BF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_nn<D>(tS, sQ, sK(st));    // S = Q K^T (over the dS of tile u - 1, in issue order)
+        issue_nn<D>(tdP, sdO, sV(st));  // dP = dO V^T
+        umma_commit(bar(BS));
+        if (!mbar_wait_fast(bar(BP), u & 1, cap, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_td<D>(tdQ, tS, sK(st), started);  // dQ += dS K
+        started = true;
+        umma_commit(bar(BE + st));
+      }
+      if (ok) umma_commit(bar(BO));
+      umma_commit(bar(BDONE));
+      volatile int no_abort = 0;
+      mbar_wait_fast(bar(BDONE), 0, cap, &no_abort);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ dS rows
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int qpos = wk.qt * kTile + row;
+    const uint32_t tLane = tmem_addr(tmem, quarter * 32, 0);
+    const GroupCtx ctx = group_ctx(wk.g);
+    const int64_t wi = (static_cast<int64_t>(wk.j) * p.plan.n_rows + wk.r) * kTile + row;
+    const float lse2 = p.ws_lse2[wi], dval = p.ws_d[wi];
+    const float c = p.scale_log2;
+    bool ok = true;
+    int kt_next = n > 0 ? p.plan.kv_tile[wk.e0] : 0;
+    int part_next = n > 0 ? p.plan.part[wk.e0] : -1;
+    for (int u = 0; u < n; ++u) {
+      const int kt = kt_next, part = part_next;
+      if (u + 1 < n) {
+        kt_next = p.plan.kv_tile[wk.e0 + u + 1];
+        part_next = p.plan.part[wk.e0 + u + 1];
+      }
+      uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (part >= 0 || (kt + 1) * kTile > wk.g.k_len) row_mask_words(p.plan, ctx, qpos, row, kt, part, am);
+      const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
+      if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sv[32], dp[32];
+        tmem_ld_32x32b_x32(tLane + cc * 32, sv);
+        tmem_ld_32x32b_x32(tLane + 128 + cc * 32, dp);
+        tmem_wait_ld();
+        reg_fence(sv);
+        reg_fence(dp);
+        const uint32_t bits = am[cc];
+        uint32_t pk[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int c0 = 2 * jj, c1 = 2 * jj + 1;
+          const float p0 = ((bits >> c0) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[c0]), c, -lse2)) : 0.f;
+          const float p1 = ((bits >> c1) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[c1]), c, -lse2)) : 0.f;
+          pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dp[c0]) - dval), p1 * (__uint_as_float(dp[c1]) - dval));
+        }
+        tmem_st_32x32b_x16(tLane + cc * 16, pk);  // dS over S columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BP));
+    }
+    bool done = ok;
+    if (ok && n > 0) {
+      const bool got = mbar_wait(bar(BO), 0, cap, &abort_flag);
+      done = !__any_sync(0xffffffffu, !got);
+    }
+    tc_fence_after();
+    if (done) {
+      const int64_t tok = static_cast<int64_t>(wk.g.q_off) + qpos;
+      __nv_bfloat16* dst =
+          p.dq + static_cast<int64_t>(wk.b) * p.dq_sb + tok * p.dq_ss + static_cast<int64_t>(wk.h) * p.dq_sh;
+      store_row<D>(tLane + 256, n > 0, p.scale, dst, qpos < wk.g.q_len);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_flag && threadIdx.x == 0) atomicOr(p.plan.err, DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// dK / dV pass: one CTA per (key-tile column, kv replica), over the column's
+// query tiles for every query head that reads the kv head
+// ----------------------------------------------------------------------------
+struct KvWork {
+  GroupInfo g;
+  int32_t kt, e0, nq, nh, b, hk, steps;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    k_bwd_dkdv(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
+  using C = BCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* const sK = smem;
+  uint8_t* const sV = smem + C::kTileBytes;
+  uint8_t* const sQ0 = smem + 2 * C::kTileBytes;                      // + 2 st tiles
+  float* const sVec0 = reinterpret_cast<float*>(smem + (2 + 2 * kBwdStages) * C::kTileBytes);  // + st * 256
+  // BKV: K and V.  BF / BE [2]: Q, dO and the query vectors of a step full /
+  // free.  BS: S^T and dP^T ready.  BP: P^T and dS^T written (4 warps).  BO:
+  // every product done.
+  enum { BKV = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 7, BDONE = 8, NBAR = 9 };
+  __shared__ __align__(8) uint64_t bars[NBAR];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ KvWork wk_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto sQ = [&](int st) { return sQ0 + (2 * st) * C::kTileBytes; };
+  auto sdO = [&](int st) { return sQ0 + (2 * st + 1) * C::kTileBytes; };
+  auto sVec = [&](int st) { return sVec0 + st * 2 * kTile; };  // [lse2 x 128][D x 128]
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), i == BP ? 4 : 1);
+    fence_barrier_init();
+    int i, jk;
+    chunked_decode(blockIdx.x, p.n_cols, p.rep_kv, p.kv_chunk, i, jk);
+    const int c = p.col_order[i];
+    const int grp = p.col_group[c];
+    KvWork w;
+    w.g = p.plan.groups[grp];
+    w.kt = c - p.col0[grp];
+    w.e0 = p.col_ptr[c];
+    w.nq = p.col_ptr[c + 1] - w.e0;
+    w.nh = p.H / p.Hkv;
+    kv_replica_bh(p, w.g, jk, w.b, w.hk);
+    w.steps = w.nq * w.nh;
+    wk_s = w;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const KvWork& wk = wk_s;
+  const uint64_t cap = p.wait_ns;
+  const int steps = wk.steps;
+  // step s -> query head and list entry
+  auto step_head = [&](int s) { return wk.hk * wk.nh + s / wk.nq; };
+  auto step_entry = [&](int s) { return wk.e0 + s % wk.nq; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && steps > 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmdO);
+      const int ks = wk.g.k_off + wk.kt * kTile;
+      mbar_expect_tx(bar(BKV), 2 * C::kTileBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_4d(smem_u32(sK + pn * 16384), &tmK, bar(BKV), pn * 64, wk.hk, ks, wk.b);
+        tma_load_4d(smem_u32(sV + pn * 16384), &tmV, bar(BKV), pn * 64, wk.hk, ks, wk.b);
+      }
+      int last[kBwdStages] = {-1, -1};
+      for (int s = 0; s < steps; ++s) {
+        const int st = s & 1;
+        if (s >= kBwdStages && !mbar_wait_fast(bar(BE + st), ((s >> 1) - 1) & 1, cap, &abort_flag)) break;
+        const int h = step_head(s);
+        const int qt = p.q_tile[step_entry(s)];
+        const int r = wk.g.row0 + qt;
+        const int64_t wi = (static_cast<int64_t>(replica_of(p, wk.g, wk.b, h)) * p.plan.n_rows + r) * kTile;
+        const uint32_t f = bar(BF + st);
+        mbar_expect_tx(f, 2 * C::kTileBytes + C::kVecBytes);
+        const int qs = wk.g.q_off + qt * kTile;
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_4d(smem_u32(sQ(st) + pn * 16384), &tmQ, f, pn * 64, h, qs, wk.b);
+          tma_load_4d(smem_u32(sdO(st) + pn * 16384), &tmdO, f, pn * 64, h, qs, wk.b);
+        }
+        bulk_load(smem_u32(sVec(st)), p.ws_lse2 + wi, kTile * 4, f);
+        bulk_load(smem_u32(sVec(st) + kTile), p.ws_d + wi, kTile * 4, f);
+        last[st] = s;
+      }
+      volatile int no_abort = 0;
+      mbar_wait_fast(bar(BKV), 0, cap, &no_abort);
+      for (int st = 0; st < kBwdStages; ++st)
+        if (last[st] >= 0) mbar_wait_fast(bar(BF + st), (last[st] >> 1) & 1, cap, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && steps > 0) {
+      const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+      bool ok = mbar_wait_fast(bar(BKV), 0, cap, &abort_flag);
+      bool started = false;
+      for (int s = 0; ok && s < steps; ++s) {
+        const int st = s & 1;
+        if (!mbar_wait_fast(bar(BF + st), (s >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_nn<D>(tS, sK, sQ(st));    // S^T = K Q^T (over P^T of step s - 1, in issue order)
+        issue_nn<D>(tdP, sV, sdO(st));  // dP^T = V dO^T
+        umma_commit(bar(BS));
+        if (!mbar_wait_fast(bar(BP), s & 1, cap, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        issue_td<D>(tdV, tS, sdO(st), started);  // dV += P^T dO
+        issue_td<D>(tdK, tdP, sQ(st), started);  // dK += dS^T Q
+        started = true;
+        umma_commit(bar(BE + st));
+      }
+      if (ok) umma_commit(bar(BO));
+      umma_commit(bar(BDONE));
+      volatile int no_abort = 0;
+      mbar_wait_fast(bar(BDONE), 0, cap, &no_abort);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ P^T, dS^T rows (one key per thread)
+    const int quarter = warp & 3;
+    const int krow = quarter * 32 + lane;
+    const int kpos = wk.kt * kTile + krow;
+    const uint32_t tLane = tmem_addr(tmem, quarter * 32, 0);
+    const GroupCtx ctx = group_ctx(wk.g);
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < steps; ++s) {
+      const int st = s & 1;
+      const int e = step_entry(s);
+      const int qt = p.q_tile[e], part = p.tpart[e];
+      uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (part >= 0 || (qt + 1) * kTile > wk.g.q_len) col_mask_words(p.plan, ctx, kpos, krow, qt, part, am);
+      // the step's query vectors (bulk copy on BF) and its S^T, dP^T (BS)
+      const bool gv = mbar_wait(bar(BF + st), (s >> 1) & 1, cap, &abort_flag);
+      const bool gs = gv && mbar_wait(bar(BS), s & 1, cap, &abort_flag);
+      if (__any_sync(0xffffffffu, !gs)) { ok = false; break; }
+      tc_fence_after();
+      const float* lse2 = sVec(st);
+      const float* dvec = sVec(st) + kTile;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sv[32], dp[32];
+        tmem_ld_32x32b_x32(tLane + cc * 32, sv);
+        tmem_ld_32x32b_x32(tLane + 128 + cc * 32, dp);
+        tmem_wait_ld();
+        reg_fence(sv);
+        reg_fence(dp);
+        const uint32_t bits = am[cc];
+        uint32_t pkp[16], pks[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 L = *reinterpret_cast<const float4*>(lse2 + cc * 32 + q4 * 4);
+          const float4 Dv = *reinterpret_cast<const float4*>(dvec + cc * 32 + q4 * 4);
+          const float Ls[4] = {L.x, L.y, L.z, L.w}, Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int col = q4 * 4 + t;
+            pv[t] = ((bits >> col) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[col]), c, -Ls[t])) : 0.f;
+            dsv[t] = pv[t] * (__uint_as_float(dp[col]) - Ds[t]);
+          }
+          pkp[2 * q4] = pack_bf16x2(pv[0], pv[1]);
+          pkp[2 * q4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          pks[2 * q4] = pack_bf16x2(dsv[0], dsv[1]);
+          pks[2 * q4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        }
+        tmem_st_32x32b_x16(tLane + cc * 16, pkp);        // P^T over S^T columns already read
+        tmem_st_32x32b_x16(tLane + 128 + cc * 16, pks);  // dS^T over dP^T columns already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BP));
+    }
+    bool done = ok;
+    if (ok && steps > 0) {
+      const bool got = mbar_wait(bar(BO), 0, cap, &abort_flag);
+      done = !__any_sync(0xffffffffu, !got);
+    }
+    tc_fence_after();
+    if (done) {
+      const bool store = kpos < wk.g.k_len;
+      const int64_t tok = static_cast<int64_t>(wk.g.k_off) + kpos;
+      __nv_bfloat16* dvp =
+          p.dv + static_cast<int64_t>(wk.b) * p.dv_sb + tok * p.dv_ss + static_cast<int64_t>(wk.hk) * p.dv_sh;
+      __nv_bfloat16* dkp =
+          p.dk + static_cast<int64_t>(wk.b) * p.dk_sb + tok * p.dk_ss + static_cast<int64_t>(wk.hk) * p.dk_sh;
+      store_row<D>(tLane + 256, steps > 0, 1.f, dvp, store);
+      store_row<D>(tLane + 256 + D, steps > 0, p.scale, dkp, store);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_flag && threadIdx.x == 0) atomicOr(p.plan.err, DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// launchers (host)
+// ----------------------------------------------------------------------------
+int bwd_smem_bytes(int D) { return D == 64 ? BCfg<64>::kSmemBytes : BCfg<128>::kSmemBytes; }
+
+cudaError_t launch_bwd_prep(const BwdParams& p, cudaStream_t s) {
+  const int64_t blocks = static_cast<int64_t>(p.rep) * p.plan.n_rows;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (p.D == 64) k_bwd_prep<64><<<static_cast<unsigned>(blocks), 128, 0, s>>>(p);
+  else k_bwd_prep<128><<<static_cast<unsigned>(blocks), 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename K>
+static cudaError_t bwd_prepare(K kernel, int smem) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const BwdParams& p, int64_t n_work, cudaStream_t s) {
+  if (n_work <= 0) return cudaSuccess;
+  if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (D == 64) {
+    static cudaError_t ready = bwd_prepare(k_bwd_dq<64>, BCfg<64>::kSmemBytes);
+    if (ready != cudaSuccess) return ready;
+    k_bwd_dq<64><<<static_cast<unsigned>(n_work), kBwdThreads, BCfg<64>::kSmemBytes, s>>>(tq, tdo, tk, tv, p);
+  } else {
+    static cudaError_t ready = bwd_prepare(k_bwd_dq<128>, BCfg<128>::kSmemBytes);
+    if (ready != cudaSuccess) return ready;
+    k_bwd_dq<128><<<static_cast<unsigned>(n_work), kBwdThreads, BCfg<128>::kSmemBytes, s>>>(tq, tdo, tk, tv, p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv(int D, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                            const CUtensorMap& tdo, const BwdParams& p, int64_t n_work, cudaStream_t s) {
+  if (n_work <= 0) return cudaSuccess;
+  if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (D == 64) {
+    static cudaError_t ready = bwd_prepare(k_bwd_dkdv<64>, BCfg<64>::kSmemBytes);
+    if (ready != cudaSuccess) return ready;
+    k_bwd_dkdv<64><<<static_cast<unsigned>(n_work), kBwdThreads, BCfg<64>::kSmemBytes, s>>>(tk, tv, tq, tdo, p);
+  } else {
+    static cudaError_t ready = bwd_prepare(k_bwd_dkdv<128>, BCfg<128>::kSmemBytes);
+    if (ready != cudaSuccess) return ready;
+    k_bwd_dkdv<128><<<static_cast<unsigned>(n_work), kBwdThreads, BCfg<128>::kSmemBytes, s>>>(tk, tv, tq, tdo, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace bfa

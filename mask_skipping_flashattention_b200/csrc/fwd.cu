@@ -36,6 +36,7 @@
 #include "plan_types.cuh"
 #include "pred.cuh"
 #include "ptx.cuh"
+#include "tile_mask.cuh"
 
 namespace bfa {
 
@@ -188,71 +189,6 @@ struct UnionWalk {
     return true;
   }
 };
-
-// attend-bits of one query row (position qpos in its group) against the 128
-// columns of key tile `kt`
-__device__ __forceinline__ void row_mask_words(const FwdParams& p, const Work& wk, int qpos, int row, int kt,
-                                               int part, uint32_t (&am)[4]) {
-  const int ncols = wk.k_len - kt * kTile;  // in-range columns (may exceed 128)
-  if (p.plan.mask_mode == MASK_BITS) {
-    if (part >= 0) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.plan.fine + static_cast<int64_t>(part) * kFineWordsPerTile +
-                                                           row * kWordsPerTileRow));
-      am[0] = v.x; am[1] = v.y; am[2] = v.z; am[3] = v.w;
-    } else {
-      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
-    }
-  } else if (p.plan.mask_mode == MASK_BLOCKID) {
-    if (part >= 0) {
-      const int32_t qb = p.plan.qid[wk.qid_off + qpos];
-      const bool qv = p.plan.qvalid[wk.qid_off + qpos] != 0;
-      const int4* kb4 = reinterpret_cast<const int4*>(p.plan.kid + wk.kid_off + kt * kTile);
-      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(p.plan.kbits + wk.kbit_off + kt * kWordsPerTileRow));
-      const uint32_t kvw[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t bits = 0;
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const int4 k = __ldg(kb4 + w * 8 + c4);
-          bits |= (k.x <= qb ? 1u : 0u) << (c4 * 4 + 0);
-          bits |= (k.y <= qb ? 1u : 0u) << (c4 * 4 + 1);
-          bits |= (k.z <= qb ? 1u : 0u) << (c4 * 4 + 2);
-          bits |= (k.w <= qb ? 1u : 0u) << (c4 * 4 + 3);
-        }
-        am[w] = qv ? (bits & kvw[w]) : 0u;
-      }
-    } else {
-      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
-    }
-  } else if (p.plan.mask_mode == MASK_PRED) {
-    if (part >= 0) {
-      pred_words(p.plan.terms, p.plan.n_terms, qpos, kt, wk.k_len, am);
-    } else {
-      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
-    }
-  } else {  // MASK_POS: causal kv_pos <= q_pos, optional window q_pos - kv_pos < W
-    int hi = p.plan.causal ? (qpos - kt * kTile) : 127;                           // last attended column
-    int lo = (p.plan.window >= 0) ? (qpos - kt * kTile - p.plan.window + 1) : 0;  // first attended column
-    if (part < 0) { hi = 127; lo = 0; }
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int a = lo - 32 * w, z = hi - 32 * w;  // attended range inside this word
-      uint32_t m_hi = (z >= 31) ? 0xffffffffu : (z < 0 ? 0u : ((2u << z) - 1u));
-      uint32_t m_lo = (a <= 0) ? 0xffffffffu : (a > 31 ? 0u : ~((1u << a) - 1u));
-      am[w] = m_hi & m_lo;
-    }
-  }
-  // key tokens past the group's end (edge tile) are never attended
-  if (ncols < kTile) {
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int z = ncols - 32 * w;
-      const uint32_t m = (z >= 32) ? 0xffffffffu : (z <= 0 ? 0u : ((1u << z) - 1u));
-      am[w] &= m;
-    }
-  }
-}
 
 // TMA of one 128-token K or V tile (all D/64 panels) into `dst`, completing on
 // `bar`.  Contiguous layouts take one box per panel at token row `ks`; paged
@@ -504,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool masked = part >= 0 || (kt + 1) * kTile > wk.k_len;
         uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        if (masked) row_mask_words(p, wk, qpos, row, kt, part, am);
+        if (masked) row_mask_words(p.plan, wk, qpos, row, kt, part, am);
 
         const bool got = mbar_wait(barS, t & 1, cap, &abort_flag);
         if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit

@@ -42,4 +42,25 @@ __device__ __forceinline__ void pred_words(const int32_t* __restrict__ terms, in
   }
 }
 
+// attend-bits of key position j against the 128 queries of query tile qt, the
+// transposed form for the backward's key-tile pass (queries beyond q_len never
+// attend): for a fixed key each term keeps one interval of queries
+__device__ __forceinline__ void pred_words_col(const int32_t* __restrict__ terms, int n_terms, int j, int qt,
+                                               int q_len, uint32_t (&am)[4]) {
+  am[0] = am[1] = am[2] = am[3] = 0u;
+  const int64_t r0 = static_cast<int64_t>(qt) * 128;
+  for (int t = 0; t < n_terms; ++t) {
+    const int32_t* T = terms + t * kTermInts;
+    if (j < T[4] || j >= T[5]) continue;
+    int64_t lo = static_cast<int64_t>(j) + T[0];          // i - j >= diag_lo
+    int64_t hi = static_cast<int64_t>(j) + T[1];          // i - j <= diag_hi
+    lo = lo > T[2] ? lo : static_cast<int64_t>(T[2]);     // i >= q_lo
+    hi = hi < static_cast<int64_t>(T[3]) - 1 ? hi : static_cast<int64_t>(T[3]) - 1;  // i < q_hi
+    lo = lo > 0 ? lo : 0;
+    hi = hi < static_cast<int64_t>(q_len) - 1 ? hi : static_cast<int64_t>(q_len) - 1;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) am[w] |= interval_word(lo, hi, r0 + 32 * w);
+  }
+}
+
 }  // namespace bfa

@@ -1,0 +1,141 @@
+// Attend-bits of one row of a tile, for the mask forms of a plan (shared by the
+// forward, the backward's query-tile pass and, transposed, its key-tile pass).
+// `Ctx` carries the group fields the forms need: k_len, q_len, qid_off, kid_off,
+// kbit_off.  The forms: packed fine words (dense and generic block-sparse plans),
+// the block-id predicate q_valid & k_valid & (k_blk <= q_blk) (opentau
+// flash_attn_blockmask), position terms (pred.cuh) and causal / window positions;
+// full tiles need no mask except past the end of the keys (or queries).
+#pragma once
+
+#include <cstdint>
+
+#include "plan_types.cuh"
+#include "pred.cuh"
+
+namespace bfa {
+
+// attend-bits of one query row (position qpos in its group) against the 128
+// columns of key tile `kt`
+template <typename Ctx>
+__device__ __forceinline__ void row_mask_words(const PlanDev& plan, const Ctx& wk, int qpos, int row, int kt, int part,
+                                               uint32_t (&am)[4]) {
+  const int ncols = wk.k_len - kt * kTile;  // in-range columns (may exceed 128)
+  if (plan.mask_mode == MASK_BITS) {
+    if (part >= 0) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(plan.fine + static_cast<int64_t>(part) * kFineWordsPerTile +
+                                                           row * kWordsPerTileRow));
+      am[0] = v.x; am[1] = v.y; am[2] = v.z; am[3] = v.w;
+    } else {
+      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
+    }
+  } else if (plan.mask_mode == MASK_BLOCKID) {
+    if (part >= 0) {
+      const int32_t qb = plan.qid[wk.qid_off + qpos];
+      const bool qv = plan.qvalid[wk.qid_off + qpos] != 0;
+      const int4* kb4 = reinterpret_cast<const int4*>(plan.kid + wk.kid_off + kt * kTile);
+      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(plan.kbits + wk.kbit_off + kt * kWordsPerTileRow));
+      const uint32_t kvw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const int4 k = __ldg(kb4 + w * 8 + c4);
+          bits |= (k.x <= qb ? 1u : 0u) << (c4 * 4 + 0);
+          bits |= (k.y <= qb ? 1u : 0u) << (c4 * 4 + 1);
+          bits |= (k.z <= qb ? 1u : 0u) << (c4 * 4 + 2);
+          bits |= (k.w <= qb ? 1u : 0u) << (c4 * 4 + 3);
+        }
+        am[w] = qv ? (bits & kvw[w]) : 0u;
+      }
+    } else {
+      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
+    }
+  } else if (plan.mask_mode == MASK_PRED) {
+    if (part >= 0) {
+      pred_words(plan.terms, plan.n_terms, qpos, kt, wk.k_len, am);
+    } else {
+      am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
+    }
+  } else {  // MASK_POS: causal kv_pos <= q_pos, optional window q_pos - kv_pos < W
+    int hi = plan.causal ? (qpos - kt * kTile) : 127;                           // last attended column
+    int lo = (plan.window >= 0) ? (qpos - kt * kTile - plan.window + 1) : 0;  // first attended column
+    if (part < 0) { hi = 127; lo = 0; }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int a = lo - 32 * w, z = hi - 32 * w;  // attended range inside this word
+      uint32_t m_hi = (z >= 31) ? 0xffffffffu : (z < 0 ? 0u : ((2u << z) - 1u));
+      uint32_t m_lo = (a <= 0) ? 0xffffffffu : (a > 31 ? 0u : ~((1u << a) - 1u));
+      am[w] = m_hi & m_lo;
+    }
+  }
+  // key tokens past the group's end (edge tile) are never attended
+  if (ncols < kTile) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int z = ncols - 32 * w;
+      const uint32_t m = (z >= 32) ? 0xffffffffu : (z <= 0 ? 0u : ((1u << z) - 1u));
+      am[w] &= m;
+    }
+  }
+}
+
+
+// Attend-bits of one key (position kpos in its group, row `col` of key tile kt)
+// against the 128 queries of query tile qt: bit i of word w is query 32 w + i of
+// the tile.  `part` is the tile's entry in the transposed lists (-1 full).
+// Queries past the group's end (edge tile) never attend.
+template <typename Ctx>
+__device__ __forceinline__ void col_mask_words(const PlanDev& plan, const Ctx& wk, int kpos, int col, int qt, int part,
+                                               uint32_t (&am)[4]) {
+  if (part < 0) {
+    am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
+  } else if (plan.mask_mode == MASK_BITS) {
+    // column `col` of the tile's row-major fine words: one word per query row,
+    // the same word for all lanes of a warp (col / 32 is warp-uniform)
+    const uint32_t* f = plan.fine + static_cast<int64_t>(part) * kFineWordsPerTile + (col >> 5);
+    const int b = col & 31;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t bits = 0;
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) bits |= ((__ldg(f + (32 * w + i) * kWordsPerTileRow) >> b) & 1u) << i;
+      am[w] = bits;
+    }
+  } else if (plan.mask_mode == MASK_BLOCKID) {
+    const int32_t kb = plan.kid[wk.kid_off + kpos];
+    const bool kv = (plan.kbits[wk.kbit_off + (kpos >> 5)] >> (kpos & 31)) & 1u;
+    const int32_t* qb = plan.qid + wk.qid_off + qt * kTile;
+    const uint8_t* qv = plan.qvalid + wk.qid_off + qt * kTile;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t bits = 0;
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) bits |= ((qv[32 * w + i] != 0 && kb <= qb[32 * w + i]) ? 1u : 0u) << i;
+      am[w] = kv ? bits : 0u;
+    }
+  } else if (plan.mask_mode == MASK_PRED) {
+    pred_words_col(plan.terms, plan.n_terms, kpos, qt, wk.q_len, am);
+  } else {  // MASK_POS: causal q_pos >= kv_pos, optional window q_pos - kv_pos < W
+    const int lo = plan.causal ? (kpos - qt * kTile) : 0;                                  // first attended row
+    const int hi = (plan.window >= 0) ? (kpos - qt * kTile + plan.window - 1) : 127;      // last attended row
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int a = lo - 32 * w, z = hi - 32 * w;
+      uint32_t m_hi = (z >= 31) ? 0xffffffffu : (z < 0 ? 0u : ((2u << z) - 1u));
+      uint32_t m_lo = (a <= 0) ? 0xffffffffu : (a > 31 ? 0u : ~((1u << a) - 1u));
+      am[w] = m_hi & m_lo;
+    }
+  }
+  const int nrows = wk.q_len - qt * kTile;  // in-range query rows (may exceed 128)
+  if (nrows < kTile) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int z = nrows - 32 * w;
+      const uint32_t m = (z >= 32) ? 0xffffffffu : (z <= 0 ? 0u : ((1u << z) - 1u));
+      am[w] &= m;
+    }
+  }
+}
+
+}  // namespace bfa

@@ -1,0 +1,188 @@
+"""GPU backward parity: dQ, dK, dV against the float64 oracle (oracle.backward).
+
+The library's forward supplies out and lse (bf16 / fp32), as a training step
+would; the oracle differentiates the exact forward definition in float64 on the
+same bf16 inputs.  Tolerance: the kernel rounds P and dS to bf16 before their
+products (relative 2^-9 each), uses the bf16 output for D = dO . O and rounds
+the gradients to bf16; per gradient tensor the max-abs error must stay below
+1e-2 of the tensor's largest magnitude plus 1e-3 (bf16 N(0, 1) inputs at the
+default scale).  Rows that attend nothing and keys that no query attends get
+exact zeros.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import backward as ob
+from oracle import masks as om
+
+pytestmark = pytest.mark.gpu
+
+bfa = pytest.importorskip("mask_skipping_flashattention_b200")
+
+REL = 1e-2
+ABS = 1e-3
+
+
+def _cuda(x):
+    return torch.as_tensor(np.ascontiguousarray(x)).cuda()
+
+
+def _close(got, ref, name):
+    got = np.asarray(got.float().cpu(), dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"non-finite {name}"
+    err = np.abs(got - ref).max() if ref.size else 0.0
+    bound = REL * (np.abs(ref).max() if ref.size else 0.0) + ABS
+    assert err <= bound, f"{name}: max-abs {err:.3e} > {bound:.3e}"
+    return err
+
+
+def _run_bshd(P, q, k, v, do, mask_for, scale=None):
+    qc, kc, vc, dc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out, lse = bfa.fwd(P, qc, kc, vc, scale=scale)
+    dq, dk, dv = bfa.bwd(P, qc, kc, vc, out, dc, lse, scale=scale)
+    torch.cuda.synchronize()
+    P.device_status()
+    rq, rk, rv = ob.attention_bwd_bshd(q, k, v, do, mask_for, scale)
+    return (_close(dq, rq, "dq"), _close(dk, rk, "dk"), _close(dv, rv, "dv")), (dq, dk, dv)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("shape,density", [((300, 300), 0.3), ((129, 257), 0.9), ((512, 512), 0.02)])
+def test_dense_random_masks(D, shape, density):
+    Sq, Sk = shape
+    rng = np.random.default_rng(Sq * 3 + Sk + D)
+    M = rng.random((Sq, Sk)) < density
+    M[:, 0] |= rng.random(Sq) < 0.5
+    B, H = 1, 2
+    q = workloads.randn_bf16((B, Sq, H, D), 11)
+    k = workloads.randn_bf16((B, Sk, H, D), 12)
+    v = workloads.randn_bf16((B, Sk, H, D), 13)
+    do = workloads.randn_bf16((B, Sq, H, D), 14)
+    _run_bshd(bfa.plan_dense(_cuda(M)), q, k, v, do, lambda b, h: M)
+
+
+def test_dense_causal_gqa_two_batches():
+    B, H, Hkv, N, D = 2, 4, 2, 384, 128
+    M = np.tril(np.ones((N, N), dtype=bool))
+    q = workloads.randn_bf16((B, N, H, D), 21)
+    k = workloads.randn_bf16((B, N, Hkv, D), 22)
+    v = workloads.randn_bf16((B, N, Hkv, D), 23)
+    do = workloads.randn_bf16((B, N, H, D), 24)
+    _run_bshd(bfa.plan_dense(_cuda(M)), q, k, v, do, lambda b, h: M, scale=0.1)
+
+
+def test_blockids_with_padding_and_cross_columns():
+    w = workloads.tiny_blockcausal()
+    ids_ref = om.make_att_block_ids(w["pad_masks"], w["att_masks"])
+    M = om.blockid_dense(*ids_ref)[0]
+    P = bfa.plan_blockids(*bfa.make_att_block_ids(_cuda(w["pad_masks"]), _cuda(w["att_masks"])))
+    do = workloads.randn_bf16(tuple(w["q"].shape), 31)
+    errs, (dq, dk, dv) = _run_bshd(P, w["q"], w["k"], w["v"], do, lambda b, h: M, w["scale"])
+    # padded query rows attend nothing; padded keys are attended by nothing
+    assert torch.all(dq[0, 240:] == 0)
+    assert torch.all(dk[0, 240:] == 0) and torch.all(dv[0, 240:] == 0)
+
+
+def test_positional_window_batched():
+    B, H, Sq, Sk, D, W = 2, 2, 700, 650, 64, 100
+    P = bfa.plan_blockids(B=B, Sq=Sq, Sk=Sk, window_left=W)
+    M = om.positional_dense(Sq, Sk, True, W)
+    q = workloads.randn_bf16((B, Sq, H, D), 41)
+    k = workloads.randn_bf16((B, Sk, H, D), 42)
+    v = workloads.randn_bf16((B, Sk, H, D), 43)
+    do = workloads.randn_bf16((B, Sq, H, D), 44)
+    _run_bshd(P, q, k, v, do, lambda b, h: M)
+
+
+def test_predicate_terms():
+    terms = [om.term(diag_lo=0, diag_hi=255), om.term(q_hi=64), om.term(k_hi=64)]
+    B, H, Sq, Sk, D = 1, 2, 600, 600, 128
+    P = bfa.plan_predicate(terms, B=B, Sq=Sq, Sk=Sk)
+    M = om.predicate_dense(terms, Sq, Sk)
+    q = workloads.randn_bf16((B, Sq, H, D), 51)
+    k = workloads.randn_bf16((B, Sk, H, D), 52)
+    v = workloads.randn_bf16((B, Sk, H, D), 53)
+    do = workloads.randn_bf16((B, Sq, H, D), 54)
+    _run_bshd(P, q, k, v, do, lambda b, h: M)
+
+
+def test_general_block_sparse_with_validity():
+    B, H, Hkv, Sq, Skv, qb, kb, D = 1, 4, 2, 450, 600, 32, 8, 128
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    rng = np.random.default_rng(5)
+    indptr = np.zeros((B, Hkv, nqb + 1), dtype=np.int32)
+    idx, pos = [], 0
+    for b in range(B):
+        for h in range(Hkv):
+            indptr[b, h, 0] = pos
+            for r in range(nqb):
+                row = np.sort(rng.choice(nkb, size=int(rng.binomial(nkb, 0.3)), replace=False))
+                idx.append(row)
+                pos += row.size
+                indptr[b, h, r + 1] = pos
+    indices = np.concatenate(idx).astype(np.int32)
+    valid = rng.random((B, Skv)) < 0.9
+    kvb = np.zeros((B, -(-Skv // 32)), dtype=np.uint32)
+    for b in range(B):
+        for j in np.nonzero(valid[b])[0]:
+            kvb[b, j // 32] |= np.uint32(1) << np.uint32(j % 32)
+    P = bfa.plan_bsr(_cuda(indptr), _cuda(indices), Sq, Skv, qb, kb, causal=True,
+                     kv_valid_bits=_cuda(kvb.view(np.int32)))
+    Dm = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=True,
+                             kv_valid_bits=kvb)
+    q = workloads.randn_bf16((B, Sq, H, D), 61)
+    k = workloads.randn_bf16((B, Skv, Hkv, D), 62)
+    v = workloads.randn_bf16((B, Skv, Hkv, D), 63)
+    do = workloads.randn_bf16((B, Sq, H, D), 64)
+    _run_bshd(P, q, k, v, do, lambda b, h: Dm[b, h // (H // Hkv)])
+
+
+def test_varlen_causal_packed():
+    cu = np.array([0, 5, 300, 300, 777], dtype=np.int32)  # includes an empty sequence
+    T, H, Hkv, D = int(cu[-1]), 4, 2, 64
+    P = bfa.plan_blockids(cu_seqlens_q=_cuda(cu), cu_seqlens_k=_cuda(cu), max_q=512, max_k=512)
+    M = np.zeros((T, T), dtype=bool)
+    for s in range(len(cu) - 1):
+        a, z = cu[s], cu[s + 1]
+        M[a:z, a:z] = np.tril(np.ones((z - a, z - a), dtype=bool))
+    q = workloads.randn_bf16((T, H, D), 71)
+    k = workloads.randn_bf16((T, Hkv, D), 72)
+    v = workloads.randn_bf16((T, Hkv, D), 73)
+    do = workloads.randn_bf16((T, H, D), 74)
+    qc, kc, vc, dc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    dq, dk, dv = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    rq, rk, rv = ob.attention_bwd_thd(q, k, v, do, M)
+    _close(dq, rq, "dq")
+    _close(dk, rk, "dk")
+    _close(dv, rv, "dv")
+
+
+def test_all_false_mask_gives_zero_gradients():
+    M = np.zeros((200, 300), dtype=bool)
+    q = workloads.randn_bf16((1, 200, 1, 64), 81).cuda()
+    k = workloads.randn_bf16((1, 300, 1, 64), 82).cuda()
+    v = workloads.randn_bf16((1, 300, 1, 64), 83).cuda()
+    do = workloads.randn_bf16((1, 200, 1, 64), 84).cuda()
+    P = bfa.plan_dense(_cuda(M))
+    out, lse = bfa.fwd(P, q, k, v)
+    dq, dk, dv = bfa.bwd(P, q, k, v, out, do, lse)
+    torch.cuda.synchronize()
+    assert torch.all(dq == 0) and torch.all(dk == 0) and torch.all(dv == 0)
+
+
+def test_bwd_rejects_bad_arguments():
+    M = np.ones((128, 128), dtype=bool)
+    q = workloads.randn_bf16((1, 128, 1, 64), 91).cuda()
+    P = bfa.plan_dense(_cuda(M))
+    out, lse = bfa.fwd(P, q, q, q)
+    with pytest.raises(TypeError):
+        bfa.bwd(P, q, q, q, out, q, None)
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.bwd(P, q.cpu(), q, q, out, q, lse)
+    assert e.value.status == "BFA_ERR_NOT_DEVICE"
