@@ -14,11 +14,13 @@
 //               padded to whole tiles (HBM-bound, one pass over O and dO);
 //   k_bwd_dq    one CTA per (plan row, replica), walking the row's key-tile list:
 //               S = Q K^T and dP = dO V^T (SS), dS into TMEM as bf16, dQ += dS K
-//               (TS); the mask on partial and edge tiles only;
+//               (TS) chunk by chunk while the next chunk of dS is made; the mask
+//               on partial and edge tiles only;
 //   k_bwd_dkdv  one CTA per (key-tile column, kv replica), walking the column's
 //               query-tile list for every query head of the kv head (GQA sums in
 //               TMEM, no atomics): S^T = K Q^T and dP^T = V dO^T (SS), P^T and dS^T
-//               into TMEM as bf16, dV += P^T dO and dK += dS^T Q (TS).
+//               into TMEM as bf16, dV += P^T dO and dK += dS^T Q (TS), chunk by
+//               chunk as in k_bwd_dq.
 // Warp roles of the two tile kernels (256 threads): warp 0 TMA producer, warp 1
 // TMEM owner and single-thread tcgen05.mma issuer, warps 4..7 one tile row per
 // thread (query rows in k_bwd_dq, key rows in k_bwd_dkdv).  Every wait is
@@ -124,15 +126,6 @@ __device__ __forceinline__ void issue_nn(uint32_t tD, const uint8_t* sA, const u
   }
 }
 
-// D (tmem, N = D columns) (+)= A (tmem, bf16 128 x 128) * B (smem tile, rows = the K axis)
-template <int D>
-__device__ __forceinline__ void issue_td(uint32_t tD, uint32_t tA, const uint8_t* sB, bool acc) {
-#pragma unroll
-  for (int kk = 0; kk < kTile / 16; ++kk)
-    umma_ts(tD, tA + kk * 8, smem_desc(smem_u32(sB + kk * 2048), 16384, 1024), BCfg<D>::kIdescD,
-            (acc || kk > 0) ? 1u : 0u);
-}
-
 // fp32 accumulator row (TMEM, D columns) * scale -> bf16 row in global memory
 template <int D>
 __device__ __forceinline__ void store_row(uint32_t tAcc, bool have, float scale, __nv_bfloat16* dst, bool store) {
@@ -224,8 +217,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* const sK0 = smem + 2 * C::kTileBytes;
   uint8_t* const sV0 = smem + (2 + kBwdStages) * C::kTileBytes;
   // BQ: Q and dO.  BF / BE [2]: K, V stage full / free.  BS: S and dP of the
-  // current tile ready.  BP: dS written (4 warps).  BO: every product done.
-  enum { BQ = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 7, BDONE = 8, NBAR = 9 };
+  // current tile ready.  BP [4]: dS of one 32-key chunk written (4 warps), so the
+  // dQ products of a chunk overlap the next chunk's dS.  BO: every product done.
+  enum { BQ = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 10, BDONE = 11, NBAR = 12 };
   __shared__ __align__(8) uint64_t bars[NBAR];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -237,7 +231,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), i == BP ? 4 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= BP && i < BP + 4) ? 4 : 1);
     fence_barrier_init();
     int i, j;
     chunked_decode(blockIdx.x, p.plan.n_rows, p.rep, p.head_chunk, i, j);
@@ -305,21 +299,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
-      const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+      // TMEM: S [0,128), dP [128,256), dQ [256,256+D), dS (bf16 pairs) [384,448)
+      const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256, tdS = tmem + 384;
       bool ok = mbar_wait_fast(bar(BQ), 0, cap, &abort_flag);
+      if (ok) ok = mbar_wait_fast(bar(BF), 0, cap, &abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_nn<D>(tS, sQ, sK(0));    // S = Q K^T
+        issue_nn<D>(tdP, sdO, sV(0));  // dP = dO V^T
+        umma_commit(bar(BS));
+      }
       bool started = false;
       for (int u = 0; ok && u < n; ++u) {
         const int st = u & 1;
-        if (!mbar_wait_fast(bar(BF + st), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_nn<D>(tS, sQ, sK(st));    // S = Q K^T (over the dS of tile u - 1, in issue order)
-        issue_nn<D>(tdP, sdO, sV(st));  // dP = dO V^T
-        umma_commit(bar(BS));
-        if (!mbar_wait_fast(bar(BP), u & 1, cap, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_td<D>(tdQ, tS, sK(st), started);  // dQ += dS K
+        // dQ += dS K, chunk by chunk as the rows finish them
+        for (int cc = 0; cc < 4; ++cc) {
+          if (!mbar_wait_fast(bar(BP + cc), u & 1, cap, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk)
+            umma_ts(tdQ, tdS + kk * 8, smem_desc(smem_u32(sK(st) + kk * 2048), 16384, 1024), C::kIdescD,
+                    (started || kk > 0) ? 1u : 0u);
+        }
+        if (!ok) break;
         started = true;
         umma_commit(bar(BE + st));
+        // the rows have read all of S(u) and dP(u): the next tile's products
+        if (u + 1 < n) {
+          const int st1 = (u + 1) & 1;
+          if (!mbar_wait_fast(bar(BF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_nn<D>(tS, sQ, sK(st1));
+          issue_nn<D>(tdP, sdO, sV(st1));
+          umma_commit(bar(BS));
+        }
       }
       if (ok) umma_commit(bar(BO));
       umma_commit(bar(BDONE));
@@ -350,29 +363,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
       if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
       tc_fence_after();
-#pragma unroll 1
+      // chunks of 32 keys; the loads of chunk cc + 1 are in flight while chunk cc
+      // is computed (two register sets, the loop fully unrolled)
+      uint32_t sA[32], dA[32], sB[32], dB[32];
+      tmem_ld_32x32b_x32(tLane, sA);
+      tmem_ld_32x32b_x32(tLane + 128, dA);
+      tmem_wait_ld();
+      reg_fence(sA);
+      reg_fence(dA);
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32], dp[32];
-        tmem_ld_32x32b_x32(tLane + cc * 32, sv);
-        tmem_ld_32x32b_x32(tLane + 128 + cc * 32, dp);
-        tmem_wait_ld();
-        reg_fence(sv);
-        reg_fence(dp);
+        uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
+        uint32_t(&dp)[32] = (cc & 1) ? dB : dA;
+        if (cc + 1 < 4) {
+          tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
+          tmem_ld_32x32b_x32(tLane + 128 + (cc + 1) * 32, (cc & 1) ? dA : dB);
+        }
         const uint32_t bits = am[cc];
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
+          // masked scores become -inf (a select, no branch), so 2^(...) is 0
           const int c0 = 2 * jj, c1 = 2 * jj + 1;
-          const float p0 = ((bits >> c0) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[c0]), c, -lse2)) : 0.f;
-          const float p1 = ((bits >> c1) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[c1]), c, -lse2)) : 0.f;
+          const float s0 = ((bits >> c0) & 1u) ? __uint_as_float(sv[c0]) : -INFINITY;
+          const float s1 = ((bits >> c1) & 1u) ? __uint_as_float(sv[c1]) : -INFINITY;
+          const float p0 = ex2_approx(fmaf(s0, c, -lse2));
+          const float p1 = ex2_approx(fmaf(s1, c, -lse2));
           pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dp[c0]) - dval), p1 * (__uint_as_float(dp[c1]) - dval));
         }
-        tmem_st_32x32b_x16(tLane + cc * 16, pk);  // dS over S columns already read
+        tmem_st_32x32b_x16(tLane + 384 + cc * 16, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BP + cc));
+        if (cc + 1 < 4) {
+          tmem_wait_ld();
+          reg_fence((cc & 1) ? sA : sB);
+          reg_fence((cc & 1) ? dA : dB);
+        }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BP));
     }
     bool done = ok;
     if (ok && n > 0) {
@@ -418,9 +447,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* const sQ0 = smem + 2 * C::kTileBytes;                      // + 2 st tiles
   float* const sVec0 = reinterpret_cast<float*>(smem + (2 + 2 * kBwdStages) * C::kTileBytes);  // + st * 256
   // BKV: K and V.  BF / BE [2]: Q, dO and the query vectors of a step full /
-  // free.  BS: S^T and dP^T ready.  BP: P^T and dS^T written (4 warps).  BO:
-  // every product done.
-  enum { BKV = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 7, BDONE = 8, NBAR = 9 };
+  // free.  BS: S^T and dP^T ready.  BP [4]: P^T and dS^T of one 32-query chunk
+  // written (4 warps), so the chunk's dV, dK products overlap the next chunk.
+  // BO: every product done.
+  enum { BKV = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 10, BDONE = 11, NBAR = 12 };
   __shared__ __align__(8) uint64_t bars[NBAR];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -433,7 +463,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), i == BP ? 4 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= BP && i < BP + 4) ? 4 : 1);
     fence_barrier_init();
     int i, jk;
     chunked_decode(blockIdx.x, p.n_cols, p.rep_kv, p.kv_chunk, i, jk);
@@ -516,10 +546,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_nn<D>(tS, sK, sQ(st));    // S^T = K Q^T (over P^T of step s - 1, in issue order)
         issue_nn<D>(tdP, sV, sdO(st));  // dP^T = V dO^T
         umma_commit(bar(BS));
-        if (!mbar_wait_fast(bar(BP), s & 1, cap, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_td<D>(tdV, tS, sdO(st), started);  // dV += P^T dO
-        issue_td<D>(tdK, tdP, sQ(st), started);  // dK += dS^T Q
+        // dV += P^T dO and dK += dS^T Q, chunk by chunk as the rows finish them
+        for (int cc = 0; cc < 4; ++cc) {
+          if (!mbar_wait_fast(bar(BP + cc), s & 1, cap, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk) {
+            const uint32_t acc = (started || kk > 0) ? 1u : 0u;
+            umma_ts(tdV, tS + kk * 8, smem_desc(smem_u32(sdO(st) + kk * 2048), 16384, 1024), C::kIdescD, acc);
+            umma_ts(tdK, tdP + kk * 8, smem_desc(smem_u32(sQ(st) + kk * 2048), 16384, 1024), C::kIdescD, acc);
+          }
+        }
+        if (!ok) break;
         started = true;
         umma_commit(bar(BE + st));
       }
@@ -550,14 +588,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const float* lse2 = sVec(st);
       const float* dvec = sVec(st) + kTile;
-#pragma unroll 1
+      // chunks of 32 queries, loads one chunk ahead as in k_bwd_dq (a chunk's
+      // P^T / dS^T columns never overlap the next chunk's S^T / dP^T columns)
+      uint32_t sA[32], dA[32], sB[32], dB[32];
+      tmem_ld_32x32b_x32(tLane, sA);
+      tmem_ld_32x32b_x32(tLane + 128, dA);
+      tmem_wait_ld();
+      reg_fence(sA);
+      reg_fence(dA);
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32], dp[32];
-        tmem_ld_32x32b_x32(tLane + cc * 32, sv);
-        tmem_ld_32x32b_x32(tLane + 128 + cc * 32, dp);
-        tmem_wait_ld();
-        reg_fence(sv);
-        reg_fence(dp);
+        uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
+        uint32_t(&dp)[32] = (cc & 1) ? dB : dA;
+        if (cc + 1 < 4) {
+          tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
+          tmem_ld_32x32b_x32(tLane + 128 + (cc + 1) * 32, (cc & 1) ? dA : dB);
+        }
         const uint32_t bits = am[cc];
         uint32_t pkp[16], pks[16];
 #pragma unroll
@@ -569,7 +615,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const int col = q4 * 4 + t;
-            pv[t] = ((bits >> col) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[col]), c, -Ls[t])) : 0.f;
+            const float sm = ((bits >> col) & 1u) ? __uint_as_float(sv[col]) : -INFINITY;  // select, no branch
+            pv[t] = ex2_approx(fmaf(sm, c, -Ls[t]));
             dsv[t] = pv[t] * (__uint_as_float(dp[col]) - Ds[t]);
           }
           pkp[2 * q4] = pack_bf16x2(pv[0], pv[1]);
@@ -579,11 +626,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tmem_st_32x32b_x16(tLane + cc * 16, pkp);        // P^T over S^T columns already read
         tmem_st_32x32b_x16(tLane + 128 + cc * 16, pks);  // dS^T over dP^T columns already read
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BP + cc));
+        if (cc + 1 < 4) {
+          tmem_wait_ld();
+          reg_fence((cc & 1) ? sA : sB);
+          reg_fence((cc & 1) ? dA : dB);
+        }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BP));
     }
     bool done = ok;
     if (ok && steps > 0) {
