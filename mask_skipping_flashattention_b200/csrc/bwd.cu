@@ -193,8 +193,8 @@ __global__ void __launch_bounds__(128) k_bwd_prep(const BwdParams p) {
     lse2 = (L == -INFINITY) ? 0.f : L * 1.4426950408889634f;  // a row that attends nothing has no listed pair
   }
   const int64_t wi = (static_cast<int64_t>(j) * p.plan.n_rows + r) * kTile + threadIdx.x;
-  p.ws_lse2[wi] = lse2;
-  p.ws_d[wi] = dval;
+  p.ws_lse2[wi] = -lse2;  // stored negated: the tile kernels add them
+  p.ws_d[wi] = -dval;
 }
 
 // ----------------------------------------------------------------------------
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tLane = tmem_addr(tmem, quarter * 32, 0);
     const GroupCtx ctx = group_ctx(wk.g);
     const int64_t wi = (static_cast<int64_t>(wk.j) * p.plan.n_rows + wk.r) * kTile + row;
-    const float lse2 = p.ws_lse2[wi], dval = p.ws_d[wi];
+    const float nlse2 = p.ws_lse2[wi], nd = p.ws_d[wi];  // -LSE * log2(e), -D
     const float c = p.scale_log2;
     bool ok = true;
     int kt_next = n > 0 ? p.plan.kv_tile[wk.e0] : 0;
@@ -387,9 +387,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int c0 = 2 * jj, c1 = 2 * jj + 1;
           const float s0 = ((bits >> c0) & 1u) ? __uint_as_float(sv[c0]) : -INFINITY;
           const float s1 = ((bits >> c1) & 1u) ? __uint_as_float(sv[c1]) : -INFINITY;
-          const float p0 = ex2_approx(fmaf(s0, c, -lse2));
-          const float p1 = ex2_approx(fmaf(s1, c, -lse2));
-          pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dp[c0]) - dval), p1 * (__uint_as_float(dp[c1]) - dval));
+          const float p0 = ex2_approx(fmaf(s0, c, nlse2));
+          const float p1 = ex2_approx(fmaf(s1, c, nlse2));
+          pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dp[c0]) + nd), p1 * (__uint_as_float(dp[c1]) + nd));
         }
         tmem_st_32x32b_x16(tLane + 384 + cc * 16, pk);
         tmem_wait_st();
@@ -574,6 +574,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tLane = tmem_addr(tmem, quarter * 32, 0);
     const GroupCtx ctx = group_ctx(wk.g);
     const float c = p.scale_log2;
+    const uint64_t c2 = f2_pack(c, c);
     bool ok = true;
     for (int s = 0; s < steps; ++s) {
       const int st = s & 1;
@@ -586,8 +587,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool gs = gv && mbar_wait(bar(BS), s & 1, cap, &abort_flag);
       if (__any_sync(0xffffffffu, !gs)) { ok = false; break; }
       tc_fence_after();
-      const float* lse2 = sVec(st);
-      const float* dvec = sVec(st) + kTile;
+      const uint32_t sLse = smem_u32(sVec(st)), sDv = smem_u32(sVec(st) + kTile);
       // chunks of 32 queries, loads one chunk ahead as in k_bwd_dq (a chunk's
       // P^T / dS^T columns never overlap the next chunk's S^T / dP^T columns)
       uint32_t sA[32], dA[32], sB[32], dB[32];
@@ -608,21 +608,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t pkp[16], pks[16];
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 L = *reinterpret_cast<const float4*>(lse2 + cc * 32 + q4 * 4);
-          const float4 Dv = *reinterpret_cast<const float4*>(dvec + cc * 32 + q4 * 4);
-          const float Ls[4] = {L.x, L.y, L.z, L.w}, Ds[4] = {Dv.x, Dv.y, Dv.z, Dv.w};
-          float pv[4], dsv[4];
+          const float4 L = ld_shared_f4(sLse + (cc * 32 + q4 * 4) * 4);
+          const float4 Dv = ld_shared_f4(sDv + (cc * 32 + q4 * 4) * 4);
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int col = q4 * 4 + t;
-            const float sm = ((bits >> col) & 1u) ? __uint_as_float(sv[col]) : -INFINITY;  // select, no branch
-            pv[t] = ex2_approx(fmaf(sm, c, -Ls[t]));
-            dsv[t] = pv[t] * (__uint_as_float(dp[col]) - Ds[t]);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int col = q4 * 4 + 2 * h2;
+            // masked scores become -inf (a select, no branch), so 2^(...) is 0;
+            // pairs of columns through the packed fp32x2 fma / add / mul
+            const float s0 = ((bits >> col) & 1u) ? __uint_as_float(sv[col]) : -INFINITY;
+            const float s1 = ((bits >> (col + 1)) & 1u) ? __uint_as_float(sv[col + 1]) : -INFINITY;
+            const uint64_t nl = h2 ? f2_pack(L.z, L.w) : f2_pack(L.x, L.y);     // -LSE * log2(e)
+            const uint64_t nd = h2 ? f2_pack(Dv.z, Dv.w) : f2_pack(Dv.x, Dv.y);  // -D
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s0, s1), c2, nl), x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const uint64_t pp = f2_pack(p0, p1);
+            float d0, d1;
+            f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(dp[col]), __uint_as_float(dp[col + 1])), nd)), d0, d1);
+            pkp[2 * q4 + h2] = pack_bf16x2(p0, p1);
+            pks[2 * q4 + h2] = pack_bf16x2(d0, d1);
           }
-          pkp[2 * q4] = pack_bf16x2(pv[0], pv[1]);
-          pkp[2 * q4 + 1] = pack_bf16x2(pv[2], pv[3]);
-          pks[2 * q4] = pack_bf16x2(dsv[0], dsv[1]);
-          pks[2 * q4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
         tmem_st_32x32b_x16(tLane + cc * 16, pkp);        // P^T over S^T columns already read
         tmem_st_32x32b_x16(tLane + 128 + cc * 16, pks);  // dS^T over dP^T columns already read

@@ -32,8 +32,8 @@ struct BwdParams {
   int64_t dk_sb, dk_ss, dk_sh;
   __nv_bfloat16* dv;
   int64_t dv_sb, dv_ss, dv_sh;
-  // per (replica, plan row, row of the tile): LSE * log2(e) and D = dO . O, with
-  // rows past a sequence (and rows that attend nothing) holding 0
+  // per (replica, plan row, row of the tile), negated: -LSE * log2(e) and
+  // -D = -dO . O, with rows past a sequence (and rows that attend nothing) 0
   float* ws_lse2;
   float* ws_d;
   // transposed lists of the plan
