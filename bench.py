@@ -290,6 +290,28 @@ def run_bfa(args, rank, world, local_rank):
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dist, dev)[0]
     e2e_value = whole_job_tflops(flops, world, e2e_ms)
 
+    # backward (f1) on the same workload, timed on its own after the forward
+    # metric: dq, dk, dv for a seeded upstream gradient, plan and LSE reused
+    g = torch.Generator(device="cpu")
+    g.manual_seed(4242)
+    dout = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    plan = bfa.plan_dense(mask)
+    bfa.fwd(plan, q, k, v, out=out, lse=lse)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for _ in range(2):
+        bfa.bwd(plan, q, k, v, out, dout, lse, dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bwd_steps = max(1, min(args.steps, 5))
+    b0.record(stream)
+    for _ in range(bwd_steps):
+        bfa.bwd(plan, q, k, v, out, dout, lse, dq=dq, dk=dk, dv=dv)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    plan.device_status()
+    plan.destroy()
+    bwd_ms = max_over_ranks([b0.elapsed_time(b1) / bwd_steps], dist, dev)[0]
+
     peaks, src = _peaks()
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     # bytes the forward must move at least: read q, k, v once, write out and lse
@@ -311,11 +333,15 @@ def run_bfa(args, rank, world, local_rank):
         "fwd_ms": fwd_ms, "plan_ms": plan_ms,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
+        "bwd": {"ms_per_step": bwd_ms, "tflops": 2.5 * flops / (bwd_ms * 1e-3) / 1e12,
+                "frac": 2.5 * flops / (bwd_ms * 1e-3) / 1e12 / peak,
+                "flops_counted": "2.5 x the forward's attended-pair flops (dV, dP, dQ, dK and the recomputed S)",
+                "kernels": "k_bwd_prep, k_bwd_dq, k_bwd_dkdv", "steps": bwd_steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        v_cpu, dt, n = cpu_oracle_sample(w, n_heads=2)
+        v_cpu, dt, n = cpu_oracle_sample(w, n_heads=16)  # about 10 s of float64 work
         line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": _threads_used(), "kind": "oracle",
                                 "sample": f"{n} of 128 (batch, head) pairs, all 8192 rows, {dt:.1f} s float64"}
     if rank == 0:
