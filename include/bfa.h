@@ -13,7 +13,7 @@
  *
  * Sources (page title, section):
  *   - BinFlash, "Efficiently Dispatching FlashAttention For Partially Filled
- *     Attention Masks": coarse block mask + 32-bit packed fine mask, pre-sorted
+ *     Attention Masks": a coarse per-block mask with the partial blocks' bits packed 32 to a word, sorted
  *     non-empty key-block list per query row, all-True blocks with no mask loads,
  *     all-False blocks skipped; mask (N, N) bool, True = attend; scale 1/sqrt(D).
  *   - opentau.policies.flash_attn_cuda, make_att_block_ids / flash_attn_blockmask:
@@ -187,8 +187,8 @@ bfa_status bfa_plan_predicate(const bfa_mask_term* terms, int n_terms, int B, in
  *   indptr [B, Hkv, ceil(Sq/q_block)+1] i32: absolute offsets into indices, each
  *   (b, hkv) slice non-decreasing; indices [n_indices] i32: KV block ids, each
  *   row strictly increasing in [0, ceil(Skv/kv_block)).
- *   q_block >= 1 query tokens per BSR row; kv_block in {8, 16, 32} or a positive
- *   multiple of 64 key tokens per block id (the page's allowed sizes).
+ *   q_block >= 1 query tokens per BSR row; kv_block key tokens per block id,
+ *   one of 8, 16, 32 or 64 m for an integer m >= 1 (the sizes the page allows).
  *   causal != 0 applies kv_idx <= q_idx on absolute positions inside the selected
  *   blocks (mask_type "causal"); otherwise every pair of a selected block attends.
  *   kv_valid_bits [B, ceil(Skv/32)] u32 or NULL: bit j % 32 of word j / 32 of row b
@@ -239,9 +239,9 @@ bfa_status bfa_fwd(const bfa_plan* plan, const void* q, const void* k, const voi
                    float* lse, void* stream);
 
 /*
- * Backward of bfa_fwd (BinFlash: "Backward uses two passes (dKdV over K-blocks,
- * dQ over Q-blocks)"; the LSE is the forward's auxiliary output that the
- * backward reuses, tensorplay varlen): for an upstream gradient dout of `out`,
+ * Backward of bfa_fwd (BinFlash: two passes, dK/dV over key blocks and dQ over
+ * query blocks; tensorplay varlen: the forward's log-sum-exp serves the backward
+ * again): for an upstream gradient dout of `out`,
  *   dV = P^T dO,  dS = P * (dO V^T - D),  D_i = dO_i . O_i,
  *   dQ = scale dS K,  dK = scale dS^T Q,  P = exp(scale Q K^T - LSE) on attended pairs.
  *   q, k, v, out, lse, scale, B, H, Hkv, D and the plan: exactly as given to (and
@@ -325,8 +325,8 @@ bfa_status bfa_plan_export(const bfa_plan* plan, int32_t* row_ptr, int32_t* kv_t
 bfa_status bfa_plan_export_pairs(const bfa_plan* plan, int32_t* pair_row, int32_t* pair_order, void* stream);
 
 /* Copy the plan's transposed lists to HOST buffers (built on first use, on
- * `stream`; synchronises it).  For the backward's key-tile pass (BinFlash:
- * "dKdV over K-blocks"): column c (group g, key tile kt; groups in order, key
+ * `stream`; synchronises it).  For the backward's key-tile pass (BinFlash's
+ * dK/dV pass over key blocks): column c (group g, key tile kt; groups in order, key
  * tiles ascending) lists the query tiles whose tile (qt, kt) is not empty,
  * ascending, in q_tile[col_ptr[c] .. col_ptr[c+1]); tpart holds -1 for full tiles
  * and, for partial ones, the index of their packed fine words (the same index the

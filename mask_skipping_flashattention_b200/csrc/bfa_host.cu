@@ -708,7 +708,7 @@ BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, i
                 (long long)n_indices);
   if (q_block <= 0) return fail(BFA_ERR_INVALID_ARG, "q_block=%d must be positive", q_block);
   if (!kv_block_ok(kv_block))
-    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d must be 8, 16, 32 or a positive multiple of 64", kv_block);
+    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d: allowed sizes are 8, 16, 32 and the multiples of 64", kv_block);
   bfa_status s;
   if ((s = need_device(indptr, "block_indptr"))) return s;
   if (n_indices > 0 && (s = need_device(indices, "block_indices"))) return s;
@@ -763,7 +763,7 @@ BFA_API bfa_status bfa_plan_block_bits(const uint32_t* block_bits, int B, int Hk
     return fail(BFA_ERR_INVALID_ARG, "bad sizes B=%d Hkv=%d Sq=%d Skv=%d", B, Hkv, Sq, Skv);
   if (q_block <= 0) return fail(BFA_ERR_INVALID_ARG, "q_block=%d must be positive", q_block);
   if (!kv_block_ok(kv_block))
-    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d must be 8, 16, 32 or a positive multiple of 64", kv_block);
+    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d: allowed sizes are 8, 16, 32 and the multiples of 64", kv_block);
   bfa_status s;
   if ((s = need_device(block_bits, "exact_block_bits")) || (s = need_device(kv_valid_bits, "kv_valid_bits", true)))
     return s;

@@ -1,9 +1,10 @@
 // Backward of the mask-aware attention for sm_100a: gradients of
 //   O = softmax(scale Q K^T + mask) V
 // with respect to Q, K and V for an upstream gradient dO, reusing the forward's
-// plan and LSE (BinFlash: "Backward uses two passes (dKdV over K-blocks, dQ over
-// Q-blocks) with the same gathered-dispatch machinery"; tensorplay varlen: the
-// log-sum-exp is the auxiliary output "that the backward pass reuses").
+// plan and LSE (BinFlash, "How it works": the backward is two passes, one over
+// key blocks for dK and dV and one over query blocks for dQ, both dispatched from
+// the same gathered block lists; tensorplay varlen: the log-sum-exp is returned
+// by the forward so that the backward can use it again).
 //
 // With P = exp(scale S - LSE) (S = Q K^T, masked pairs 0), dP = dO V^T and
 // D_i = dO_i . O_i, the score gradient is dS = P * (dP - D), and

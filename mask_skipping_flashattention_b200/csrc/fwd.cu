@@ -3,7 +3,7 @@
 // Each CTA runs two 128-row query tiles ("slots") that share their keys and
 // values: either two heads of one kv head on the same query tile (GQA with an
 // even group), or two consecutive query tiles of one head.  The CTA walks the
-// union of the two tiles' plan lists (BinFlash: iterate a pre-sorted list of
+// union of the two tiles' plan lists (BinFlash: walk each query block's sorted list of
 // non-empty key blocks, run all-True blocks with no mask loads, apply the mask on
 // partial blocks only, skip all-False blocks).  Work items are taken in the
 // plan's longest-first order, so the hardware's in-order CTA dispatch balances

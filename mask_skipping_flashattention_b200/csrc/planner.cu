@@ -3,8 +3,8 @@
 // first row order), plus packed fine masks for the partial tiles of dense masks.
 //
 // The method is BinFlash's preprocessing ("Efficiently Dispatching FlashAttention
-// For Partially Filled Attention Masks": coarse block mask + 32-bit packed fine
-// mask + pre-sorted non-empty key-block lists), with the block-id rule of
+// For Partially Filled Attention Masks": a coarse per-block mask, the partial
+// blocks' bits packed 32 to a word, and sorted lists of the non-empty key blocks), with the block-id rule of
 // opentau flash_attn_cuda and the BSR routing of flashinfer block_sparse_attention
 // as the other two mask sources.  Everything is deterministic: counts are integer
 // reductions, lists come from ballot prefix sums, and the order is a stable
@@ -367,8 +367,8 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
   block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
 }
 
-// Transposed lists for the backward's key-tile pass (BinFlash: "dKdV over
-// K-blocks"): for every key-tile column (group g, key tile kt), the ascending
+// Transposed lists for the backward's key-tile pass (BinFlash's dK/dV pass over
+// key blocks): for every key-tile column (group g, key tile kt), the ascending
 // query tiles whose class is not empty, each with its fine-word index when the
 // tile is partial (-1 when full), and the columns in longest-first order.
 // One CTA of 1024 threads; dynamic shared memory: max_nqt + 1 ints.

@@ -7,7 +7,7 @@ Definition restated from the pages:
 * output = softmax(scale * Q K^T + mask) V with a boolean mask, True = attend
   (BinFlash "Inputs": mask is (N, N) bool, True = attend; opentau
   ``flash_attn_blockmask``), masked scores are -inf before the softmax;
-* ``scale`` defaults to 1/sqrt(D) (BinFlash "Inputs" ``sm_scale``; tensorplay varlen
+* without an explicit ``scale`` the scores are multiplied by D^(-1/2) (BinFlash "Inputs" ``sm_scale``; tensorplay varlen
   keyword ``scale``; flashinfer ``sm_scale``);
 * LSE is the natural-log log-sum-exp of the scaled attended scores of a row
   (tensorplay omni_attention, "Outputs", ``return_lse``);

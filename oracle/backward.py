@@ -2,11 +2,10 @@
 
 Oracle (test infrastructure only).
 
-The pages ship a forward + backward (BinFlash: "Backward uses two passes (dKdV
-over K-blocks, dQ over Q-blocks)"; its usage example calls ``out.sum().backward()``
-and populates q.grad, k.grad, v.grad; opentau: "fused attention forward +
-backward"; tensorplay varlen: the log-sum-exp is the auxiliary output "that the
-backward pass reuses").  What the backward computes is the gradient of the
+The pages ship a forward and a backward (BinFlash runs the backward as two
+passes, dK/dV over key blocks and dQ over query blocks, and its usage example
+back-propagates ``out.sum()`` into q, k and v; opentau fuses both directions;
+tensorplay varlen returns the log-sum-exp so that the backward can use it again).  What the backward computes is the gradient of the
 forward's definition (``oracle.attention``) with respect to q, k and v, for an
 upstream gradient dO of the output.  Written out (the softmax Jacobian):
 

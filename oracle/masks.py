@@ -8,7 +8,7 @@ design notes):
 
 * block id of a token = inclusive running count of ``att_masks`` ones up to and
   including the token; tokens before the first 1 have id 0
-  (opentau ``make_att_block_ids``: "1 opens a new attention block, 0 continues").
+  (opentau ``make_att_block_ids``: a 1 starts a new block, a 0 extends the current one).
 * cross-attention key columns are prepended with block id INT32_MIN and their own
   padding mask, and they are still gated by the query's padding
   (opentau module docstring and ``make_att_block_ids`` parameters).
@@ -16,7 +16,8 @@ design notes):
   (tensorplay omni_attention, "Block masks", the ``causal`` predicate).
 * sliding window keeps keys with ``0 <= q_idx - kv_idx < W``
   (tensorplay omni_attention, "Block masks", the ``window`` predicate, where the
-  printed example keeps "at most 4 past keys" with ``q_idx - kv_idx < 4``).
+  printed example limits every query to its own key and the three before it,
+  written ``q_idx - kv_idx < 4``).
 * varlen: sequences packed along the token axis, delimited by ``cu_seqlens``
   starting at 0; positions are local to each sequence and keys of another
   sequence are never attended (tensorplay varlen, "Packed layout").

@@ -4,8 +4,8 @@ Oracle (test infrastructure only).  The plan restates BinFlash's preprocessing
 (BinFlash, "Efficiently Dispatching FlashAttention For Partially Filled Attention
 Masks"): the (N, N) bool mask is reduced to a coarse (N/BM x N/BN) block mask with
 three tile classes -- all-True ("full"), mixed ("partial") and all-False
-("empty") -- plus a 32-bit-packed fine mask for the partial tiles, and each row of
-query tiles gets a pre-sorted list of its non-empty key tiles.
+("empty") -- with the partial tiles' bits packed 32 to a word, and each row of
+query tiles gets its non-empty key tiles as a sorted list.
 
 Readings fixed here (the pages leave them open):
 
@@ -127,9 +127,9 @@ def plan_masks(masks, BM=128, BN=128):
 def transpose_plan(cls_groups):
     """Key-tile columns of a plan: the work lists of the backward's key-tile pass.
 
-    BinFlash ("Backward uses two passes (dKdV over K-blocks, dQ over Q-blocks)
-    with the same gathered-dispatch machinery"): the dK/dV pass visits, for every
-    key tile, the query tiles whose tile is not empty.  Column c enumerates the
+    BinFlash (its backward runs dK/dV over key blocks and dQ over query blocks,
+    from the same gathered block lists): the dK/dV pass visits, for every key
+    tile, the query tiles whose tile is not empty.  Column c enumerates the
     groups in order and, inside a group, the key tiles ascending; its list holds
     the query tiles qt with class(qt, kt) != empty, ascending, with a partial flag;
     columns are ordered longest first, ties by column index (the row order's rule).
