@@ -186,3 +186,45 @@ def test_bwd_rejects_bad_arguments():
     with pytest.raises(bfa.BfaError) as e:
         bfa.bwd(P, q.cpu(), q, q, out, q, lse)
     assert e.value.status == "BFA_ERR_NOT_DEVICE"
+
+
+def test_blockcausal_gqa_cross_columns_one_batch():
+    # the block-causal GQA workload (H=16 over Hkv=4, 256 cross columns, padding): all heads of one batch
+    w = workloads.blockcausal_gqa(B=2)
+    ids = bfa.make_att_block_ids(_cuda(w["pad_masks"]), _cuda(w["att_masks"]), w["n_cross"],
+                                 _cuda(w["cross_pad_masks"]))
+    P = bfa.plan_blockids(*ids)
+    dense = om.blockid_dense(*om.make_att_block_ids(w["pad_masks"], w["att_masks"], w["n_cross"],
+                                                    w["cross_pad_masks"]))
+    do = workloads.randn_bf16(tuple(w["q"].shape), 101)
+    qc, kc, vc, dc = w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), do.cuda()
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    dq, dk, dv = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    b = 1
+    rq, rk, rv = ob.attention_bwd_bshd(w["q"][b:b + 1], w["k"][b:b + 1], w["v"][b:b + 1], do[b:b + 1],
+                                       lambda _b, h: dense[b])
+    _close(dq[b:b + 1], rq, "dq")
+    _close(dk[b:b + 1], rk, "dk")
+    _close(dv[b:b + 1], rv, "dv")
+
+
+def test_causal_8192_bench_workload_sampled_heads():
+    # the bench's workload (B=4, H=32, N=8192, D=128) in the bench's launch; the oracle
+    # differentiates two (batch, head) pairs in full
+    w = workloads.causal_8192()
+    M = w["mask"].numpy()
+    do = workloads.randn_bf16(tuple(w["q"].shape), 4242)
+    qc, kc, vc, dc = w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), do.cuda()
+    P = bfa.plan_dense(w["mask"].cuda())
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    dq, dk, dv = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    for (b, h) in [(0, 0), (3, 31)]:
+        rq, rk, rv, _ = ob.masked_attention_bwd(w["q"][b, :, h], w["k"][b, :, h], w["v"][b, :, h], M,
+                                                do[b, :, h], w["scale"])
+        _close(dq[b, :, h], rq, f"dq {b},{h}")
+        _close(dk[b, :, h], rk, f"dk {b},{h}")
+        _close(dv[b, :, h], rv, f"dv {b},{h}")
