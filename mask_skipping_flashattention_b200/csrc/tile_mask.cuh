@@ -91,16 +91,24 @@ __device__ __forceinline__ void col_mask_words(const PlanDev& plan, const Ctx& w
   if (part < 0) {
     am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
   } else if (plan.mask_mode == MASK_BITS) {
-    // column `col` of the tile's row-major fine words: one word per query row,
-    // the same word for all lanes of a warp (col / 32 is warp-uniform)
+    // column `col` of the tile's row-major fine words.  A warp holds the keys
+    // 32 (col / 32) .. + 31; for each block of 32 query rows its lane l loads row
+    // l's word of those keys, and a 32 x 32 bit transpose across the warp (five
+    // butterfly rounds of shuffles) hands lane l the column of its own key.  All
+    // 32 lanes must call this together.
     const uint32_t* f = plan.fine + static_cast<int64_t>(part) * kFineWordsPerTile + (col >> 5);
-    const int b = col & 31;
+    const int lane = col & 31;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      uint32_t bits = 0;
-#pragma unroll 8
-      for (int i = 0; i < 32; ++i) bits |= ((__ldg(f + (32 * w + i) * kWordsPerTileRow) >> b) & 1u) << i;
-      am[w] = bits;
+      uint32_t x = __ldg(f + (32 * w + lane) * kWordsPerTileRow);
+#pragma unroll
+      for (int j = 16; j > 0; j >>= 1) {
+        const uint32_t m = j == 16 ? 0x0000ffffu : j == 8 ? 0x00ff00ffu : j == 4 ? 0x0f0f0f0fu
+                         : j == 2 ? 0x33333333u : 0x55555555u;
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+        x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
+      }
+      am[w] = x;
     }
   } else if (plan.mask_mode == MASK_BLOCKID) {
     const int32_t kb = plan.kid[wk.kid_off + kpos];
