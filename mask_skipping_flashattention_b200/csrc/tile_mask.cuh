@@ -113,13 +113,24 @@ __device__ __forceinline__ void col_mask_words(const PlanDev& plan, const Ctx& w
   } else if (plan.mask_mode == MASK_BLOCKID) {
     const int32_t kb = plan.kid[wk.kid_off + kpos];
     const bool kv = (plan.kbits[wk.kbit_off + (kpos >> 5)] >> (kpos & 31)) & 1u;
-    const int32_t* qb = plan.qid + wk.qid_off + qt * kTile;
-    const uint8_t* qv = plan.qvalid + wk.qid_off + qt * kTile;
+    // the tile's 128 query ids and validity bytes, read 16 bytes at a time (the
+    // per-group copies are padded to whole tiles, so each tile starts 16-byte aligned)
+    const int4* qb4 = reinterpret_cast<const int4*>(plan.qid + wk.qid_off + qt * kTile);
+    const uint4* qv16 = reinterpret_cast<const uint4*>(plan.qvalid + wk.qid_off + qt * kTile);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
+      const uint4 v16a = __ldg(qv16 + 2 * w), v16b = __ldg(qv16 + 2 * w + 1);
+      const uint32_t vw[8] = {v16a.x, v16a.y, v16a.z, v16a.w, v16b.x, v16b.y, v16b.z, v16b.w};
       uint32_t bits = 0;
-#pragma unroll 8
-      for (int i = 0; i < 32; ++i) bits |= ((qv[32 * w + i] != 0 && kb <= qb[32 * w + i]) ? 1u : 0u) << i;
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const int4 q = __ldg(qb4 + w * 8 + c4);
+        const uint32_t vb = vw[c4];
+        bits |= ((vb & 0xffu) != 0 && kb <= q.x ? 1u : 0u) << (c4 * 4 + 0);
+        bits |= ((vb & 0xff00u) != 0 && kb <= q.y ? 1u : 0u) << (c4 * 4 + 1);
+        bits |= ((vb & 0xff0000u) != 0 && kb <= q.z ? 1u : 0u) << (c4 * 4 + 2);
+        bits |= ((vb & 0xff000000u) != 0 && kb <= q.w ? 1u : 0u) << (c4 * 4 + 3);
+      }
       am[w] = kv ? bits : 0u;
     }
   } else if (plan.mask_mode == MASK_PRED) {
