@@ -6,6 +6,7 @@ for B=4, H=Hkv=32, N=8192, D=128.  FLOPs are counted on attended pairs only:
 4 * D * nnz per (batch, head), nnz = N (N + 1) / 2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bfa|reference]
+    python bench.py --sweep      # forward and backward on every workload, one JSON line each
 
 Multi-GPU (torchrun): every rank runs its own full workload (weak scaling, no
 collective on the data path); value = all ranks' FLOPs / max-over-ranks time.
@@ -352,6 +353,87 @@ def run_bfa(args, rank, world, local_rank):
     return 0
 
 
+def _time_ms(fn, reps):
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_sweep(args):
+    """Forward and backward throughput (attended-pair TFLOP/s) on every workload
+    configuration, one JSON line each (information; not the driver's metric line)."""
+    import numpy as np
+    import torch
+
+    import mask_skipping_flashattention_b200 as bfa
+    import workloads
+    from oracle import masks as om
+
+    torch.cuda.set_device(0)
+    reps = max(3, args.steps)
+
+    def cuda(x):
+        return torch.as_tensor(np.ascontiguousarray(x)).cuda()
+
+    def measure(name, P, q, k, v, pairs, D, plan_desc):
+        out, lse = bfa.fwd(P, q, k, v)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(7)
+        dout = torch.randn(q.shape, device="cuda", generator=g).to(torch.bfloat16)
+        fms = _time_ms(lambda: bfa.fwd(P, q, k, v, out=out, lse=lse), reps)
+        bms = _time_ms(lambda: bfa.bwd(P, q, k, v, out, dout, lse), reps)
+        P.device_status()
+        flops = 4.0 * D * pairs
+        print(json.dumps({"workload": name, "plan": plan_desc, "attended_pairs": pairs, "fwd_ms": fms,
+                          "fwd_tflops": flops / (fms * 1e-3) / 1e12, "bwd_ms": bms,
+                          "bwd_tflops": 2.5 * flops / (bms * 1e-3) / 1e12, "reps": reps}), flush=True)
+
+    w = workloads.causal_8192()
+    measure("causal_8192", bfa.plan_dense(w["mask"].cuda()), w["q"].cuda(), w["k"].cuda(), w["v"].cuda(),
+            float(w["mask"].sum()) * w["B"] * w["H"], w["D"], "dense")
+    del w
+    w = workloads.blockcausal_gqa()
+    ids = bfa.make_att_block_ids(cuda(w["pad_masks"]), cuda(w["att_masks"]), w["n_cross"], cuda(w["cross_pad_masks"]))
+    dense = om.blockid_dense(*om.make_att_block_ids(w["pad_masks"], w["att_masks"], w["n_cross"],
+                                                    w["cross_pad_masks"]))
+    measure("blockcausal_gqa", bfa.plan_blockids(*ids), w["q"].cuda(), w["k"].cuda(), w["v"].cuda(),
+            float(dense.sum()) * w["H"], w["D"], "block ids")
+    w = workloads.varlen_16()
+    cu = cuda(w["cu_seqlens"])
+    lens = np.diff(w["cu_seqlens"]).astype(np.int64)
+    for W in (-1, w["window"]):
+        P = bfa.plan_blockids(cu_seqlens_q=cu, cu_seqlens_k=cu, max_q=w["max_len"], max_k=w["max_len"],
+                              window_left=W)
+        per_head = float((lens * (lens + 1) // 2).sum()) if W < 0 else \
+            float(sum(int(np.minimum(np.arange(1, L + 1), W).sum()) for L in lens))
+        measure(f"varlen_16 window={W}", P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), per_head * 32, w["D"],
+                "varlen positions")
+    del w
+    w = workloads.bsr_16384()
+    ip, ix = w["block_indptr"], w["block_indices"]
+    nb = -(-w["S"] // w["block"])
+    per_group = 0.0
+    for b in range(ip.shape[0]):
+        for h in range(ip.shape[1]):
+            for r in range(nb):
+                sel = ix[ip[b, h, r]:ip[b, h, r + 1]]
+                per_group += float((sel < r).sum()) * 128 * 128 + float((sel == r).sum()) * 128 * 129 / 2
+    P = bfa.plan_bsr(cuda(ip), cuda(ix), w["S"], w["S"], w["block"], w["block"], causal=True)
+    measure("bsr_16384", P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), per_group * (w["H"] // w["Hkv"]), w["D"],
+            "BSR, causal inside blocks")
+    u = workloads.union_16384(with_qkv=False)
+    measure("union_16384", bfa.plan_dense(u["mask"].cuda()), w["q"].cuda(), w["k"].cuda(), w["v"].cuda(),
+            float(u["mask"].sum()) * w["B"] * w["H"], w["D"], "dense")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -359,6 +441,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["bfa", "reference"], default="bfa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="forward/backward on every workload (information)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -367,6 +450,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.sweep:
+        return run_sweep(args)
     return run_bfa(args, rank, world, local_rank)
 
 
