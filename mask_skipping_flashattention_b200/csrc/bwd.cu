@@ -15,17 +15,18 @@
 //               padded to whole tiles (HBM-bound, one pass over O and dO);
 //   k_bwd_dq    one CTA per (plan row, replica), walking the row's key-tile list:
 //               S = Q K^T and dP = dO V^T (SS), dS into TMEM as bf16, dQ += dS K
-//               (TS) chunk by chunk while the next chunk of dS is made; the mask
-//               on partial and edge tiles only;
+//               (TS); the next tile's S and dP run while this tile's dS is made
+//               (dS double-buffered in TMEM); the mask on partial and edge tiles
+//               only;
 //   k_bwd_dkdv  one CTA per (key-tile column, kv replica), walking the column's
 //               query-tile list for every query head of the kv head (GQA sums in
 //               TMEM, no atomics): S^T = K Q^T and dP^T = V dO^T (SS), P^T and dS^T
 //               into TMEM as bf16, dV += P^T dO and dK += dS^T Q (TS), chunk by
 //               chunk as in k_bwd_dq.
-// Warp roles of the two tile kernels (256 threads): warp 0 TMA producer, warp 1
-// TMEM owner and single-thread tcgen05.mma issuer, warps 4..7 one tile row per
-// thread (query rows in k_bwd_dq, key rows in k_bwd_dkdv).  Every wait is
-// bounded.
+// Warp roles of the two tile kernels: warp 0 TMA producer, warp 1 TMEM owner and
+// single-thread tcgen05.mma issuer; k_bwd_dq (384 threads): warps 4..11, one
+// query row per thread and half of the tile's keys per warp; k_bwd_dkdv (256
+// threads): warps 4..7, one key row per thread.  Every wait is bounded.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,6 +45,7 @@ namespace {
 
 constexpr int kBwdThreads = 256;
 constexpr int kBwdStages = 2;
+constexpr int kDqKStages = 3;  // K(u) stays until dQ(u) is done, a tile after V(u) is free
 
 template <int D>
 struct BCfg {
@@ -52,6 +54,8 @@ struct BCfg {
   static constexpr int kVecBytes = 2 * kTile * 4;  // LSE * log2(e) and D of one query tile
   // two resident tiles, then kBwdStages stages of two tiles (+ the vectors in k_bwd_dkdv)
   static constexpr int kSmemBytes = (2 + 2 * kBwdStages) * kTileBytes + kBwdStages * kVecBytes + 1024;
+  // k_bwd_dq: Q, dO, kDqKStages K stages and kBwdStages V stages
+  static constexpr int kDqSmemBytes = (2 + kDqKStages + kBwdStages) * kTileBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdescNN = idesc_bf16_f32(128, 128, 0);  // both operands K-major, N = 128
   static constexpr uint32_t kIdescD = idesc_bf16_f32(128, D, 1);     // B MN-major, N = D
@@ -206,8 +210,18 @@ struct DqWork {
   int32_t r, e0, n, qt, b, h, hk, j;
 };
 
+// Warp roles of k_bwd_dq (384 threads): warp 0 TMA producer, warp 1 TMEM owner
+// and MMA issuer, warps 2..3 idle, warps 4..11 the dS rows: warps 4..7 take keys
+// [0, 64) of a tile and warps 8..11 keys [64, 128), one query row per thread (a
+// warp reaches the TMEM lanes of its rank in the warpgroup).  Each warp loads its
+// half of S and dP at once and releases the S / dP columns, so the next tile's
+// S and dP products run on the tensor core while this tile's dS is made; dS
+// alternates between two TMEM buffers, so a tile's dS never overwrites the one
+// the previous tile's dQ products may still read.
+constexpr int kDqThreads = 384;
+
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const BwdParams p) {
   using C = BCfg<D>;
@@ -216,11 +230,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* const sQ = smem;
   uint8_t* const sdO = smem + C::kTileBytes;
   uint8_t* const sK0 = smem + 2 * C::kTileBytes;
-  uint8_t* const sV0 = smem + (2 + kBwdStages) * C::kTileBytes;
-  // BQ: Q and dO.  BF / BE [2]: K, V stage full / free.  BS: S and dP of the
-  // current tile ready.  BP [4]: dS of one 32-key chunk written (4 warps), so the
-  // dQ products of a chunk overlap the next chunk's dS.  BO: every product done.
-  enum { BQ = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 10, BDONE = 11, NBAR = 12 };
+  uint8_t* const sV0 = smem + (2 + kDqKStages) * C::kTileBytes;
+  // BQ: Q and dO.  BF [2]: K(u) and V(u) landed (by tile parity).  KE [3]: K
+  // stage free (dQ(u) done).  VE [2]: V stage free (dP(u) done).  BS: S and dP of
+  // a tile ready.  BC: every dS warp has loaded its S / dP columns (8 warps).
+  // BP [2]: dS of the tile written (8 warps), per tile parity, so a warp a tile
+  // ahead never arrives on a phase the MMA thread still waits for.  BO: every
+  // product done.
+  enum { BQ = 0, BF = 1, KE = 3, VE = 6, BS = 8, BC = 9, BP = 10, BO = 12, BDONE = 13, NBAR = 14 };
   __shared__ __align__(8) uint64_t bars[NBAR];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -232,7 +249,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= BP && i < BP + 4) ? 4 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == BC || i == BP || i == BP + 1) ? 8 : 1);
     fence_barrier_init();
     int i, j;
     chunked_decode(blockIdx.x, p.plan.n_rows, p.rep, p.head_chunk, i, j);
@@ -280,14 +297,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int u = 0; u < n; ++u) {
         const int kt = kt_next;
         if (u + 1 < n) kt_next = kv[u + 1];
-        const int st = u & 1;
-        if (u >= kBwdStages && !mbar_wait_fast(bar(BE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
+        const int st = u & 1, sk = u % kDqKStages;
+        // K(u) over K(u - 3) once dQ(u - 3) is done; V(u) over V(u - 2) once dP(u - 2) is
+        if (u >= kDqKStages && !mbar_wait_fast(bar(KE + sk), (u / kDqKStages - 1) & 1, cap, &abort_flag)) break;
+        if (u >= kBwdStages && !mbar_wait_fast(bar(VE + st), ((u >> 1) - 1) & 1, cap, &abort_flag)) break;
         const uint32_t f = bar(BF + st);
         mbar_expect_tx(f, 2 * C::kTileBytes);
         const int ks = wk.g.k_off + kt * kTile;
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_4d(smem_u32(sK(st) + pn * 16384), &tmK, f, pn * 64, wk.hk, ks, wk.b);
+          tma_load_4d(smem_u32(sK(sk) + pn * 16384), &tmK, f, pn * 64, wk.hk, ks, wk.b);
           tma_load_4d(smem_u32(sV(st) + pn * 16384), &tmV, f, pn * 64, wk.hk, ks, wk.b);
         }
         last[st] = u;
@@ -299,9 +318,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per tile u: once every dS warp holds S(u) and dP(u), S(u+1) and dP(u+1)
+    // go to the tensor core; then, once dS(u) is written, dQ += dS(u) K(u) in one
+    // burst (it queues behind S(u+1), dP(u+1), so finer grains gain nothing and
+    // cost a wait each).  The commit after S(t), dP(t) also frees V(t); the one
+    // after dQ(u) frees K(u).
     if (lane == 0 && n > 0) {
-      // TMEM: S [0,128), dP [128,256), dQ [256,256+D), dS (bf16 pairs) [384,448)
-      const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256, tdS = tmem + 384;
+      // TMEM: S [0,128), dP [128,256), dQ [256,256+D), dS (bf16 pairs) [384,448) / [448,512)
+      const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
       bool ok = mbar_wait_fast(bar(BQ), 0, cap, &abort_flag);
       if (ok) ok = mbar_wait_fast(bar(BF), 0, cap, &abort_flag);
       if (ok) {
@@ -309,31 +333,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_nn<D>(tS, sQ, sK(0));    // S = Q K^T
         issue_nn<D>(tdP, sdO, sV(0));  // dP = dO V^T
         umma_commit(bar(BS));
+        umma_commit(bar(VE + 0));
       }
-      bool started = false;
       for (int u = 0; ok && u < n; ++u) {
-        const int st = u & 1;
-        // dQ += dS K, chunk by chunk as the rows finish them
-        for (int cc = 0; cc < 4; ++cc) {
-          if (!mbar_wait_fast(bar(BP + cc), u & 1, cap, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk)
-            umma_ts(tdQ, tdS + kk * 8, smem_desc(smem_u32(sK(st) + kk * 2048), 16384, 1024), C::kIdescD,
-                    (started || kk > 0) ? 1u : 0u);
-        }
-        if (!ok) break;
-        started = true;
-        umma_commit(bar(BE + st));
-        // the rows have read all of S(u) and dP(u): the next tile's products
+        const int sk = u % kDqKStages;
+        const uint32_t tdS = tmem + 384 + 64 * (u & 1);
+        if (!mbar_wait_fast(bar(BC), u & 1, cap, &abort_flag)) { ok = false; break; }
         if (u + 1 < n) {
           const int st1 = (u + 1) & 1;
           if (!mbar_wait_fast(bar(BF + st1), ((u + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
           tc_fence_after();
-          issue_nn<D>(tS, sQ, sK(st1));
+          issue_nn<D>(tS, sQ, sK((u + 1) % kDqKStages));
           issue_nn<D>(tdP, sdO, sV(st1));
           umma_commit(bar(BS));
+          umma_commit(bar(VE + st1));
         }
+        if (!mbar_wait_fast(bar(BP + (u & 1)), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tdQ, tdS + kk * 8, smem_desc(smem_u32(sK(sk) + kk * 2048), 16384, 1024), C::kIdescD,
+                  (u > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(KE + sk));
       }
       if (ok) umma_commit(bar(BO));
       umma_commit(bar(BDONE));
@@ -343,6 +364,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dS rows
     const int quarter = warp & 3;
+    const int half = (warp >> 2) - 1;  // keys [64 half, 64 half + 64) of each tile
     const int row = quarter * 32 + lane;
     const int qpos = wk.qt * kTile + row;
     const uint32_t tLane = tmem_addr(tmem, quarter * 32, 0);
@@ -364,45 +386,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
       if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
       tc_fence_after();
-      // chunks of 32 keys; the loads of chunk cc + 1 are in flight while chunk cc
-      // is computed (two register sets, the loop fully unrolled)
-      uint32_t sA[32], dA[32], sB[32], dB[32];
-      tmem_ld_32x32b_x32(tLane, sA);
-      tmem_ld_32x32b_x32(tLane + 128, dA);
+      // this warp's 64 columns of S and dP in one round of loads; then the
+      // columns are released for the next tile's products
+      uint32_t sv[2][32], dv[2][32];
+      tmem_ld_32x32b_x32(tLane + 64 * half, sv[0]);
+      tmem_ld_32x32b_x32(tLane + 64 * half + 32, sv[1]);
+      tmem_ld_32x32b_x32(tLane + 128 + 64 * half, dv[0]);
+      tmem_ld_32x32b_x32(tLane + 128 + 64 * half + 32, dv[1]);
       tmem_wait_ld();
-      reg_fence(sA);
-      reg_fence(dA);
+      reg_fence(sv[0]);
+      reg_fence(sv[1]);
+      reg_fence(dv[0]);
+      reg_fence(dv[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BC));
+      const uint32_t tdS = tLane + 384 + 64 * (u & 1);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
-        uint32_t(&dp)[32] = (cc & 1) ? dB : dA;
-        if (cc + 1 < 4) {
-          tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
-          tmem_ld_32x32b_x32(tLane + 128 + (cc + 1) * 32, (cc & 1) ? dA : dB);
-        }
-        const uint32_t bits = am[cc];
+      for (int cc = 0; cc < 2; ++cc) {
+        const int gc = 2 * half + cc;  // 32-key chunk of the tile
+        const uint32_t bits = half ? am[2 + cc] : am[cc];
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           // masked scores become -inf (a select, no branch), so 2^(...) is 0
           const int c0 = 2 * jj, c1 = 2 * jj + 1;
-          const float s0 = ((bits >> c0) & 1u) ? __uint_as_float(sv[c0]) : -INFINITY;
-          const float s1 = ((bits >> c1) & 1u) ? __uint_as_float(sv[c1]) : -INFINITY;
+          const float s0 = ((bits >> c0) & 1u) ? __uint_as_float(sv[cc][c0]) : -INFINITY;
+          const float s1 = ((bits >> c1) & 1u) ? __uint_as_float(sv[cc][c1]) : -INFINITY;
           const float p0 = ex2_approx(fmaf(s0, c, nlse2));
           const float p1 = ex2_approx(fmaf(s1, c, nlse2));
-          pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dp[c0]) + nd), p1 * (__uint_as_float(dp[c1]) + nd));
+          pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dv[cc][c0]) + nd), p1 * (__uint_as_float(dv[cc][c1]) + nd));
         }
-        tmem_st_32x32b_x16(tLane + 384 + cc * 16, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BP + cc));
-        if (cc + 1 < 4) {
-          tmem_wait_ld();
-          reg_fence((cc & 1) ? sA : sB);
-          reg_fence((cc & 1) ? dA : dB);
-        }
+        tmem_st_32x32b_x16(tdS + gc * 16, pk);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BP + (u & 1)));
     }
     bool done = ok;
     if (ok && n > 0) {
@@ -414,7 +434,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int64_t tok = static_cast<int64_t>(wk.g.q_off) + qpos;
       __nv_bfloat16* dst =
           p.dq + static_cast<int64_t>(wk.b) * p.dq_sb + tok * p.dq_ss + static_cast<int64_t>(wk.h) * p.dq_sh;
-      store_row<D>(tLane + 256, n > 0, p.scale, dst, qpos < wk.g.q_len);
+      // each half of the warps writes half of the row's D columns
+      store_row<D / 2>(tLane + 256 + half * (D / 2), n > 0, p.scale, dst + half * (D / 2), qpos < wk.g.q_len);
     }
   }
 
@@ -673,7 +694,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ----------------------------------------------------------------------------
 // launchers (host)
 // ----------------------------------------------------------------------------
-int bwd_smem_bytes(int D) { return D == 64 ? BCfg<64>::kSmemBytes : BCfg<128>::kSmemBytes; }
+int bwd_smem_bytes(int D) {
+  return D == 64 ? max(BCfg<64>::kSmemBytes, BCfg<64>::kDqSmemBytes) : max(BCfg<128>::kSmemBytes, BCfg<128>::kDqSmemBytes);
+}
 
 cudaError_t launch_bwd_prep(const BwdParams& p, cudaStream_t s) {
   const int64_t blocks = static_cast<int64_t>(p.rep) * p.plan.n_rows;
@@ -694,13 +717,13 @@ cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tdo, 
   if (n_work <= 0) return cudaSuccess;
   if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (D == 64) {
-    static cudaError_t ready = bwd_prepare(k_bwd_dq<64>, BCfg<64>::kSmemBytes);
+    static cudaError_t ready = bwd_prepare(k_bwd_dq<64>, BCfg<64>::kDqSmemBytes);
     if (ready != cudaSuccess) return ready;
-    k_bwd_dq<64><<<static_cast<unsigned>(n_work), kBwdThreads, BCfg<64>::kSmemBytes, s>>>(tq, tdo, tk, tv, p);
+    k_bwd_dq<64><<<static_cast<unsigned>(n_work), kDqThreads, BCfg<64>::kDqSmemBytes, s>>>(tq, tdo, tk, tv, p);
   } else {
-    static cudaError_t ready = bwd_prepare(k_bwd_dq<128>, BCfg<128>::kSmemBytes);
+    static cudaError_t ready = bwd_prepare(k_bwd_dq<128>, BCfg<128>::kDqSmemBytes);
     if (ready != cudaSuccess) return ready;
-    k_bwd_dq<128><<<static_cast<unsigned>(n_work), kBwdThreads, BCfg<128>::kSmemBytes, s>>>(tq, tdo, tk, tv, p);
+    k_bwd_dq<128><<<static_cast<unsigned>(n_work), kDqThreads, BCfg<128>::kDqSmemBytes, s>>>(tq, tdo, tk, tv, p);
   }
   return cudaGetLastError();
 }
