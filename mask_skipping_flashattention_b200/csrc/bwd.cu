@@ -21,8 +21,9 @@
 //   k_bwd_dkdv  one CTA per (key-tile column, kv replica), walking the column's
 //               query-tile list for every query head of the kv head (GQA sums in
 //               TMEM, no atomics): S^T = K Q^T and dP^T = V dO^T (SS), P^T and dS^T
-//               into TMEM as bf16, dV += P^T dO and dK += dS^T Q (TS), chunk by
-//               chunk as in k_bwd_dq.
+//               into TMEM as bf16 over them, dV += P^T dO and dK += dS^T Q (TS);
+//               the products run in the order dV(s), S^T(s+1), dK(s), dP^T(s+1),
+//               so the next step's P^T is made while dK(s) and dP^T(s+1) run.
 // Warp roles of the two tile kernels: warp 0 TMA producer, warp 1 TMEM owner and
 // single-thread tcgen05.mma issuer; k_bwd_dq (384 threads): warps 4..11, one
 // query row per thread and half of the tile's keys per warp; k_bwd_dkdv (256
@@ -469,10 +470,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* const sQ0 = smem + 2 * C::kTileBytes;                      // + 2 st tiles
   float* const sVec0 = reinterpret_cast<float*>(smem + (2 + 2 * kBwdStages) * C::kTileBytes);  // + st * 256
   // BKV: K and V.  BF / BE [2]: Q, dO and the query vectors of a step full /
-  // free.  BS: S^T and dP^T ready.  BP [4]: P^T and dS^T of one 32-query chunk
-  // written (4 warps), so the chunk's dV, dK products overlap the next chunk.
-  // BO: every product done.
-  enum { BKV = 0, BF = 1, BE = 3, BS = 5, BP = 6, BO = 10, BDONE = 11, NBAR = 12 };
+  // free.  BS1 / BS2: S^T / dP^T of a step ready.  BP1 [4]: P^T of one 32-query
+  // chunk written, BP2: dS^T of the step written (4 warps each).  BO: every
+  // product done.
+  enum { BKV = 0, BF = 1, BE = 3, BS1 = 5, BS2 = 6, BP1 = 7, BP2 = 11, BO = 12, BDONE = 13, NBAR = 14 };
   __shared__ __align__(8) uint64_t bars[NBAR];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= BP && i < BP + 4) ? 4 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= BP1 && i <= BP2) ? 4 : 1);
     fence_barrier_init();
     int i, jk;
     chunked_decode(blockIdx.x, p.n_cols, p.rep_kv, p.kv_chunk, i, jk);
@@ -558,30 +559,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && steps > 0) {
+      // Pipe order: dV(s), S^T(s+1), dK(s), dP^T(s+1), dV(s+1), ...  S^T(s+1) goes
+      // over P^T(s) once dV(s) is issued and dP^T(s+1) over dS^T(s) once dK(s) is,
+      // so the rows turn S^T(s+1) into P^T(s+1) while dK(s) and dP^T(s+1) run.
       const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
       bool ok = mbar_wait_fast(bar(BKV), 0, cap, &abort_flag);
-      bool started = false;
-      for (int s = 0; ok && s < steps; ++s) {
-        const int st = s & 1;
-        if (!mbar_wait_fast(bar(BF + st), (s >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+      if (ok) ok = mbar_wait_fast(bar(BF), 0, cap, &abort_flag);
+      if (ok) {
         tc_fence_after();
-        issue_nn<D>(tS, sK, sQ(st));    // S^T = K Q^T (over P^T of step s - 1, in issue order)
-        issue_nn<D>(tdP, sV, sdO(st));  // dP^T = V dO^T
-        umma_commit(bar(BS));
-        // dV += P^T dO and dK += dS^T Q, chunk by chunk as the rows finish them
+        issue_nn<D>(tS, sK, sQ(0));  // S^T = K Q^T
+        umma_commit(bar(BS1));
+        issue_nn<D>(tdP, sV, sdO(0));  // dP^T = V dO^T
+        umma_commit(bar(BS2));
+      }
+      for (int s = 0; ok && s < steps; ++s) {
+        const int st = s & 1, st1 = st ^ 1;
+        // dV += P^T dO, chunk by chunk as the rows write P^T
         for (int cc = 0; cc < 4; ++cc) {
-          if (!mbar_wait_fast(bar(BP + cc), s & 1, cap, &abort_flag)) { ok = false; break; }
+          if (!mbar_wait_fast(bar(BP1 + cc), s & 1, cap, &abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk) {
-            const uint32_t acc = (started || kk > 0) ? 1u : 0u;
-            umma_ts(tdV, tS + kk * 8, smem_desc(smem_u32(sdO(st) + kk * 2048), 16384, 1024), C::kIdescD, acc);
-            umma_ts(tdK, tdP + kk * 8, smem_desc(smem_u32(sQ(st) + kk * 2048), 16384, 1024), C::kIdescD, acc);
-          }
+          for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk)
+            umma_ts(tdV, tS + kk * 8, smem_desc(smem_u32(sdO(st) + kk * 2048), 16384, 1024), C::kIdescD,
+                    (s > 0 || kk > 0) ? 1u : 0u);
         }
         if (!ok) break;
-        started = true;
+        if (s + 1 < steps) {
+          if (!mbar_wait_fast(bar(BF + st1), ((s + 1) >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_nn<D>(tS, sK, sQ(st1));
+          umma_commit(bar(BS1));
+        }
+        // dK += dS^T Q
+        if (!mbar_wait_fast(bar(BP2), s & 1, cap, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tdK, tdP + kk * 8, smem_desc(smem_u32(sQ(st) + kk * 2048), 16384, 1024), C::kIdescD,
+                  (s > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(BE + st));
+        if (s + 1 < steps) {
+          issue_nn<D>(tdP, sV, sdO(st1));
+          umma_commit(bar(BS2));
+        }
       }
       if (ok) umma_commit(bar(BO));
       umma_commit(bar(BDONE));
@@ -604,65 +624,95 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int qt = p.q_tile[e], part = p.tpart[e];
       uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (part >= 0 || (qt + 1) * kTile > wk.g.q_len) col_mask_words(p.plan, ctx, kpos, krow, qt, part, am);
-      // the step's query vectors (bulk copy on BF) and its S^T, dP^T (BS)
+      // the step's query vectors (bulk copy on BF) and its S^T (BS1)
       const bool gv = mbar_wait(bar(BF + st), (s >> 1) & 1, cap, &abort_flag);
-      const bool gs = gv && mbar_wait(bar(BS), s & 1, cap, &abort_flag);
+      const bool gs = gv && mbar_wait(bar(BS1), s & 1, cap, &abort_flag);
       if (__any_sync(0xffffffffu, !gs)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sLse = smem_u32(sVec(st)), sDv = smem_u32(sVec(st) + kTile);
-      // chunks of 32 queries, loads one chunk ahead as in k_bwd_dq (a chunk's
-      // P^T / dS^T columns never overlap the next chunk's S^T / dP^T columns)
-      uint32_t sA[32], dA[32], sB[32], dB[32];
-      tmem_ld_32x32b_x32(tLane, sA);
-      tmem_ld_32x32b_x32(tLane + 128, dA);
-      tmem_wait_ld();
-      reg_fence(sA);
-      reg_fence(dA);
+      // phase 1: P^T = 2^(scale log2(e) S^T - LSE log2(e)) for the 128 queries, kept
+      // in fp32 for phase 2 and written as bf16 over S^T (chunks of 32 queries,
+      // the next chunk's load in flight; a chunk's P^T columns lie in columns
+      // already read)
+      uint64_t pv[64];  // P pairs
+      {
+        uint32_t sA[32], sB[32];
+        tmem_ld_32x32b_x32(tLane, sA);
+        tmem_wait_ld();
+        reg_fence(sA);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
-        uint32_t(&dp)[32] = (cc & 1) ? dB : dA;
-        if (cc + 1 < 4) {
-          tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
-          tmem_ld_32x32b_x32(tLane + 128 + (cc + 1) * 32, (cc & 1) ? dA : dB);
-        }
-        const uint32_t bits = am[cc];
-        uint32_t pkp[16], pks[16];
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
+          if (cc + 1 < 4) tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
+          const uint32_t bits = am[cc];
+          uint32_t pkp[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 L = ld_shared_f4(sLse + (cc * 32 + q4 * 4) * 4);
-          const float4 Dv = ld_shared_f4(sDv + (cc * 32 + q4 * 4) * 4);
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 L = ld_shared_f4(sLse + (cc * 32 + q4 * 4) * 4);
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int col = q4 * 4 + 2 * h2;
-            // masked scores become -inf (a select, no branch), so 2^(...) is 0;
-            // pairs of columns through the packed fp32x2 fma / add / mul
-            const float s0 = ((bits >> col) & 1u) ? __uint_as_float(sv[col]) : -INFINITY;
-            const float s1 = ((bits >> (col + 1)) & 1u) ? __uint_as_float(sv[col + 1]) : -INFINITY;
-            const uint64_t nl = h2 ? f2_pack(L.z, L.w) : f2_pack(L.x, L.y);     // -LSE * log2(e)
-            const uint64_t nd = h2 ? f2_pack(Dv.z, Dv.w) : f2_pack(Dv.x, Dv.y);  // -D
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(s0, s1), c2, nl), x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            const uint64_t pp = f2_pack(p0, p1);
-            float d0, d1;
-            f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(dp[col]), __uint_as_float(dp[col + 1])), nd)), d0, d1);
-            pkp[2 * q4 + h2] = pack_bf16x2(p0, p1);
-            pks[2 * q4 + h2] = pack_bf16x2(d0, d1);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int col = q4 * 4 + 2 * h2;
+              // masked scores become -inf (a select, no branch), so 2^(...) is 0
+              const float s0 = ((bits >> col) & 1u) ? __uint_as_float(sv[col]) : -INFINITY;
+              const float s1 = ((bits >> (col + 1)) & 1u) ? __uint_as_float(sv[col + 1]) : -INFINITY;
+              const uint64_t nl = h2 ? f2_pack(L.z, L.w) : f2_pack(L.x, L.y);  // -LSE * log2(e)
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(s0, s1), c2, nl), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              pv[cc * 16 + 2 * q4 + h2] = f2_pack(p0, p1);
+              pkp[2 * q4 + h2] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st_32x32b_x16(tLane + cc * 16, pkp);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BP1 + cc));
+          if (cc + 1 < 4) {
+            tmem_wait_ld();
+            reg_fence((cc & 1) ? sA : sB);
           }
         }
-        tmem_st_32x32b_x16(tLane + cc * 16, pkp);        // P^T over S^T columns already read
-        tmem_st_32x32b_x16(tLane + 128 + cc * 16, pks);  // dS^T over dP^T columns already read
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BP + cc));
-        if (cc + 1 < 4) {
-          tmem_wait_ld();
-          reg_fence((cc & 1) ? sA : sB);
-          reg_fence((cc & 1) ? dA : dB);
+      }
+      // phase 2: dS^T = P^T * (dP^T - D), written as bf16 over dP^T
+      const bool gd = mbar_wait(bar(BS2), s & 1, cap, &abort_flag);
+      if (__any_sync(0xffffffffu, !gd)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t dA[32], dB[32];
+        tmem_ld_32x32b_x32(tLane + 128, dA);
+        tmem_wait_ld();
+        reg_fence(dA);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t(&dp)[32] = (cc & 1) ? dB : dA;
+          if (cc + 1 < 4) tmem_ld_32x32b_x32(tLane + 128 + (cc + 1) * 32, (cc & 1) ? dA : dB);
+          uint32_t pks[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 Dv = ld_shared_f4(sDv + (cc * 32 + q4 * 4) * 4);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int col = q4 * 4 + 2 * h2;
+              const uint64_t nd = h2 ? f2_pack(Dv.z, Dv.w) : f2_pack(Dv.x, Dv.y);  // -D
+              float d0, d1;
+              f2_unpack(f2_mul(pv[cc * 16 + 2 * q4 + h2],
+                               f2_add(f2_pack(__uint_as_float(dp[col]), __uint_as_float(dp[col + 1])), nd)),
+                        d0, d1);
+              pks[2 * q4 + h2] = pack_bf16x2(d0, d1);
+            }
+          }
+          tmem_st_32x32b_x16(tLane + 128 + cc * 16, pks);
+          if (cc + 1 < 4) {
+            tmem_wait_ld();
+            reg_fence((cc & 1) ? dA : dB);
+          }
         }
       }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BP2));
     }
     bool done = ok;
     if (ok && steps > 0) {

@@ -516,11 +516,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[64];
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, nm2), x0, x1);
-            const bool fma_pipe = (j & 7) < kPolyPairs;
-            const float p0 = fma_pipe ? ex2_poly(x0) : ex2_approx(x0);
-            const float p1 = fma_pipe ? ex2_poly(x1) : ex2_approx(x1);
+            const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, nm2);
+            float p0, p1;
+            if ((j & 7) < kPolyPairs) {  // this pair on the FMA pipe
+              f2_unpack(ex2_poly2(x2), p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             rs2[j & 3] = f2_add(rs2[j & 3], f2_pack(p0, p1));
             pk[j] = pack_bf16x2(p0, p1);
           }
@@ -607,11 +612,19 @@ __global__ void k_wait_selftest(uint32_t* err, uint64_t cap) {
 }
 
 // ----------------------------------------------------------------------------
-// FMA-pipe exp2 self test: y[i] = ex2_poly(x[i])
+// FMA-pipe exp2 self test: y[i] = 2^x[i], pairs through ex2_poly2 (the form the
+// softmax uses), a lone last element through ex2_poly
 // ----------------------------------------------------------------------------
 __global__ void k_exp2_selftest(const float* x, float* y, int64_t n) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = ex2_poly(x[i]);
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    float a, b;
+    f2_unpack(ex2_poly2(f2_pack(x[i], x[i + 1])), a, b);
+    y[i] = a;
+    y[i + 1] = b;
+  } else if (i < n) {
+    y[i] = ex2_poly(x[i]);
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -650,7 +663,7 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
 
 cudaError_t launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  k_exp2_selftest<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(x, y, n);
+  k_exp2_selftest<<<static_cast<unsigned>((n + 511) / 512), 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 

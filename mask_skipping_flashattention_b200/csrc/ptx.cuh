@@ -366,6 +366,24 @@ __device__ __forceinline__ float ex2_poly(float x) {
   q = fmaf(q, f, 1.0f);
   return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
+// ex2_poly on a pair of fp32 lanes, with the packed fp32x2 add and fma for the
+// rounding, the reduced argument and the polynomial (bit-identical to two
+// ex2_poly calls: the same operations lane by lane).
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));
+  const uint64_t f = f2_add(x, f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(12582912.f, 12582912.f)));  // x - (t - 1.5 2^23)
+  uint64_t q = f2_fma(f, f2_pack(5.500858277e-02f, 5.500858277e-02f), f2_pack(2.422103733e-01f, 2.422103733e-01f));
+  q = f2_fma(q, f, f2_pack(6.932829022e-01f, 6.932829022e-01f));
+  q = f2_fma(q, f, f2_pack(1.0f, 1.0f));
+  float t0, t1, q0, q1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(q, q0, q1);
+  return f2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
