@@ -383,7 +383,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         part_next = p.plan.part[wk.e0 + u + 1];
       }
       uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (part >= 0 || (kt + 1) * kTile > wk.g.k_len) row_mask_words(p.plan, ctx, qpos, row, kt, part, am);
+      const bool masked = part >= 0 || (kt + 1) * kTile > wk.g.k_len;
+      if (masked) row_mask_words(p.plan, ctx, qpos, row, kt, part, am);
       const bool got = mbar_wait(bar(BS), u & 1, cap, &abort_flag);
       if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
       tc_fence_after();
@@ -406,14 +407,17 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int gc = 2 * half + cc;  // 32-key chunk of the tile
-        const uint32_t bits = half ? am[2 + cc] : am[cc];
+        if (masked) {  // masked scores become -inf, so 2^(...) is 0 (partial and edge tiles only)
+          const uint32_t bits = half ? am[2 + cc] : am[cc];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (!((bits >> j) & 1u)) sv[cc][j] = __float_as_uint(-INFINITY);
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-          // masked scores become -inf (a select, no branch), so 2^(...) is 0
           const int c0 = 2 * jj, c1 = 2 * jj + 1;
-          const float s0 = ((bits >> c0) & 1u) ? __uint_as_float(sv[cc][c0]) : -INFINITY;
-          const float s1 = ((bits >> c1) & 1u) ? __uint_as_float(sv[cc][c1]) : -INFINITY;
+          const float s0 = __uint_as_float(sv[cc][c0]), s1 = __uint_as_float(sv[cc][c1]);
           const float p0 = ex2_approx(fmaf(s0, c, nlse2));
           const float p1 = ex2_approx(fmaf(s1, c, nlse2));
           pk[jj] = pack_bf16x2(p0 * (__uint_as_float(dv[cc][c0]) + nd), p1 * (__uint_as_float(dv[cc][c1]) + nd));
@@ -623,7 +627,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int e = step_entry(s);
       const int qt = p.q_tile[e], part = p.tpart[e];
       uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (part >= 0 || (qt + 1) * kTile > wk.g.q_len) col_mask_words(p.plan, ctx, kpos, krow, qt, part, am);
+      const bool masked = part >= 0 || (qt + 1) * kTile > wk.g.q_len;
+      if (masked) col_mask_words(p.plan, ctx, kpos, krow, qt, part, am);
       // the step's query vectors (bulk copy on BF) and its S^T (BS1)
       const bool gv = mbar_wait(bar(BF + st), (s >> 1) & 1, cap, &abort_flag);
       const bool gs = gv && mbar_wait(bar(BS1), s & 1, cap, &abort_flag);
@@ -644,7 +649,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
           if (cc + 1 < 4) tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
-          const uint32_t bits = am[cc];
+          if (masked) {  // masked scores become -inf, so 2^(...) is 0 (partial and edge steps only)
+            const uint32_t bits = am[cc];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (!((bits >> j) & 1u)) sv[j] = __float_as_uint(-INFINITY);
+          }
           uint32_t pkp[16];
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
@@ -652,9 +662,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int col = q4 * 4 + 2 * h2;
-              // masked scores become -inf (a select, no branch), so 2^(...) is 0
-              const float s0 = ((bits >> col) & 1u) ? __uint_as_float(sv[col]) : -INFINITY;
-              const float s1 = ((bits >> (col + 1)) & 1u) ? __uint_as_float(sv[col + 1]) : -INFINITY;
+              const float s0 = __uint_as_float(sv[col]), s1 = __uint_as_float(sv[col + 1]);
               const uint64_t nl = h2 ? f2_pack(L.z, L.w) : f2_pack(L.x, L.y);  // -LSE * log2(e)
               float x0, x1;
               f2_unpack(f2_fma(f2_pack(s0, s1), c2, nl), x0, x1);
