@@ -410,8 +410,9 @@ def run_sweep(args):
         g = torch.Generator(device="cuda")
         g.manual_seed(7)
         dout = torch.randn(q.shape, device="cuda", generator=g).to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         fms = _time_ms(lambda: bfa.fwd(P, q, k, v, out=out, lse=lse), reps)
-        bms = _time_ms(lambda: bfa.bwd(P, q, k, v, out, dout, lse), reps)
+        bms = _time_ms(lambda: bfa.bwd(P, q, k, v, out, dout, lse, dq=dq, dk=dk, dv=dv), reps)
         P.device_status()
         flops = 4.0 * D * pairs
         print(json.dumps({"workload": name, "plan": plan_desc, "attended_pairs": pairs, "fwd_ms": fms,
