@@ -847,8 +847,10 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
                                  void* out, const int64_t* os, float* lse, uint64_t wait_ns, cudaStream_t st,
                                  std::string* why, const PagedKV& pg = PagedKV(), float skip_log2 = 0.f) {
   const int bq = P->varlen ? 1 : B;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why)) return cudaErrorInvalidValue;
+  // the output with the query layout: whole in-range tiles leave through TMA stores
+  if (!make_tmap(&to, out, D, H, P->sq, bq, os[2], os[1], P->varlen ? 0 : os[0], why)) return cudaErrorInvalidValue;
   if (pg.page_size == 0) {
     if (!make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], why) ||
         !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], why))
@@ -919,7 +921,7 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.pages_per_seq = pg.pages_per_seq;
   p.skip_log2 = skip_log2;
   const int64_t n_work = units * items;
-  return launch_fwd(D, tq, tk, tv, p, n_work, st);
+  return launch_fwd(D, tq, tk, tv, to, p, n_work, st);
 }
 
 }  // namespace

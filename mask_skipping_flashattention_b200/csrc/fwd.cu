@@ -256,7 +256,8 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint8_t* sV, 
 template <int D, bool kSkip>
 __global__ void __launch_bounds__(kThreads, 1)
     bfa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -548,12 +549,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const bool store = qpos < wk.q_len;  // TMEM loads below stay whole-warp; only stores are per row
-      if (ok) {
+      const int h = slot ? wk.h[1] : wk.h[0];
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const int qt0 = (slot ? wk.qt[1] : wk.qt[0]) * kTile;  // first row of the tile in its group
+      if (qt0 + kTile <= wk.q_len) {
+        // A tile wholly inside its sequence leaves as one TMA store: each row goes,
+        // as bf16, into this slot's Q buffer (free: every product is done) in the
+        // 128-byte swizzled layout of the box, then one thread stores the tile.
+        // All four warps of the slot reach the barrier whatever happened before,
+        // and the store is skipped if any wait of the block gave up.
+        const uint32_t stg = smem_u32(slot ? sQ1 : sQ0);
+        if (ok) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            if (n > 0) {
+              tmem_ld_32x32b_x32(tO + cc * 32, o);
+              tmem_wait_ld();
+              reg_fence(o);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = 0u;
+            }
+            uint32_t pkd[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              pkd[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv, __uint_as_float(o[2 * j + 1]) * inv);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c16 = cc * 4 + j;  // 16-byte chunk of the row
+              const uint32_t addr = stg + (c16 >> 3) * 16384 + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
+              st_shared_v4(addr, pkd[4 * j], pkd[4 * j + 1], pkd[4 * j + 2], pkd[4 * j + 3]);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + slot, 128);
+        if (quarter == 0 && lane == 0 && ok && !*static_cast<volatile int*>(&abort_flag)) {
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_store_4d(&tmO, stg + pn * 16384, pn * 64, h, wk.q_off + qt0, wk.b);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+      } else if (ok) {
         const int64_t tok = static_cast<int64_t>(wk.q_off) + qpos;
-        const int h = slot ? wk.h[1] : wk.h[0];
         __nv_bfloat16* op =
             p.out + static_cast<int64_t>(wk.b) * p.o_sb + tok * p.o_ss + static_cast<int64_t>(h) * p.o_sh;
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -576,6 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[j] = make_uint4(pkd[4 * j], pkd[4 * j + 1], pkd[4 * j + 2], pkd[4 * j + 3]);
           }
         }
+      }
+      if (ok) {
+        const int64_t tok = static_cast<int64_t>(wk.q_off) + qpos;
         if (p.lse && store) {
           const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
           const int64_t li = p.varlen ? static_cast<int64_t>(h) * p.Sq_lse + tok
@@ -645,20 +690,21 @@ static cudaError_t prepare(K kernel, int smem) {
 
 template <int D, bool kSkip>
 static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const FwdParams& p, int64_t n_work, cudaStream_t s) {
+                              const CUtensorMap& to, const FwdParams& p, int64_t n_work, cudaStream_t s) {
   static cudaError_t ready = prepare(bfa_fwd_kernel<D, kSkip>, Cfg<D>::kSmemBytes);
   if (ready != cudaSuccess) return ready;
-  bfa_fwd_kernel<D, kSkip><<<static_cast<unsigned>(n_work), kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv, p);
+  bfa_fwd_kernel<D, kSkip><<<static_cast<unsigned>(n_work), kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdParams& p, int64_t n_work, cudaStream_t s) {
+                       const CUtensorMap& to, const FwdParams& p, int64_t n_work, cudaStream_t s) {
   if (n_work <= 0) return cudaSuccess;
   if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const bool approx = p.skip_log2 > 0.f;
-  if (D == 64) return approx ? launch_one<64, true>(tq, tk, tv, p, n_work, s) : launch_one<64, false>(tq, tk, tv, p, n_work, s);
-  return approx ? launch_one<128, true>(tq, tk, tv, p, n_work, s) : launch_one<128, false>(tq, tk, tv, p, n_work, s);
+  if (D == 64)
+    return approx ? launch_one<64, true>(tq, tk, tv, to, p, n_work, s) : launch_one<64, false>(tq, tk, tv, to, p, n_work, s);
+  return approx ? launch_one<128, true>(tq, tk, tv, to, p, n_work, s) : launch_one<128, false>(tq, tk, tv, to, p, n_work, s);
 }
 
 cudaError_t launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t s) {
