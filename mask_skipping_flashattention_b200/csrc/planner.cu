@@ -57,7 +57,14 @@ __global__ void __launch_bounds__(256) k_dense_classify(const uint8_t* __restric
       const uint8_t* p = mask + static_cast<int64_t>(qt * kTile + r) * ld + col0;
       if (vec_ok && col0 + 16 <= Sk) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-        m = nz_bytes4(v.x) | (nz_bytes4(v.y) << 4) | (nz_bytes4(v.z) << 8) | (nz_bytes4(v.w) << 12);
+        if (((v.x | v.y | v.z | v.w) & 0xFEFEFEFEu) == 0u) {
+          // bytes 0 / 1 (a bool tensor): one multiply gathers bit 0 of the four bytes
+          // of a word into bits 24..27, in byte order (no carries between the terms)
+          m = ((v.x * 0x01020408u) >> 24) | (((v.y * 0x01020408u) >> 24) << 4) |
+              (((v.z * 0x01020408u) >> 24) << 8) | (((v.w * 0x01020408u) >> 24) << 12);
+        } else {
+          m = nz_bytes4(v.x) | (nz_bytes4(v.y) << 4) | (nz_bytes4(v.z) << 8) | (nz_bytes4(v.w) << 12);
+        }
       } else {
         for (int c = 0; c < 16; ++c)
           if (col0 + c < Sk && p[c] != 0) m |= 1u << c;

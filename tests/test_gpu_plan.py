@@ -49,6 +49,13 @@ def test_dense_plan_strided_and_uint8_mask():
     t2 = _cuda(big.astype(np.uint8) * 7)[:, 1:300]   # nonzero bytes, unaligned base
     got = bfa.plan_dense(t2).export()
     assert_plan_equal(got, oracle_plan_for_groups([big[:, 1:300]]))
+    # aligned rows of bytes other than 0 / 1 (any nonzero byte attends), mixed with
+    # bool-like 16-byte runs: both ways of packing the bits on the vector path
+    vals = rng.integers(1, 256, size=big.shape).astype(np.uint8)
+    vals[:, :256] = 1
+    t3 = _cuda(np.where(big, vals, 0).astype(np.uint8))
+    got = bfa.plan_dense(t3).export()
+    assert_plan_equal(got, oracle_plan_for_groups([big]))
 
 
 def test_dense_plan_tiny_blockcausal():
