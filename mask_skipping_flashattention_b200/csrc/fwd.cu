@@ -285,6 +285,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == BP || i == BP + 1) ? 4 : 1);
     fence_barrier_init();
     decode_work(p, blockIdx.x, wk_s);
+    // Thread 0 is the TMA producer: the Q tiles go out as soon as the work item is
+    // known, before the block-wide barrier and the key list's first entry (K(0)
+    // follows on the same barrier, whose byte count covers it).
+    if (wk_s.n[0] + wk_s.n[1] > 0) {
+      prefetch_tmap(&tmQ);
+      mbar_expect_tx(bar(BQ), ((wk_s.n[0] > 0 ? 1 : 0) + (wk_s.n[1] > 0 ? 1 : 0) + 1) * C::kTileBytes);
+      for (int s = 0; s < 2; ++s) {
+        if (wk_s.n[s] == 0) continue;
+        const int qs = wk_s.q_off + wk_s.qt[s] * kTile;
+        uint8_t* dq = s ? sQ1 : sQ0;
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk_s.h[s], qs, wk_s.b);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_slot), C::kTmemCols);
@@ -303,11 +318,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsWG0>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      // Q of both slots and K of the first union tile on BQ; then at step j, V of
-      // union tile j and K of tile j + 1 together on F[j & 1], once the MMAs of
-      // commit j - 1 (which read the previous occupants of both stages) are done.
+      // Q of both slots (issued during the set-up) and K of the first union tile on
+      // BQ; then at step j, V of union tile j and K of tile j + 1 together on
+      // F[j & 1], once the MMAs of commit j - 1 (which read the previous occupants
+      // of both stages) are done.
       if (lane == 0 && any_tiles) {
-        prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
         UnionWalk walk;
@@ -315,15 +330,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kt, kt_n;
         bool ha, hb;
         walk.next(kt, ha, hb);  // any_tiles: the union has a first tile
-        mbar_expect_tx(bar(BQ), ((wk.n[0] > 0 ? 1 : 0) + (wk.n[1] > 0 ? 1 : 0) + 1) * C::kTileBytes);
-        for (int s = 0; s < 2; ++s) {
-          if (wk.n[s] == 0) continue;
-          const int qs = wk.q_off + wk.qt[s] * kTile;
-          uint8_t* dq = s ? sQ1 : sQ0;
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h[s], qs, wk.b);
-        }
         load_kv_tile<C::kPanels>(p, wk, &tmK, sK(0), bar(BQ), kt, wk.k_off + kt * kTile);
         int last_f[2] = {-1, -1};  // last step that filled F[0] / F[1]
         for (int j = 0;; ++j) {
