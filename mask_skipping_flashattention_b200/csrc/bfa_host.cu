@@ -35,7 +35,8 @@ cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, i
 cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row = nullptr, int32_t* pair_cost = nullptr,
-                        int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr, int part_is_pos = 0);
+                        int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr, int part_is_pos = 0,
+                        int2* row_work = nullptr, int2* pair_work = nullptr);
 cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int n_groups,
                                int nqb, int nkb, int wpr, uint32_t* bits, uint32_t* err, cudaStream_t s);
 cudaError_t launch_cols(const GroupInfo* groups, int n_groups, const uint8_t* cls, const int32_t* row_ptr,
@@ -91,6 +92,8 @@ struct bfa_plan {
   int32_t* pair_cost = nullptr;   // listed tiles of the pair
   int32_t* pair_order = nullptr;  // longest-first order of the pairs
   int32_t* pair_idx = nullptr;    // scratch: pair index of each row
+  int2* row_work = nullptr;       // rows in longest-first order with their group
+  int2* pair_work = nullptr;      // pairs in longest-first order with the group of their first row
   int32_t* qid = nullptr;
   uint8_t* qvalid = nullptr;
   int32_t* kid = nullptr;
@@ -215,6 +218,8 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   const size_t o_pcost = L.take<int32_t>(std::max(P->n_rows, 1));
   const size_t o_pord = L.take<int32_t>(std::max(P->n_rows, 1));
   const size_t o_pidx = L.take<int32_t>(std::max(P->n_rows, 1));
+  const size_t o_rwork = L.take<int2>(std::max(P->n_rows, 1));
+  const size_t o_pwork = L.take<int2>(std::max(P->n_rows, 1));
   const size_t o_err = L.take<uint32_t>(1);
   const size_t o_mw = L.take<int32_t>(1);
   const size_t o_qid = L.take<int32_t>(std::max<int64_t>(qid_elems, 1));
@@ -242,6 +247,8 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->pair_cost = reinterpret_cast<int32_t*>(base + o_pcost);
   P->pair_order = reinterpret_cast<int32_t*>(base + o_pord);
   P->pair_idx = reinterpret_cast<int32_t*>(base + o_pidx);
+  P->row_work = reinterpret_cast<int2*>(base + o_rwork);
+  P->pair_work = reinterpret_cast<int2*>(base + o_pwork);
   P->err = reinterpret_cast<uint32_t*>(base + o_err);
   P->max_width = reinterpret_cast<int32_t*>(base + o_mw);
   P->qid = reinterpret_cast<int32_t*>(base + o_qid);
@@ -292,7 +299,7 @@ bfa_status build_rows(bfa_plan* P, int part_is_pos = 0) {
   if (P->max_nkt > kMaxKvTiles) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
   cudaError_t e = launch_rows(P->groups, P->row_group, P->cls, P->n_rows, P->max_nkt, P->row_cnt, P->row_ptr,
                               P->kv_tile, P->part, P->order, P->stream, P->pair_row, P->pair_cost,
-                              P->pair_order, P->pair_idx, part_is_pos);
+                              P->pair_order, P->pair_idx, part_is_pos, P->row_work, P->pair_work);
   return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
 }
 
@@ -870,6 +877,8 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.plan.part = P->part;
   p.plan.fine = P->fine;
   p.plan.order = P->order;
+  p.plan.row_work = P->row_work;
+  p.plan.pair_work = P->pair_work;
   p.plan.qid = P->qid;
   p.plan.qvalid = P->qvalid;
   p.plan.kid = P->kid;
@@ -995,6 +1004,8 @@ bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const
   p.plan.part = P->part;
   p.plan.fine = P->fine;
   p.plan.order = P->order;
+  p.plan.row_work = P->row_work;
+  p.plan.pair_work = P->pair_work;
   p.plan.qid = P->qid;
   p.plan.qvalid = P->qvalid;
   p.plan.kid = P->kid;

@@ -254,9 +254,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     fence_barrier_init();
     int i, j;
     chunked_decode(blockIdx.x, p.plan.n_rows, p.rep, p.head_chunk, i, j);
-    const int r = p.plan.order[i];
+    const int2 rw = p.plan.row_work[i];  // {row, its group}, longest first
+    const int r = rw.x;
     DqWork w;
-    w.g = p.plan.groups[p.plan.row_group[r]];
+    w.g = p.plan.groups[rw.y];
     w.r = r;
     w.e0 = p.plan.row_ptr[r];
     w.n = p.plan.row_ptr[r + 1] - w.e0;

@@ -107,15 +107,18 @@ __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk)
   const int64_t gs = min(chunk, items - hg * chunk);
   const int i = static_cast<int>(rem / gs);
   const int j = static_cast<int>(hg * chunk + rem % gs);
-  int r0, r1;
+  // the plan lists the work items in longest-first order with their group
+  int r0, r1, grp;
   if (p.pair_heads) {
-    r0 = r1 = p.plan.order[i];
+    const int2 rw = p.plan.row_work[i];
+    r0 = r1 = rw.x;
+    grp = rw.y;
   } else {
-    const int pr = p.plan.pair_row[p.plan.pair_order[i]];
-    r0 = pr >= 0 ? pr : ~pr;
-    r1 = pr >= 0 ? r0 + 1 : -1;
+    const int2 pw = p.plan.pair_work[i];
+    r0 = pw.x >= 0 ? pw.x : ~pw.x;
+    r1 = pw.x >= 0 ? r0 + 1 : -1;
+    grp = pw.y;
   }
-  const int grp = p.plan.row_group[r0];
   const GroupInfo g = p.plan.groups[grp];
   wk.same_row = p.pair_heads;
   wk.row[0] = r0;

@@ -52,6 +52,8 @@ struct PlanDev {
   const int32_t* order;      // [n_rows] longest first
   const int32_t* pair_row;   // [n_pairs] first row of each work pair (~row: single row)
   const int32_t* pair_order; // [n_pairs] longest first
+  const int2* row_work;      // [n_rows] longest first: {row, group of the row}
+  const int2* pair_work;     // [n_pairs] longest first: {pair_row, group of its first row}
   const int32_t* qid;        // padded q block ids  (block-id plans)
   const uint8_t* qvalid;     // padded q validity   (block-id plans)
   const int32_t* kid;        // padded k block ids  (block-id plans)

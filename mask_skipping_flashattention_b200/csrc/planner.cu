@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
                                                int32_t* __restrict__ kv_tile, int32_t* __restrict__ part,
                                                int32_t* __restrict__ order, int32_t* __restrict__ pair_row,
                                                int32_t* __restrict__ pair_cost, int32_t* __restrict__ pair_order,
-                                               int32_t* __restrict__ pair_idx, int part_is_pos) {
+                                               int32_t* __restrict__ pair_idx, int part_is_pos,
+                                               int2* __restrict__ row_work, int2* __restrict__ pair_work) {
   extern __shared__ int32_t bucket[];
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
@@ -353,6 +354,10 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
   // 4. longest-first stable row order
   __syncthreads();
   block_stable_order_desc(n_rows, row_cnt, max_nkt, bucket, order);
+  // work items in that order with the group of their row, so a kernel finds its
+  // row and group with one load
+  if (row_work != nullptr)
+    for (int i = tid; i < n_rows; i += blockDim.x) row_work[i] = make_int2(order[i], row_group[order[i]]);
   if (pair_row == nullptr) return;
 
   // 5. pairs: a row opens a pair when its tile index inside its group is even;
@@ -372,6 +377,11 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
   }
   __syncthreads();
   block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
+  if (pair_work != nullptr)
+    for (int i = tid; i < n_pairs; i += blockDim.x) {
+      const int pr = pair_row[pair_order[i]];
+      pair_work[i] = make_int2(pr, row_group[pr >= 0 ? pr : ~pr]);
+    }
 }
 
 // Transposed lists for the backward's key-tile pass (BinFlash's dK/dV pass over
@@ -755,7 +765,8 @@ cudaError_t launch_bsr_classify(const int32_t* indptr, const int32_t* indices, i
 cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const uint8_t* cls, int n_rows,
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row, int32_t* pair_cost,
-                        int32_t* pair_order, int32_t* pair_idx, int part_is_pos) {
+                        int32_t* pair_order, int32_t* pair_idx, int part_is_pos, int2* row_work,
+                        int2* pair_work) {
   const size_t smem = sizeof(int32_t) * static_cast<size_t>(2 * max_nkt + 1);
   if (smem > 48 * 1024) {
     cudaError_t e =
@@ -763,7 +774,7 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
     if (e != cudaSuccess) return e;
   }
   k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order,
-                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos);
+                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos, row_work, pair_work);
   return cudaGetLastError();
 }
 
