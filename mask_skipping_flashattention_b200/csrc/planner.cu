@@ -296,6 +296,26 @@ __device__ void block_stable_order_desc(int n, const int32_t* keys, int max_key,
   }
 }
 
+// The same order for n <= kSmallOrder keys: every thread ranks its own element
+// directly (larger keys first, ties by index) against the keys in shared memory;
+// cheaper than the bucket passes for the few hundred rows most plans have.
+constexpr int kSmallOrder = 256;
+__device__ void block_stable_order_desc_small(int n, const int32_t* keys, int32_t* skeys, int32_t* order) {
+  const int tid = threadIdx.x;
+  if (tid < n) skeys[tid] = keys[tid];
+  __syncthreads();
+  if (tid < n) {
+    const int k = skeys[tid];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const int kj = skeys[j];
+      rank += (kj > k || (kj == k && j < tid)) ? 1 : 0;
+    }
+    order[rank] = tid;
+  }
+  __syncthreads();
+}
+
 // Rows -> lists and row order; with pair outputs also the work pairs (two
 // consecutive query tiles of one group) and their longest-first order.
 // Dynamic shared memory: (2 * max_nkt + 1) ints.
@@ -309,6 +329,7 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
                                                int32_t* __restrict__ pair_idx, int part_is_pos,
                                                int2* __restrict__ row_work, int2* __restrict__ pair_work) {
   extern __shared__ int32_t bucket[];
+  __shared__ int32_t small_keys[kSmallOrder];
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
@@ -353,7 +374,8 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
 
   // 4. longest-first stable row order
   __syncthreads();
-  block_stable_order_desc(n_rows, row_cnt, max_nkt, bucket, order);
+  if (n_rows <= kSmallOrder) block_stable_order_desc_small(n_rows, row_cnt, small_keys, order);
+  else block_stable_order_desc(n_rows, row_cnt, max_nkt, bucket, order);
   // work items in that order with the group of their row, so a kernel finds its
   // row and group with one load
   if (row_work != nullptr)
@@ -376,7 +398,8 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
     pair_cost[pi] = row_cnt[r] + (two ? row_cnt[r + 1] : 0);
   }
   __syncthreads();
-  block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
+  if (n_pairs <= kSmallOrder) block_stable_order_desc_small(n_pairs, pair_cost, small_keys, pair_order);
+  else block_stable_order_desc(n_pairs, pair_cost, 2 * max_nkt, bucket, pair_order);
   if (pair_work != nullptr)
     for (int i = tid; i < n_pairs; i += blockDim.x) {
       const int pr = pair_row[pair_order[i]];
