@@ -56,7 +56,8 @@ cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B,
 cudaError_t launch_pred_classify(const int32_t* terms, int n_terms, const GroupInfo* groups, int n_groups, int nqt,
                                  uint8_t* cls, cudaStream_t s);
 cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
-                                       GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s);
+                                       GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s,
+                                       uint32_t* err = nullptr, int32_t* max_width = nullptr);
 
 
 }  // namespace bfa
@@ -259,8 +260,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->fine = reinterpret_cast<uint32_t*>(base + o_fine);
 
   if (P->regular) {
+    // the same launch clears the status words (err, max_width)
     e = launch_init_regular_groups(P->groups_h[0], P->n_groups, P->regular_hkv, P->kind == BFA_PLAN_BSR ? 1 : 0,
-                                   P->copy_ids ? 1 : 0, P->groups, P->row_group, P->n_rows, P->stream);
+                                   P->copy_ids ? 1 : 0, P->groups, P->row_group, P->n_rows, P->stream, P->err,
+                                   P->max_width);
     if (e != cudaSuccess) return cuda_fail(e, "plan group table kernel");
   } else {
     // irregular (varlen) layouts: the planner has synchronised already to read
@@ -276,8 +279,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
     e = cudaMemcpyAsync(P->row_group, rg.data(), sizeof(int32_t) * rg.size(), cudaMemcpyHostToDevice, P->stream);
     if (e != cudaSuccess) return cuda_fail(e, "upload plan rows");
   }
-  e = cudaMemsetAsync(P->err, 0, 2 * 256, P->stream);  // err and max_width slots
-  if (e != cudaSuccess) return cuda_fail(e, "clear plan status");
+  if (!P->regular) {  // regular layouts cleared them in the group-table launch
+    e = cudaMemsetAsync(P->err, 0, 2 * 256, P->stream);  // err and max_width slots
+    if (e != cudaSuccess) return cuda_fail(e, "clear plan status");
+  }
   return BFA_OK;
 }
 

@@ -722,8 +722,12 @@ __global__ void __launch_bounds__(1024) k_make_block_ids(const uint8_t* __restri
 // ----------------------------------------------------------------------------
 __global__ void k_init_regular_groups(GroupInfo tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
                                       GroupInfo* __restrict__ groups, int32_t* __restrict__ row_group,
-                                      int n_rows) {
+                                      int n_rows, uint32_t* __restrict__ err, int32_t* __restrict__ max_width) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i == 0 && err != nullptr) {  // the plan's status words start cleared
+    *err = 0u;
+    *max_width = 0;
+  }
   if (i < n_groups) {
     GroupInfo g = tmpl;
     g.b = (tmpl.b < 0) ? -1 : i / n_hkv;
@@ -742,11 +746,15 @@ __global__ void k_init_regular_groups(GroupInfo tmpl, int n_groups, int n_hkv, i
 // launchers (host)
 // ----------------------------------------------------------------------------
 cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
-                                       GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s) {
-  const int n = n_groups > n_rows ? n_groups : n_rows;
-  if (n <= 0) return cudaSuccess;
+                                       GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s,
+                                       uint32_t* err, int32_t* max_width) {
+  int n = n_groups > n_rows ? n_groups : n_rows;
+  if (n <= 0) {
+    if (err == nullptr) return cudaSuccess;
+    n = 1;  // the status words still need clearing
+  }
   k_init_regular_groups<<<(n + 255) / 256, 256, 0, s>>>(tmpl, n_groups, n_hkv, bsr, copy_ids, groups, row_group,
-                                                       n_rows);
+                                                       n_rows, err, max_width);
   return cudaGetLastError();
 }
 
