@@ -30,23 +30,51 @@ __device__ __forceinline__ void row_mask_words(const PlanDev& plan, const Ctx& w
     }
   } else if (plan.mask_mode == MASK_BLOCKID) {
     if (part >= 0) {
+      // called by whole warps (the tile is the same for the warp's 32 rows)
       const int32_t qb = plan.qid[wk.qid_off + qpos];
       const bool qv = plan.qvalid[wk.qid_off + qpos] != 0;
-      const int4* kb4 = reinterpret_cast<const int4*>(plan.kid + wk.kid_off + kt * kTile);
+      const int32_t* kids = plan.kid + wk.kid_off + kt * kTile;
+      const int4* kb4 = reinterpret_cast<const int4*>(kids);
       const uint4 kv = __ldg(reinterpret_cast<const uint4*>(plan.kbits + wk.kbit_off + kt * kWordsPerTileRow));
       const uint32_t kvw[4] = {kv.x, kv.y, kv.z, kv.w};
+      // Key ids non-decreasing across the tile (the usual form: cross columns at
+      // INT32_MIN, then running block counts) make {j : k_blk[j] <= q_blk} a prefix
+      // of the tile, whose length one binary search finds; otherwise every key is
+      // compared.  The warp checks the order with one 16-byte load per lane.
+      const int lane = row & 31;
+      const int4 mine = __ldg(kb4 + lane);
+      const int prev = __shfl_up_sync(0xffffffffu, mine.w, 1);
+      const bool in_order = mine.x <= mine.y && mine.y <= mine.z && mine.z <= mine.w && (lane == 0 || prev <= mine.x);
+      if (__all_sync(0xffffffffu, in_order)) {
+        int lo = 0, hi = kTile;  // the first key with k_blk > q_blk lies in [lo, hi]
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t bits = 0;
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const int4 k = __ldg(kb4 + w * 8 + c4);
-          bits |= (k.x <= qb ? 1u : 0u) << (c4 * 4 + 0);
-          bits |= (k.y <= qb ? 1u : 0u) << (c4 * 4 + 1);
-          bits |= (k.z <= qb ? 1u : 0u) << (c4 * 4 + 2);
-          bits |= (k.w <= qb ? 1u : 0u) << (c4 * 4 + 3);
+        for (int it = 0; it < 8; ++it) {
+          if (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(kids + mid) <= qb) lo = mid + 1;
+            else hi = mid;
+          }
         }
-        am[w] = qv ? (bits & kvw[w]) : 0u;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int z = lo - 32 * w;  // attended keys of this word: [0, z)
+          const uint32_t bits = (z >= 32) ? 0xffffffffu : (z <= 0 ? 0u : ((1u << z) - 1u));
+          am[w] = qv ? (bits & kvw[w]) : 0u;
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          uint32_t bits = 0;
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const int4 k = __ldg(kb4 + w * 8 + c4);
+            bits |= (k.x <= qb ? 1u : 0u) << (c4 * 4 + 0);
+            bits |= (k.y <= qb ? 1u : 0u) << (c4 * 4 + 1);
+            bits |= (k.z <= qb ? 1u : 0u) << (c4 * 4 + 2);
+            bits |= (k.w <= qb ? 1u : 0u) << (c4 * 4 + 3);
+          }
+          am[w] = qv ? (bits & kvw[w]) : 0u;
+        }
       }
     } else {
       am[0] = am[1] = am[2] = am[3] = 0xffffffffu;
