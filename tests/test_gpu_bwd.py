@@ -86,6 +86,25 @@ def test_blockids_with_padding_and_cross_columns():
     assert torch.all(dk[0, 240:] == 0) and torch.all(dv[0, 240:] == 0)
 
 
+def test_blockids_unsorted_and_sorted_key_tiles():
+    # arbitrary key-id order on some key tiles, non-decreasing on others: both forms
+    # of the block-id mask in the dQ pass (rows) and the dK/dV pass (columns)
+    rng = np.random.default_rng(77)
+    B, Sq, Sk, H, D = 1, 300, 400, 2, 64
+    qb = np.sort(rng.integers(0, 9, size=(B, Sq)), axis=1).astype(np.int32)
+    kb = rng.integers(-2, 10, size=(B, Sk)).astype(np.int32)
+    kb[:, 128:256] = np.sort(kb[:, 128:256], axis=1)
+    qv = rng.random((B, Sq)) < 0.9
+    kv = rng.random((B, Sk)) < 0.85
+    P = bfa.plan_blockids(_cuda(qb), _cuda(kb), _cuda(qv), _cuda(kv))
+    M = om.blockid_dense(qb, kb, qv, kv)
+    q = workloads.randn_bf16((B, Sq, H, D), 91)
+    k = workloads.randn_bf16((B, Sk, H, D), 92)
+    v = workloads.randn_bf16((B, Sk, H, D), 93)
+    do = workloads.randn_bf16((B, Sq, H, D), 94)
+    _run_bshd(P, q, k, v, do, lambda b, h: M[b])
+
+
 def test_positional_window_batched():
     B, H, Sq, Sk, D, W = 2, 2, 700, 650, 64, 100
     P = bfa.plan_blockids(B=B, Sq=Sq, Sk=Sk, window_left=W)

@@ -62,6 +62,30 @@ def test_blockcausal_gqa_cross_columns():
     check_bshd(out.cpu(), lse.cpu(), w["q"], w["k"], w["v"], lambda b, h: dense[b], None, pairs, where="cfg3")
 
 
+@pytest.mark.parametrize("seed", range(2))
+def test_blockids_unsorted_and_sorted_key_tiles(seed):
+    # key ids in arbitrary order on some key tiles (every key compared) and
+    # non-decreasing on others (one binary search per row): both forms of the
+    # block-id mask against the dense mask the ids define
+    rng = np.random.default_rng(70 + seed)
+    B, Sq, Sk, H, D = 2, 300, 520, 2, 64
+    qb = np.sort(rng.integers(0, 9, size=(B, Sq)), axis=1).astype(np.int32)
+    kb = rng.integers(-2, 10, size=(B, Sk)).astype(np.int32)
+    kb[:, 128:384] = np.sort(kb[:, 128:384], axis=1)      # key tiles 1 and 2 in order
+    kb[:, :7] = np.iinfo(np.int32).min
+    qv = rng.random((B, Sq)) < 0.9
+    kv = rng.random((B, Sk)) < 0.85
+    P = bfa.plan_blockids(_cuda(qb), _cuda(kb), _cuda(qv), _cuda(kv))
+    dense = om.blockid_dense(qb, kb, qv, kv)
+    q = _rand((B, Sq, H, D), 81 + seed)
+    k = _rand((B, Sk, H, D), 83 + seed)
+    v = _rand((B, Sk, H, D), 85 + seed)
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: dense[b], None, pairs, where="unsorted ids")
+
+
 # ---------------------------------------------------------------- causal 8192
 def test_causal_8192_reduced_heads_all_rows():
     w = workloads.causal_8192(B=1, H=2)
