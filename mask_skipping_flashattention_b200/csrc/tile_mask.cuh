@@ -143,23 +143,54 @@ __device__ __forceinline__ void col_mask_words(const PlanDev& plan, const Ctx& w
     const bool kv = (plan.kbits[wk.kbit_off + (kpos >> 5)] >> (kpos & 31)) & 1u;
     // the tile's 128 query ids and validity bytes, read 16 bytes at a time (the
     // per-group copies are padded to whole tiles, so each tile starts 16-byte aligned)
-    const int4* qb4 = reinterpret_cast<const int4*>(plan.qid + wk.qid_off + qt * kTile);
+    const int32_t* qids = plan.qid + wk.qid_off + qt * kTile;
+    const int4* qb4 = reinterpret_cast<const int4*>(qids);
     const uint4* qv16 = reinterpret_cast<const uint4*>(plan.qvalid + wk.qid_off + qt * kTile);
+    // Whole warps call this (one tile per warp).  Query ids non-decreasing over the
+    // tile with every query valid (the usual form) make the attended rows a suffix
+    // {i : q_blk[i] >= k_blk}, found by one binary search; otherwise every query is
+    // compared.  The warp checks with one 16-byte id load and one 4-byte validity
+    // load per lane.
+    const int lane = col & 31;
+    const int4 mine = __ldg(qb4 + lane);
+    const uint32_t vmine = __ldg(reinterpret_cast<const uint32_t*>(qv16) + lane);
+    const int prev = __shfl_up_sync(0xffffffffu, mine.w, 1);
+    const bool fast = mine.x <= mine.y && mine.y <= mine.z && mine.z <= mine.w && (lane == 0 || prev <= mine.x) &&
+                      (vmine & 0xffu) != 0 && (vmine & 0xff00u) != 0 && (vmine & 0xff0000u) != 0 &&
+                      (vmine & 0xff000000u) != 0;
+    if (__all_sync(0xffffffffu, fast)) {
+      int lo = 0, hi = kTile;  // the first query with q_blk >= k_blk lies in [lo, hi]
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const uint4 v16a = __ldg(qv16 + 2 * w), v16b = __ldg(qv16 + 2 * w + 1);
-      const uint32_t vw[8] = {v16a.x, v16a.y, v16a.z, v16a.w, v16b.x, v16b.y, v16b.z, v16b.w};
-      uint32_t bits = 0;
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const int4 q = __ldg(qb4 + w * 8 + c4);
-        const uint32_t vb = vw[c4];
-        bits |= ((vb & 0xffu) != 0 && kb <= q.x ? 1u : 0u) << (c4 * 4 + 0);
-        bits |= ((vb & 0xff00u) != 0 && kb <= q.y ? 1u : 0u) << (c4 * 4 + 1);
-        bits |= ((vb & 0xff0000u) != 0 && kb <= q.z ? 1u : 0u) << (c4 * 4 + 2);
-        bits |= ((vb & 0xff000000u) != 0 && kb <= q.w ? 1u : 0u) << (c4 * 4 + 3);
+      for (int it = 0; it < 8; ++it) {
+        if (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (__ldg(qids + mid) < kb) lo = mid + 1;
+          else hi = mid;
+        }
       }
-      am[w] = kv ? bits : 0u;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int a = lo - 32 * w;  // attended rows of this word: [a, 32)
+        const uint32_t bits = (a <= 0) ? 0xffffffffu : (a >= 32 ? 0u : ~((1u << a) - 1u));
+        am[w] = kv ? bits : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint4 v16a = __ldg(qv16 + 2 * w), v16b = __ldg(qv16 + 2 * w + 1);
+        const uint32_t vw[8] = {v16a.x, v16a.y, v16a.z, v16a.w, v16b.x, v16b.y, v16b.z, v16b.w};
+        uint32_t bits = 0;
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const int4 q = __ldg(qb4 + w * 8 + c4);
+          const uint32_t vb = vw[c4];
+          bits |= ((vb & 0xffu) != 0 && kb <= q.x ? 1u : 0u) << (c4 * 4 + 0);
+          bits |= ((vb & 0xff00u) != 0 && kb <= q.y ? 1u : 0u) << (c4 * 4 + 1);
+          bits |= ((vb & 0xff0000u) != 0 && kb <= q.z ? 1u : 0u) << (c4 * 4 + 2);
+          bits |= ((vb & 0xff000000u) != 0 && kb <= q.w ? 1u : 0u) << (c4 * 4 + 3);
+        }
+        am[w] = kv ? bits : 0u;
+      }
     }
   } else if (plan.mask_mode == MASK_PRED) {
     pred_words_col(plan.terms, plan.n_terms, kpos, qt, wk.q_len, am);
