@@ -247,3 +247,62 @@ def test_causal_8192_bench_workload_sampled_heads():
         _close(dq[b, :, h], rq, f"dq {b},{h}")
         _close(dk[b, :, h], rk, f"dk {b},{h}")
         _close(dv[b, :, h], rv, f"dv {b},{h}")
+
+
+# ---------------------------------------------------------------- full-size workloads
+def _group_bwd_check(dq, dk, dv, q, k, v, do, M, g, rep, scale, rows, where):
+    """Oracle gradients of kv head g (all `rep` query heads that read it) on the row range
+    `rows` of packed (T, H, D) tensors, compared with the library's."""
+    a, z = rows
+    rk = np.zeros((z - a, k.shape[-1]))
+    rv = np.zeros((z - a, v.shape[-1]))
+    for h in range(g * rep, (g + 1) * rep):
+        rq, k_, v_, _ = ob.masked_attention_bwd(q[a:z, h], k[a:z, g], v[a:z, g], M, do[a:z, h], scale)
+        _close(dq[a:z, h], rq, f"{where} dq head {h}")
+        rk += k_
+        rv += v_
+    _close(dk[a:z, g], rk, f"{where} dk kv head {g}")
+    _close(dv[a:z, g], rv, f"{where} dv kv head {g}")
+
+
+@pytest.mark.parametrize("window", [-1, 1024])
+def test_varlen_workload_sampled_sequences(window):
+    # the varlen workload (16 sequences of 512-4096 tokens, H=32 / Hkv=8, packed) in full on
+    # the GPU; the oracle differentiates the first, the longest and the last sequence for the
+    # first and the last kv-head group (the four query heads of a group sum into its dK / dV)
+    w = workloads.varlen_16()
+    cu = w["cu_seqlens"]
+    P = bfa.plan_blockids(cu_seqlens_q=_cuda(cu), cu_seqlens_k=_cuda(cu), max_q=w["max_len"],
+                          max_k=w["max_len"], window_left=window)
+    do = workloads.randn_bf16(tuple(w["q"].shape), 4343)
+    qc, kc, vc, dc = w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), do.cuda()
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    dq, dk, dv = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()
+    rep = w["H"] // w["Hkv"]
+    for s in sorted({0, int(np.argmax(w["lens"])), len(w["lens"]) - 1}):
+        a, z = int(cu[s]), int(cu[s + 1])
+        M = om.positional_dense(z - a, z - a, True, window)
+        for g in (0, w["Hkv"] - 1):
+            _group_bwd_check(dq, dk, dv, w["q"], w["k"], w["v"], do, M, g, rep, w["scale"], (a, z),
+                             f"varlen seq {s} window {window}")
+
+
+def test_bsr_workload_one_kv_group():
+    # the BSR workload (B=2, S=16384, H=32 / Hkv=8, causal inside the routed blocks) in full on
+    # the GPU; the oracle differentiates kv head 5 of batch 1 with its four query heads
+    w = workloads.bsr_16384()
+    P = bfa.plan_bsr(_cuda(w["block_indptr"]), _cuda(w["block_indices"]), w["S"], w["S"], causal=True)
+    do = workloads.randn_bf16(tuple(w["q"].shape), 4444)
+    qc, kc, vc, dc = w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), do.cuda()
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    dq, dk, dv = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    b, g = 1, 5
+    M = om.bsr_dense(w["block_indptr"][b:b + 1, g:g + 1], w["block_indices"], w["S"], w["S"], 128, 128,
+                     causal=True)[0, 0]
+    _group_bwd_check(dq[b].cpu(), dk[b].cpu(), dv[b].cpu(), w["q"][b], w["k"][b], w["v"][b], do[b], M, g,
+                     w["H"] // w["Hkv"], w["scale"], (0, w["S"]), "bsr")
