@@ -13,7 +13,7 @@ def _declared():
     return sorted(set(re.findall(r"\b(bfa_[a-z0-9_]+)\s*\(", src)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_plan_and_forward_calls():
     names = _declared()
     for n in ("bfa_plan_dense", "bfa_plan_blockids", "bfa_plan_bsr", "bfa_fwd"):
         assert n in names
