@@ -122,13 +122,28 @@ __device__ __forceinline__ void chunked_decode(int64_t w, int64_t units, int64_t
   j = static_cast<int>(hg * chunk + rem % gs);
 }
 
+// The base descriptors pass through an empty asm so that the compiler builds
+// them at the point of use (one add per step) instead of hoisting every step's
+// descriptor out of the tile loop into the MMA thread's registers.  A step's
+// descriptor is the base plus its byte offset / 16 (the start-address field).
+__device__ __forceinline__ uint64_t opaque_u64(uint64_t x) {
+  asm volatile("" : "+l"(x));
+  return x;
+}
+
+// MN-major operand of a TS product: 16-key steps 2048 bytes apart
+__device__ __forceinline__ uint64_t mn_desc(const uint8_t* s) {
+  return opaque_u64(smem_desc(smem_u32(s), 16384, 1024));
+}
+
 template <int D>
 __device__ __forceinline__ void issue_nn(uint32_t tD, const uint8_t* sA, const uint8_t* sB) {
+  const uint64_t da = opaque_u64(smem_desc(smem_u32(sA), 16, 1024));
+  const uint64_t db = opaque_u64(smem_desc(smem_u32(sB), 16, 1024));
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    umma_ss(tD, smem_desc(smem_u32(sA + off), 16, 1024), smem_desc(smem_u32(sB + off), 16, 1024), BCfg<D>::kIdescNN,
-            kk > 0);
+    const uint32_t off16 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+    umma_ss(tD, da + off16, db + off16, BCfg<D>::kIdescNN, kk > 0);
   }
 }
 
@@ -352,10 +367,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         if (!mbar_wait_fast(bar(BP + (u & 1)), (u >> 1) & 1, cap, &abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint64_t dk = mn_desc(sK(sk));
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tdQ, tdS + kk * 8, smem_desc(smem_u32(sK(sk) + kk * 2048), 16384, 1024), C::kIdescD,
-                  (u > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tdQ, tdS + kk * 8, dk + kk * (2048 >> 4), C::kIdescD, (u > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(KE + sk));
       }
       if (ok) umma_commit(bar(BO));
@@ -583,10 +598,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int cc = 0; cc < 4; ++cc) {
           if (!mbar_wait_fast(bar(BP1 + cc), s & 1, cap, &abort_flag)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t ddo = mn_desc(sdO(st));
 #pragma unroll
           for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk)
-            umma_ts(tdV, tS + kk * 8, smem_desc(smem_u32(sdO(st) + kk * 2048), 16384, 1024), C::kIdescD,
-                    (s > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tdV, tS + kk * 8, ddo + kk * (2048 >> 4), C::kIdescD, (s > 0 || kk > 0) ? 1u : 0u);
         }
         if (!ok) break;
         if (s + 1 < steps) {
@@ -598,10 +613,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dK += dS^T Q
         if (!mbar_wait_fast(bar(BP2), s & 1, cap, &abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint64_t dq = mn_desc(sQ(st));
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tdK, tdP + kk * 8, smem_desc(smem_u32(sQ(st) + kk * 2048), 16384, 1024), C::kIdescD,
-                  (s > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tdK, tdP + kk * 8, dq + kk * (2048 >> 4), C::kIdescD, (s > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(BE + st));
         if (s + 1 < steps) {
           issue_nn<D>(tdP, sV, sdO(st1));

@@ -236,22 +236,33 @@ __device__ __forceinline__ bool tile_skipped(const int (&votes)[2][4], int t) {
   return (v[0] & v[1] & v[2] & v[3]) != 0;
 }
 
+// The base descriptors pass through an empty asm so that the compiler builds
+// them at the point of use (one add per step) instead of hoisting every step's
+// descriptor out of the tile loop, where they would stay live in the MMA
+// thread's registers.  A step's descriptor is the base plus its byte offset / 16
+// (the start-address field; shared-memory offsets stay inside the field).
+__device__ __forceinline__ uint64_t opaque_u64(uint64_t x) {
+  asm volatile("" : "+l"(x));
+  return x;
+}
+
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t tS, uint8_t* sQ, uint8_t* sK) {
+  const uint64_t dq = opaque_u64(smem_desc(smem_u32(sQ), 16, 1024));
+  const uint64_t dk = opaque_u64(smem_desc(smem_u32(sK), 16, 1024));
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    umma_ss(tS, smem_desc(smem_u32(sQ + off), 16, 1024), smem_desc(smem_u32(sK + off), 16, 1024),
-            Cfg<D>::kIdescQK, kk > 0);
+    const uint32_t off16 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+    umma_ss(tS, dq + off16, dk + off16, Cfg<D>::kIdescQK, kk > 0);
   }
 }
 
 template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint8_t* sV, bool acc) {
+  const uint64_t dv = opaque_u64(smem_desc(smem_u32(sV), 16384, 1024));
 #pragma unroll
   for (int kk = 0; kk < kTile / 16; ++kk)
-    umma_ts(tO, tP + kk * 8, smem_desc(smem_u32(sV + kk * 2048), 16384, 1024), Cfg<D>::kIdescPV,
-            (acc || kk > 0) ? 1u : 0u);
+    umma_ts(tO, tP + kk * 8, dv + kk * (2048 >> 4), Cfg<D>::kIdescPV, (acc || kk > 0) ? 1u : 0u);
 }
 
 // kSkip: approximate mode (content-based block skipping); the exact kernel is
