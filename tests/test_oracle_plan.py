@@ -160,3 +160,78 @@ def test_transposed_plan_lists_the_same_tiles_as_the_rows(seed):
         r0 += nqt
     assert rows_pairs == cols_pairs
     assert np.array_equal(tp["order"], np.lexsort((np.arange(len(tp["counts"])), -tp["counts"])))
+
+
+def _brute_pairs(masks, BM=128, BN=128):
+    """Work pairs recomputed from the masks with plain loops: inside each group,
+    query tiles (2i, 2i + 1) form a pair, the last tile of an odd group stands
+    alone (stored as ~row); a pair costs the non-empty key tiles of its rows; the
+    order is longest first, ties by pair index (insertion sort, stable)."""
+    pair_row, cost = [], []
+    r0 = 0
+    for M in masks:
+        Sq, Sk = M.shape
+        nqt, nkt = -(-Sq // BM), -(-Sk // BN)
+        counts = []
+        for qt in range(nqt):
+            n = 0
+            for kt in range(nkt):
+                if M[qt * BM:(qt + 1) * BM, kt * BN:(kt + 1) * BN].any():
+                    n += 1
+            counts.append(n)
+        i = 0
+        while i < nqt:
+            if i + 1 < nqt:
+                pair_row.append(r0 + i)
+                cost.append(counts[i] + counts[i + 1])
+            else:
+                pair_row.append(-(r0 + i) - 1)
+                cost.append(counts[i])
+            i += 2
+        r0 += nqt
+    order = []
+    for p in range(len(cost)):
+        pos = len(order)
+        while pos > 0 and cost[order[pos - 1]] < cost[p]:
+            pos -= 1
+        order.insert(pos, p)
+    return pair_row, order
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_work_pairs_match_brute_force(seed):
+    rng = np.random.default_rng(300 + seed)
+    masks = [
+        rng.random((5 * 128 + 17, 700)) < 0.004,        # odd tile count with a ragged last tile
+        np.tril(np.ones((128, 128), dtype=bool)),       # a group of one tile
+        np.zeros((0, 256), dtype=bool),                 # an empty group (no query tiles)
+        np.zeros((300, 260), dtype=bool),               # rows with nothing listed
+        rng.random((4 * 128, 3 * 128 + 5)) < 0.5,       # even tile count
+        np.tril(np.ones((3 * 128 - 1, 3 * 128 - 1), dtype=bool)),
+    ]
+    masks[3][200, 5] = True                            # one attended pair in the middle row
+    P = op.plan_masks(masks)
+    pair_row, order = _brute_pairs(masks)
+    np.testing.assert_array_equal(P["pair_row"], np.array(pair_row, dtype=np.int32))
+    np.testing.assert_array_equal(P["pair_order"], np.array(order, dtype=np.int32))
+    # the pairs cover every row exactly once, in group order
+    rows = []
+    for pr in pair_row:
+        rows += [pr, pr + 1] if pr >= 0 else [~pr]
+    r0, want = 0, []
+    for M in masks:
+        nqt = -(-M.shape[0] // 128)
+        want += list(range(r0, r0 + nqt))
+        r0 += nqt
+    assert rows == want
+
+
+def test_work_pairs_of_the_causal_grid_closed_form():
+    """Causal 8192: pair i holds tiles 2i, 2i + 1 with 2i + 1 + 2i + 2 listed tiles,
+    so the longest-first order is the pairs in reverse."""
+    n = 64
+    M = np.tril(np.ones((n * 128, n * 128), dtype=bool))
+    P = op.plan_masks([M])
+    assert P["counts"].tolist() == list(range(1, n + 1))
+    assert P["pair_row"].tolist() == list(range(0, n, 2))
+    assert P["pair_order"].tolist() == list(range(n // 2 - 1, -1, -1))
