@@ -150,6 +150,58 @@ def _threads_used():
         return os.cpu_count()
 
 
+def _host_cores():
+    """The host's core count and torch's intra-op thread count, reported beside
+    the threads the oracle's BLAS actually used."""
+    import torch
+    return {"os_cpu_count": os.cpu_count(), "torch_threads": torch.get_num_threads()}
+
+
+def _median(xs):
+    xs = sorted(xs)
+    n = len(xs)
+    return xs[n // 2] if n % 2 else 0.5 * (xs[n // 2 - 1] + xs[n // 2])
+
+
+# Public datasheet dense bf16 tensor throughput of one B200 (context beside the
+# measured denominators).
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+def planner_leg(bfa, masks, dev, reps=10):
+    """bfa_plan_dense alone, L2 flushed before every timed call (a 256 MB write),
+    CUDA events around the call: median ms and GB/s on the algorithmic bytes
+    (mask read once + plan written: class grid, 2 KB of packed bits per partial
+    tile, 8 B per listed tile, 8 B per row)."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, mask in masks:
+        Sq, Sk = mask.shape
+        plan = bfa.plan_dense(mask)
+        n_full, n_part, n_empty = plan.stats()
+        plan.destroy()
+        nqt = -(-Sq // 128)
+        algo = Sq * Sk + (n_full + n_part + n_empty) + 2048 * n_part + 8 * (n_full + n_part) + 8 * nqt
+        times = []
+        for i in range(reps + 2):
+            flush.fill_(i & 255)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            plan = bfa.plan_dense(mask)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            plan.destroy()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1))
+        ms = _median(times)
+        out[name] = {"ms_median": ms, "algorithmic_bytes": algo, "gbs": algo / (ms * 1e-3) / 1e9,
+                     "tiles": {"full": n_full, "partial": n_part, "empty": n_empty}}
+    del flush
+    return out
+
+
 def cpu_oracle_sample(w, n_heads=4, rows=None):
     """Time the float64 oracle on a bounded sample: ``n_heads`` (b, h) pairs, all rows."""
     from oracle import attention as oa
@@ -181,15 +233,16 @@ def run_reference(args, rank, world):
         if i >= args.warmup:
             times.append(dt)
             vals.append(v)
-    value = sum(vals) / len(vals)
+    value = _median(vals)
     cores = _threads_used()
     sample = f"{per_step_heads} of 128 (batch, head) pairs per step, all 8192 rows, float64 NumPy oracle"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * _median(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(WORKLOAD, parallelism=f"dp{args.gpus}"),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample,
+                         **_host_cores()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -251,8 +304,9 @@ def run_bfa(args, rank, world, local_rank):
         dist.barrier()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
-    fwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    plan_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    # per-step forward and plan times: the median of the K event pairs
+    fwd_ms = _median([e[1].elapsed_time(e[2]) for e in evs])
+    plan_ms = _median([e[0].elapsed_time(e[1]) for e in evs])
     ms, fwd_ms, plan_ms = max_over_ranks([ms, fwd_ms, plan_ms], dist, dev)
     ms_per_step = ms / args.steps
     value = whole_job_tflops(flops, world, ms_per_step)
@@ -335,6 +389,14 @@ def run_bfa(args, rank, world, local_rank):
     plan.destroy()
     bwd_ms = max_over_ranks([b0.elapsed_time(b1) / bwd_steps], dist, dev)[0]
 
+    # the planner on its own (L2 flushed before each call), on the bench's 67 MB
+    # causal mask and the 268 MB union mask of the 16384 workload
+    plan_masks = [("causal_8192", mask)]
+    if rank == 0 and not args.no_union_planner:
+        plan_masks.append(("union_16384", workloads.union_16384(with_qkv=False)["mask"].to(dev)))
+    planner = planner_leg(bfa, plan_masks, dev)
+    del plan_masks
+
     peaks, src = _peaks()
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     # bytes the forward must move at least: read q, k, v once, write out and lse
@@ -351,9 +413,15 @@ def run_bfa(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "bfa_fwd_kernel<128>", "achieved": fwd_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": fwd_tflops / peak, "peak_source": f"{src} bf16_tflops (burst)",
                      "frac_of_sustained": fwd_tflops / peaks.get("bf16_tflops_sustained", peak),
+                     "frac_of_datasheet": fwd_tflops / DATASHEET_BF16_TFLOPS,
+                     "timing": f"median of {args.steps} per-step CUDA-event pairs around the forward",
                      "traffic": _fwd_traffic(), "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "algorithmic_bytes": algo_bytes},
         "fwd_ms": fwd_ms, "plan_ms": plan_ms,
+        "planner": {"call": "bfa_plan_dense (k_init_regular_groups, k_dense_classify, k_rows)", "bound": "hbm",
+                    "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{src} hbm_gbs",
+                    "l2": "256 MB written before every timed call", **{
+                        k: dict(v, frac=v["gbs"] / peaks["hbm_gbs"]) for k, v in planner.items()}},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
                 "overlap": "copies in, plan + forward and copies out on three streams over two device buffer sets"},
@@ -367,7 +435,8 @@ def run_bfa(args, rank, world, local_rank):
     if rank == 0 and not args.no_cpu_baseline:
         v_cpu, dt, n = cpu_oracle_sample(w, n_heads=16)  # about 10 s of float64 work
         line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": _threads_used(), "kind": "oracle",
-                                "sample": f"{n} of 128 (batch, head) pairs, all 8192 rows, {dt:.1f} s float64"}
+                                "sample": f"{n} of 128 (batch, head) pairs, all 8192 rows, {dt:.1f} s float64",
+                                **_host_cores()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -465,6 +534,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["bfa", "reference"], default="bfa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-union-planner", action="store_true", help="skip the planner leg on the 268 MB union mask")
     ap.add_argument("--sweep", action="store_true", help="forward/backward on every workload (information)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -345,8 +345,17 @@ bfa_status bfa_plan_device_status(const bfa_plan* plan, void* stream);
  * streams that reads the plan must be ordered before this call.  NULL is a no-op. */
 void bfa_plan_destroy(bfa_plan* plan);
 
-/* Bound, in nanoseconds, on every device-side wait of the kernels launched after
- * this call (default 1e9, i.e. one second).  0 restores the default. */
+/* Bound, in nanoseconds, on the device-side waits inside the kernels' loops
+ * (a TMA copy, a product or another role of the block that does not arrive),
+ * for kernels launched after this call: default 1e9, i.e. one second; 0 restores
+ * the default; other values are clamped to [BFA_WAIT_NS_MIN, BFA_WAIT_NS_MAX].
+ * Past the bound the block stops its work, and the plan's device status reports
+ * BFA_ERR_TIMEOUT (bfa_plan_device_status).  The waits that keep a block alive
+ * until the copies and products it has already issued are complete (before it
+ * releases tensor memory and exits) do not follow this bound: they have a fixed
+ * bound of 4 s, and those phases complete by themselves within microseconds. */
+#define BFA_WAIT_NS_MIN 1000ull
+#define BFA_WAIT_NS_MAX 60000000000ull
 void bfa_set_wait_timeout_ns(uint64_t ns);
 
 /* Launch a one-thread-block kernel that waits, with the current bound, on a
@@ -354,14 +363,6 @@ void bfa_set_wait_timeout_ns(uint64_t ns);
  * BFA_ERR_TIMEOUT when the bounded wait gives up as designed (and the context
  * stays usable), BFA_OK never.  Exercises the failure path without a fault. */
 bfa_status bfa_selftest_wait_timeout(void* stream);
-
-/* Evaluate, on the device, the FMA-pipe 2^x that the forward's softmax uses for
- * part of its exponentials (range reduction to n + f, f in [-1/2, 1/2], and a
- * degree-3 polynomial for 2^f): y[i] = 2^x[i] for i < n.  x and y are device
- * pointers to n floats (n >= 0), owned by the caller; arguments at or below
- * -127 give +0.  Returns BFA_ERR_INVALID_ARG for NULL pointers with n > 0 or
- * n < 0, BFA_ERR_CUDA for a launch error.  Enqueued on `stream`; no sync. */
-bfa_status bfa_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /*
  * Dense-mask planner that allocates nothing.  The source pages have no
@@ -385,7 +386,11 @@ bfa_status bfa_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
  * so make that first call before any stream capture.  All calls share the one
  * array: calls that overlap on the GPU (on different streams) race and must be
  * ordered by the caller.  Each call writes every scratch word it reads, so the
- * previous call's contents do not matter.  Stream-ordered, no synchronisation.
+ * previous call's contents do not matter.  After a device reset
+ * (cudaDeviceReset) the array may move: call bfa_is_available() once on that
+ * device before this entry point's next call there, which then looks the
+ * address up again (so it, too, must come before any stream capture).
+ * Stream-ordered, no synchronisation.
  */
 enum { BFA_NOALLOC_MAX_ROWS = 4096, BFA_NOALLOC_MAX_KV_TILES = 16384 };
 bfa_status bfa_plan_dense_noalloc(const uint8_t* mask, int64_t mask_row_stride, int Sq, int Sk,

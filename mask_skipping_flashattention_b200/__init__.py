@@ -26,7 +26,7 @@ from ._lib import BfaError, PlanInfo
 __all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_predicate", "plan_bsr", "plan_block_bits",
            "fwd", "bwd", "fwd_paged",
            "make_att_block_ids",
-           "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "selftest_exp2", "library_path"]
+           "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "library_path"]
 
 TILE = 128
 KIND_NAMES = {1: "dense", 2: "blockids", 3: "positional", 4: "bsr", 5: "predicate"}
@@ -74,19 +74,6 @@ def set_wait_timeout_ns(ns):
 def selftest_wait_timeout(stream=None):
     """Run the library's bounded-wait self test; returns the status name."""
     return _lib.STATUS.get(_L.bfa_selftest_wait_timeout(_stream(stream)))
-
-
-def selftest_exp2(x, stream=None):
-    """2^x by the forward's FMA-pipe exponential (range reduction + polynomial), on the device.
-
-    ``x``: a float32 CUDA tensor; returns a tensor of the same shape."""
-    import torch
-    if x.dtype != torch.float32 or not x.is_cuda:
-        raise ValueError("x must be a float32 CUDA tensor")
-    x = x.contiguous()
-    y = torch.empty_like(x)
-    _lib.check(_L.bfa_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
-    return y
 
 
 class Plan:

@@ -63,7 +63,6 @@ SIGNATURES = {
     "bfa_plan_destroy": (None, [c_void]),
     "bfa_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
     "bfa_selftest_wait_timeout": (ctypes.c_int, [c_void]),
-    "bfa_selftest_exp2": (ctypes.c_int, [c_void, c_void, ctypes.c_int64, c_void]),
     "bfa_plan_dense_noalloc": (ctypes.c_int, [c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int, c_void, c_void,
                                               c_void, c_void, c_void, c_void, c_void]),
 }

@@ -120,6 +120,11 @@ namespace {
 thread_local std::string g_err;
 uint64_t g_wait_ns = 1000000000ull;
 
+// Device address of the allocation-free planner's scratch array, per device
+// (looked up on that entry point's first call on a device; see below).
+std::mutex g_noalloc_mu;
+uint8_t* g_noalloc_ptr[64] = {};
+
 bfa_status fail(bfa_status s, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -427,10 +432,20 @@ BFA_API int bfa_is_available(void) {
     fail(BFA_ERR_CUDA, "kernel image does not load: %s", cudaGetErrorString(e));
     return 0;
   }
+  // A device reset reloads the library's device code, and the scratch array of
+  // the allocation-free planner may then sit at another address: forget the one
+  // looked up before, so that planner's next call on this device looks it up again.
+  if (dev >= 0 && dev < 64) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    g_noalloc_ptr[dev] = nullptr;
+  }
   return 1;
 }
 
-BFA_API void bfa_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : 1000000000ull; }
+BFA_API void bfa_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) ns = 1000000000ull;
+  g_wait_ns = std::min<uint64_t>(std::max<uint64_t>(ns, BFA_WAIT_NS_MIN), BFA_WAIT_NS_MAX);
+}
 
 BFA_API bfa_status bfa_make_block_ids(const uint8_t* pad_masks, const uint8_t* att_masks, int B, int N, int n_cross,
                                       const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
@@ -1358,14 +1373,6 @@ BFA_API bfa_status bfa_selftest_wait_timeout(void* stream) {
   return BFA_OK;
 }
 
-BFA_API bfa_status bfa_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
-  if (n < 0) return fail(BFA_ERR_INVALID_ARG, "n = %lld < 0", static_cast<long long>(n));
-  if (n > 0 && (!x || !y)) return fail(BFA_ERR_INVALID_ARG, "x or y is NULL");
-  auto cleanup = []() {};
-  BFA_CUDA(launch_exp2_selftest(x, y, n, static_cast<cudaStream_t>(stream)), "exp2 selftest kernel");
-  return BFA_OK;
-}
-
 // ----------------------------------------------------------------------------
 // Dense planner that allocates nothing
 // ----------------------------------------------------------------------------
@@ -1383,9 +1390,6 @@ constexpr size_t kNoAllocScratchBytes = 256 + 2 * sizeof(int32_t) * kNoAllocMaxR
 static_assert(sizeof(GroupInfo) <= 256, "group table slot");
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-
-std::mutex g_noalloc_mu;
-uint8_t* g_noalloc_ptr[64] = {};
 
 // Device address of the scratch array on the current device (set up once per
 // device, with that device current).  In host code the array's name is only a

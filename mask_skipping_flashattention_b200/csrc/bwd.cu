@@ -328,10 +328,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         last[st] = u;
       }
-      volatile int no_abort = 0;
-      mbar_wait_fast(bar(BQ), 0, cap, &no_abort);
+      mbar_drain(bar(BQ), 0, &abort_flag);
       for (int st = 0; st < kBwdStages; ++st)
-        if (last[st] >= 0) mbar_wait_fast(bar(BF + st), (last[st] >> 1) & 1, cap, &no_abort);
+        if (last[st] >= 0) mbar_drain(bar(BF + st), (last[st] >> 1) & 1, &abort_flag);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -375,8 +374,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       }
       if (ok) umma_commit(bar(BO));
       umma_commit(bar(BDONE));
-      volatile int no_abort = 0;
-      mbar_wait_fast(bar(BDONE), 0, cap, &no_abort);
+      mbar_drain(bar(BDONE), 0, &abort_flag);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dS rows
@@ -571,10 +569,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bulk_load(smem_u32(sVec(st) + kTile), p.ws_d + wi, kTile * 4, f);
         last[st] = s;
       }
-      volatile int no_abort = 0;
-      mbar_wait_fast(bar(BKV), 0, cap, &no_abort);
+      mbar_drain(bar(BKV), 0, &abort_flag);
       for (int st = 0; st < kBwdStages; ++st)
-        if (last[st] >= 0) mbar_wait_fast(bar(BF + st), (last[st] >> 1) & 1, cap, &no_abort);
+        if (last[st] >= 0) mbar_drain(bar(BF + st), (last[st] >> 1) & 1, &abort_flag);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -625,8 +622,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (ok) umma_commit(bar(BO));
       umma_commit(bar(BDONE));
-      volatile int no_abort = 0;
-      mbar_wait_fast(bar(BDONE), 0, cap, &no_abort);
+      mbar_drain(bar(BDONE), 0, &abort_flag);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P^T, dS^T rows (one key per thread)

@@ -52,13 +52,6 @@ constexpr uint32_t kRegsSoftmax = 216;
 static_assert(128 * kRegsWG0 + 256 * kRegsSoftmax == kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows by > 2^8
 constexpr int kStages = 2;
-// Of every 8 column pairs of a row, this many take 2^x on the FMA pipe
-// (ex2_poly) and the rest on the MUFU (ex2.approx): the exponentials are the
-// softmax's longest phase, and the two pipes run side by side.
-#ifndef BFA_POLY_PAIRS
-#define BFA_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = BFA_POLY_PAIRS;
 
 template <int D>
 struct Cfg {
@@ -357,12 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!have_next) break;
           kt = kt_n;
         }
-        // every copy this CTA issued must land before it can exit (bounded; on the
-        // normal path these phases completed long ago)
-        volatile int no_abort = 0;
-        mbar_wait_fast(bar(BQ), 0, cap, &no_abort);
+        // every copy this CTA issued must land before it can exit (on the normal
+        // path these phases completed long ago; the drain bound is fixed)
+        mbar_drain(bar(BQ), 0, &abort_flag);
         for (int b = 0; b < 2; ++b)
-          if (last_f[b] >= 0) mbar_wait_fast(bar(BF + b), (last_f[b] >> 1) & 1, cap, &no_abort);
+          if (last_f[b] >= 0) mbar_drain(bar(BF + b), (last_f[b] >> 1) & 1, &abort_flag);
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
@@ -430,8 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) umma_commit(bar(BO));
         // every MMA issued must be finished before TMEM is released (bounded)
         umma_commit(bar(BDONE));
-        volatile int no_abort = 0;
-        mbar_wait_fast(bar(BDONE), 0, cap, &no_abort);
+        mbar_drain(bar(BDONE), 0, &abort_flag);
       }
     }
   } else {
@@ -464,7 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (masked) row_mask_words(p.plan, wk, qpos, row, kt, part, am);
 
         const bool got = mbar_wait(barS, t & 1, cap, &abort_flag);
-        if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit
+        if constexpr (kSkip) {
+          // the vote below is a barrier of the slot's four warps, so they leave
+          // the loop together (slot-uniform exit)
+          if (named_bar_red_or(1 + slot, 128, !got)) { ok = false; break; }
+        } else {
+          if (__any_sync(0xffffffffu, !got)) { ok = false; break; }  // warp-uniform exit
+        }
         tc_fence_after();
         // the whole S row in registers: four loads in flight, one wait
         uint32_t sr[128];
@@ -538,15 +535,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, nm2);
-            float p0, p1;
-            if ((j & 7) < kPolyPairs) {  // this pair on the FMA pipe
-              f2_unpack(ex2_poly2(x2), p0, p1);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             rs2[j & 3] = f2_add(rs2[j & 3], f2_pack(p0, p1));
             pk[j] = pack_bf16x2(p0, p1);
           }
@@ -677,22 +668,6 @@ __global__ void k_wait_selftest(uint32_t* err, uint64_t cap) {
 }
 
 // ----------------------------------------------------------------------------
-// FMA-pipe exp2 self test: y[i] = 2^x[i], pairs through ex2_poly2 (the form the
-// softmax uses), a lone last element through ex2_poly
-// ----------------------------------------------------------------------------
-__global__ void k_exp2_selftest(const float* x, float* y, int64_t n) {
-  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    float a, b;
-    f2_unpack(ex2_poly2(f2_pack(x[i], x[i + 1])), a, b);
-    y[i] = a;
-    y[i + 1] = b;
-  } else if (i < n) {
-    y[i] = ex2_poly(x[i]);
-  }
-}
-
-// ----------------------------------------------------------------------------
 // launchers (host)
 // ----------------------------------------------------------------------------
 int fwd_smem_bytes(int D) { return D == 64 ? Cfg<64>::kSmemBytes : Cfg<128>::kSmemBytes; }
@@ -725,12 +700,6 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
   if (D == 64)
     return approx ? launch_one<64, true>(tq, tk, tv, to, p, n_work, s) : launch_one<64, false>(tq, tk, tv, to, p, n_work, s);
   return approx ? launch_one<128, true>(tq, tk, tv, to, p, n_work, s) : launch_one<128, false>(tq, tk, tv, to, p, n_work, s);
-}
-
-cudaError_t launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t s) {
-  if (n <= 0) return cudaSuccess;
-  k_exp2_selftest<<<static_cast<unsigned>((n + 511) / 512), 256, 0, s>>>(x, y, n);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s) {

@@ -38,7 +38,6 @@ int fwd_smem_bytes(int D);
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int64_t n_work, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s);
-cudaError_t launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t s);
 cudaError_t probe_fwd_kernels();
 
 }  // namespace bfa

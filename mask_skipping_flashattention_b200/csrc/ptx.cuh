@@ -93,6 +93,20 @@ __device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, ui
   return mbar_wait_slow(bar, parity, cap_ns, abort);
 }
 
+// Bound of the waits that keep a block alive until the copies and products it has
+// issued itself are complete (before it releases tensor memory or exits).  These
+// phases complete by themselves within microseconds; the bound is fixed and does
+// not follow the caller's bound on the loop waits, so a short caller bound can
+// never let a block exit with its own asynchronous writes still in flight.
+constexpr uint64_t kDrainWaitNs = 4000000000ull;
+
+// Drain wait: ignores the block's abort flag; if even this bound runs out, the
+// block's abort flag is set so that the launch reports a timeout.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, volatile int* abort) {
+  volatile int never = 0;
+  if (!mbar_wait_fast(bar, parity, kDrainWaitNs, &never)) *abort = 1;
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -368,40 +382,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x on the FMA pipe, for x <= 2^20 (the softmax only passes x <= 8).  Range
-// reduction: x = n + f with n = round(x) and f in [-1/2, 1/2]; adding 1.5 * 2^23
-// leaves n in the low mantissa bits of t, so (bits(t) << 23) is n in the exponent
-// field.  2^f is the degree-3 polynomial 1 + f (c1 + f (c2 + f c3)) fitted for
-// the least maximum relative error on [-1/2, 1/2] with p(0) = 1
-// (fit_exp2_poly.py: 1.0e-4, below the bf16 rounding of P).  Arguments are
-// clamped at -127, where p(0) = 1 makes the result exactly +0 (masked scores).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -127.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float q = fmaf(f, 5.500858277e-02f, 2.422103733e-01f);
-  q = fmaf(q, f, 6.932829022e-01f);
-  q = fmaf(q, f, 1.0f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-// ex2_poly on a pair of fp32 lanes, with the packed fp32x2 add and fma for the
-// rounding, the reduced argument and the polynomial (bit-identical to two
-// ex2_poly calls: the same operations lane by lane).
-__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  const uint64_t x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));
-  const uint64_t f = f2_add(x, f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(12582912.f, 12582912.f)));  // x - (t - 1.5 2^23)
-  uint64_t q = f2_fma(f, f2_pack(5.500858277e-02f, 5.500858277e-02f), f2_pack(2.422103733e-01f, 2.422103733e-01f));
-  q = f2_fma(q, f, f2_pack(6.932829022e-01f, 6.932829022e-01f));
-  q = f2_fma(q, f, f2_pack(1.0f, 1.0f));
-  float t0, t1, q0, q1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(q, q0, q1);
-  return f2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
-                 __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
-}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

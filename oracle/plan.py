@@ -88,9 +88,16 @@ def lpt_order(counts):
 
 def plan_masks(masks, BM=128, BN=128):
     """Plan of a sequence of group masks (each (Sq_g, Sk_g) bool), groups in order."""
+    return combine_groups([plan_group(M, BM, BN) for M in masks], BM, BN)
+
+
+def combine_groups(group_plans, BM=128, BN=128):
+    """The plan of several groups from each group's own plan (``plan_group``), in
+    group order: the groups' rows concatenated, then the row order and the work
+    pairs over all rows.  Lets a caller build a large plan one group's mask at a
+    time."""
     cls_all, lists, parts, fines = [], [], [], []
-    for M in masks:
-        cls, rl, rp, fn = plan_group(M, BM, BN)
+    for cls, rl, rp, fn in group_plans:
         cls_all.append(cls)
         lists += rl
         parts += rp

@@ -31,6 +31,7 @@ def test_reference_arm_prints_one_contract_line_on_rank0():
     assert d["config"]["workload"] == "causal_8192"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert cb["os_cpu_count"] >= 1 and cb["torch_threads"] >= 1
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

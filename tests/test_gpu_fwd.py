@@ -300,6 +300,40 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     test_default_scale_matches_explicit()
 
 
+def test_forward_and_backward_give_up_on_a_short_wait_bound():
+    """The kernels' own failure path: with the shortest loop-wait bound (1 us) the
+    first wait of a block for its scores outlasts the bound (the copies of Q and K
+    alone take longer), so blocks stop their work, drain the copies and products
+    they issued, release tensor memory and report BFA_ERR_TIMEOUT through the plan.
+    Afterwards the default bound gives oracle-exact results on the same plan."""
+    B, H, N, D = 2, 8, 2048, 128
+    M = np.tril(np.ones((N, N), dtype=bool))
+    q, k, v = (_rand((B, N, H, D), 9100 + i) for i in range(3))
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    P = bfa.plan_dense(_cuda(M))
+    bfa.set_wait_timeout_ns(1)  # clamped to the minimum, 1 us
+    try:
+        out, lse = bfa.fwd(P, qc, kc, vc)
+        torch.cuda.synchronize()
+        with pytest.raises(bfa.BfaError) as e:
+            P.device_status()
+        assert e.value.status == "BFA_ERR_TIMEOUT"
+        dout = _rand((B, N, H, D), 9199).cuda()
+        bfa.bwd(P, qc, kc, vc, out, dout, lse)
+        torch.cuda.synchronize()
+        with pytest.raises(bfa.BfaError) as e:
+            P.device_status()
+        assert e.value.status == "BFA_ERR_TIMEOUT"
+    finally:
+        bfa.set_wait_timeout_ns(0)
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    torch.cuda.synchronize()
+    P.device_status()
+    rows = sample_rows(N, 48, 5, must=(0, N - 1))
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M, None, [(0, 0), (1, H - 1)], rows=rows,
+               where="after the timeout")
+
+
 @pytest.mark.parametrize("qb,kb,causal", [(64, 32, True), (100, 192, False)])
 def test_general_block_sparse_forward(qb, kb, causal):
     from test_gpu_plan import _routing, _valid_bits

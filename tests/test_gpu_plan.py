@@ -187,26 +187,28 @@ def test_bsr_plan_small(causal):
     assert_plan_equal(P.export(), oracle_plan_for_groups(_bsr_oracle(indptr, indices, S, causal)))
 
 
-def test_bsr_plan_workload_one_head_group_full_size():
+def test_bsr_plan_workload_full_size_every_group():
+    """The BSR 16384 workload's plan, bit for bit on all 16 (batch, kv head) groups:
+    the oracle plan is built one group's 16384 x 16384 mask at a time and the groups
+    are combined (rows concatenated, then the row order and the work pairs over all
+    rows).  The same routing in the exact-block bitmask form gives the same plan
+    (with its packed fine words)."""
+    from oracle import plan as op
     w = workloads.bsr_16384(with_qkv=False)
-    P = bfa.plan_bsr(_cuda(w["block_indptr"]), _cuda(w["block_indices"]), w["S"], w["S"], causal=True)
+    ip, ix, S = w["block_indptr"], w["block_indices"], w["S"]
+    B, Hkv, _ = ip.shape
+    P = bfa.plan_bsr(_cuda(ip), _cuda(ix), S, S, causal=True)
     n_full, n_part, n_empty = P.stats()
-    assert n_part == 2 * 8 * 128 and n_full == 2 * 8 * 1984
-    got = P.export()
-    # full bit-exact check on the first two (b, hkv) groups; lists of all groups by counts
-    ip, ix = w["block_indptr"][:1, :2], w["block_indices"]
-    ref = oracle_plan_for_groups(_bsr_oracle(ip, ix, w["S"], True))
-    R = 2 * 128
-    np.testing.assert_array_equal(got["row_ptr"][:R + 1], ref["row_ptr"])
-    np.testing.assert_array_equal(got["kv_tile"][:ref["kv_tile"].size], ref["kv_tile"])
-    np.testing.assert_array_equal(got["partial"][:ref["partial"].size], ref["partial"])
-    counts = np.diff(got["row_ptr"])
-    exp = np.array([i // 4 + 1 for _ in range(16) for i in range(128)])
-    np.testing.assert_array_equal(counts, exp)
-    order = got["order"]
-    assert np.all(np.diff(counts[order]) <= 0)
-    ties = np.diff(counts[order]) == 0
-    assert np.all(np.diff(order)[ties] > 0)
+    assert n_part == B * Hkv * 128 and n_full == B * Hkv * 1984
+    groups = []
+    for b in range(B):
+        for h in range(Hkv):
+            groups.append(op.plan_group(_bsr_oracle(ip[b:b + 1, h:h + 1], ix, S, True)[0]))
+    ref = op.combine_groups(groups)
+    assert_plan_equal(P.export(), ref)
+    bits = om.bsr_to_block_bits(ip, ix, -(-S // 128))
+    P2 = bfa.plan_block_bits(_cuda(bits.view(np.int32)), S, S, causal=True)
+    assert_plan_equal(P2.export(), ref)
 
 
 def test_bsr_noncanonical_rejected():
