@@ -104,9 +104,6 @@ typedef struct bfa_plan_info {
   int32_t packed_fine;    /* 1: partial tiles carry packed fine masks (bfa_plan_export fills fine) */
   int32_t n_cols;         /* key-tile columns (sum over groups of their key tiles): the backward's
                              dK/dV work units, see bfa_plan_export_cols                         */
-  int32_t n_quads;        /* work quads: query tiles (4i .. 4i+3) of one group, the work unit of
-                             the forward on a pair of SMs; 0 when the plan has none (rows of
-                             more than 12288 key tiles)                                          */
 } bfa_plan_info;
 
 /* Library version string. */
@@ -339,13 +336,6 @@ bfa_status bfa_plan_export_pairs(const bfa_plan* plan, int32_t* pair_row, int32_
  * NULL. */
 bfa_status bfa_plan_export_cols(const bfa_plan* plan, int32_t* col_ptr, int32_t* q_tile, int32_t* tpart,
                                 int32_t* col_order, void* stream);
-
-/* Copy the plan's work quads to HOST buffers (parity checks); synchronises
- * `stream`.  Inside each group, query tiles (4i .. 4i+3) form one quad (fewer at
- * the group's end); quad_row [n_quads] holds each quad's first row, groups in
- * order; quad_order [n_quads] lists the quads longest first by their rows' total
- * listed tiles, ties by quad index.  Either pointer may be NULL. */
-bfa_status bfa_plan_export_quads(const bfa_plan* plan, int32_t* quad_row, int32_t* quad_order, void* stream);
 
 /* Synchronise `stream` and report BFA_ERR_TIMEOUT if a kernel that used the plan
  * hit its wait bound since the last call (the flag is then cleared). */

@@ -130,7 +130,7 @@ class Plan:
         return dict(col_ptr=col_ptr, q_tile=q_tile[:nnz], tpart=tpart[:nnz], col_order=col_order[:C])
 
     def export(self, stream=None):
-        """Host copy: row_ptr, kv_tile, partial, fine (packed-mask plans), order, classes, pairs, quads."""
+        """Host copy: row_ptr, kv_tile, partial, fine (packed-mask plans), order, classes, pairs."""
         n_full, n_part, _ = self.stats(stream)
         R = self.info["n_rows"]
         nnz = n_full + n_part
@@ -151,13 +151,6 @@ class Plan:
         _lib.check(_L.bfa_plan_export_pairs(self.handle, P(pair_row), P(pair_order), _stream(stream)))
         out["pair_row"] = pair_row[:n_pairs]
         out["pair_order"] = pair_order[:n_pairs]
-        n_quads = self.info["n_quads"]
-        if n_quads > 0 or R == 0:  # plans with rows of more than 12288 key tiles list no quads
-            quad_row = np.zeros(max(n_quads, 1), np.int32)
-            quad_order = np.zeros(max(n_quads, 1), np.int32)
-            _lib.check(_L.bfa_plan_export_quads(self.handle, P(quad_row), P(quad_order), _stream(stream)))
-            out["quad_row"] = quad_row[:n_quads]
-            out["quad_order"] = quad_order[:n_quads]
         if fine is not None:
             out["fine"] = fine[:n_part]
         return out

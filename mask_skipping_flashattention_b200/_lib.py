@@ -59,7 +59,6 @@ SIGNATURES = {
     "bfa_plan_export": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_void]),
     "bfa_plan_export_pairs": (ctypes.c_int, [c_void, c_void, c_void, c_void]),
     "bfa_plan_export_cols": (ctypes.c_int, [c_void, c_void, c_void, c_void, c_void, c_void]),
-    "bfa_plan_export_quads": (ctypes.c_int, [c_void, c_void, c_void, c_void]),
     "bfa_plan_device_status": (ctypes.c_int, [c_void, c_void]),
     "bfa_plan_destroy": (None, [c_void]),
     "bfa_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
@@ -74,8 +73,7 @@ class PlanInfo(ctypes.Structure):
                 ("n_rows", ctypes.c_int32), ("grid_tiles", ctypes.c_int64), ("batch", ctypes.c_int32),
                 ("hkv", ctypes.c_int32), ("sq", ctypes.c_int32), ("sk", ctypes.c_int32),
                 ("max_kv_tiles", ctypes.c_int32), ("window_left", ctypes.c_int32), ("causal", ctypes.c_int32),
-                ("n_pairs", ctypes.c_int32), ("packed_fine", ctypes.c_int32), ("n_cols", ctypes.c_int32),
-                ("n_quads", ctypes.c_int32)]
+                ("n_pairs", ctypes.c_int32), ("packed_fine", ctypes.c_int32), ("n_cols", ctypes.c_int32)]
 
 
 class MaskTerm(ctypes.Structure):

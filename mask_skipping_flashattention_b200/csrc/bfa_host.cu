@@ -36,8 +36,7 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row = nullptr, int32_t* pair_cost = nullptr,
                         int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr, int part_is_pos = 0,
-                        int2* row_work = nullptr, int2* pair_work = nullptr, int32_t* quad_row = nullptr,
-                        int32_t* quad_cost = nullptr, int32_t* quad_order = nullptr, int2* quad_work = nullptr);
+                        int2* row_work = nullptr, int2* pair_work = nullptr);
 cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int n_groups,
                                int nqb, int nkb, int wpr, uint32_t* bits, uint32_t* err, cudaStream_t s);
 cudaError_t launch_cols(const GroupInfo* groups, int n_groups, const uint8_t* cls, const int32_t* row_ptr,
@@ -70,7 +69,7 @@ using namespace bfa;
 // ----------------------------------------------------------------------------
 struct bfa_plan {
   int kind = 0, varlen = 0, batch = 0, hkv = 0, sq = 0, sk = 0, window = -1, causal = 0;
-  int n_groups = 0, n_rows = 0, n_pairs = 0, n_quads = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
+  int n_groups = 0, n_rows = 0, n_pairs = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
   int64_t grid_tiles = 0;
   int64_t fine_tiles = 0;       // tiles of packed fine words held in `fine`
   void* fine_extra = nullptr;   // separately allocated fine words (generic block sparsity)
@@ -96,10 +95,6 @@ struct bfa_plan {
   int32_t* pair_idx = nullptr;    // scratch: pair index of each row
   int2* row_work = nullptr;       // rows in longest-first order with their group
   int2* pair_work = nullptr;      // pairs in longest-first order with the group of their first row
-  int32_t* quad_row = nullptr;    // first row of each work quad (up to 4 consecutive rows of a group)
-  int32_t* quad_cost = nullptr;   // listed tiles of the quad
-  int32_t* quad_order = nullptr;  // longest-first order of the quads
-  int2* quad_work = nullptr;      // quads in longest-first order with their group
   int32_t* qid = nullptr;
   uint8_t* qvalid = nullptr;
   int32_t* kid = nullptr;
@@ -198,7 +193,6 @@ cudaError_t plan_pool(cudaMemPool_t* out) {
 }
 
 constexpr int kMaxKvTiles = 16384;  // key tiles per row: the row kernel's shared-memory buckets
-constexpr int kMaxQuadKvTiles = 12288;  // key tiles per row for which the plan also lists quads
 
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -232,10 +226,6 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   const size_t o_pidx = L.take<int32_t>(std::max(P->n_rows, 1));
   const size_t o_rwork = L.take<int2>(std::max(P->n_rows, 1));
   const size_t o_pwork = L.take<int2>(std::max(P->n_rows, 1));
-  const size_t o_qrow = L.take<int32_t>(std::max(P->n_rows, 1));
-  const size_t o_qcost = L.take<int32_t>(std::max(P->n_rows, 1));
-  const size_t o_qord = L.take<int32_t>(std::max(P->n_rows, 1));
-  const size_t o_qwork = L.take<int2>(std::max(P->n_rows, 1));
   const size_t o_err = L.take<uint32_t>(1);
   const size_t o_mw = L.take<int32_t>(1);
   const size_t o_qid = L.take<int32_t>(std::max<int64_t>(qid_elems, 1));
@@ -265,10 +255,6 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->pair_idx = reinterpret_cast<int32_t*>(base + o_pidx);
   P->row_work = reinterpret_cast<int2*>(base + o_rwork);
   P->pair_work = reinterpret_cast<int2*>(base + o_pwork);
-  P->quad_row = reinterpret_cast<int32_t*>(base + o_qrow);
-  P->quad_cost = reinterpret_cast<int32_t*>(base + o_qcost);
-  P->quad_order = reinterpret_cast<int32_t*>(base + o_qord);
-  P->quad_work = reinterpret_cast<int2*>(base + o_qwork);
   P->err = reinterpret_cast<uint32_t*>(base + o_err);
   P->max_width = reinterpret_cast<int32_t*>(base + o_mw);
   P->qid = reinterpret_cast<int32_t*>(base + o_qid);
@@ -321,15 +307,9 @@ bfa_status build_rows(bfa_plan* P, int part_is_pos = 0) {
     return e == cudaSuccess ? BFA_OK : cuda_fail(e, "empty plan");
   }
   if (P->max_nkt > kMaxKvTiles) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
-  // Quads (the SM-pair forward's work units) are ordered by a counting sort over
-  // keys up to 4 max_nkt in shared memory; past kMaxQuadKvTiles the plan has none
-  // and the forward runs one SM per work item.
-  const bool quads = P->max_nkt <= kMaxQuadKvTiles;
-  if (!quads) P->n_quads = 0;
   cudaError_t e = launch_rows(P->groups, P->row_group, P->cls, P->n_rows, P->max_nkt, P->row_cnt, P->row_ptr,
                               P->kv_tile, P->part, P->order, P->stream, P->pair_row, P->pair_cost,
-                              P->pair_order, P->pair_idx, part_is_pos, P->row_work, P->pair_work,
-                              quads ? P->quad_row : nullptr, P->quad_cost, P->quad_order, P->quad_work);
+                              P->pair_order, P->pair_idx, part_is_pos, P->row_work, P->pair_work);
   return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
 }
 
@@ -386,13 +366,11 @@ void finalize_layout(bfa_plan* P) {
   P->max_nkt = 0;
   P->max_nqt = 0;
   P->n_pairs = 0;
-  P->n_quads = 0;
   for (auto& g : P->groups_h) {
     g.row0 = row;
     g.cls_off = cls;
     row += g.nqt;
     P->n_pairs += (g.nqt + 1) / 2;
-    P->n_quads += (g.nqt + 3) / 4;
     cls += static_cast<int64_t>(g.nqt) * g.nkt;
     P->max_nkt = std::max(P->max_nkt, g.nkt);
     P->max_nqt = std::max(P->max_nqt, g.nqt);
@@ -1258,7 +1236,6 @@ BFA_API bfa_status bfa_plan_get_info(const bfa_plan* P, bfa_plan_info* info) {
   info->n_pairs = P->n_pairs;
   info->packed_fine = P->mask_mode == MASK_BITS ? 1 : 0;
   info->n_cols = plan_n_cols(P);
-  info->n_quads = P->n_quads;
   return BFA_OK;
 }
 
@@ -1332,22 +1309,6 @@ BFA_API bfa_status bfa_plan_export_pairs(const bfa_plan* P, int32_t* pair_row, i
                "read pair order");
   }
   BFA_CUDA(cudaStreamSynchronize(st), "export pairs");
-  return BFA_OK;
-}
-
-BFA_API bfa_status bfa_plan_export_quads(const bfa_plan* P, int32_t* quad_row, int32_t* quad_order, void* stream) {
-  if (!P) return fail(BFA_ERR_INVALID_ARG, "plan is NULL");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  auto cleanup = []() {};
-  if (P->n_quads > 0) {
-    if (quad_row)
-      BFA_CUDA(cudaMemcpyAsync(quad_row, P->quad_row, sizeof(int32_t) * P->n_quads, cudaMemcpyDeviceToHost, st),
-               "read quads");
-    if (quad_order)
-      BFA_CUDA(cudaMemcpyAsync(quad_order, P->quad_order, sizeof(int32_t) * P->n_quads, cudaMemcpyDeviceToHost, st),
-               "read quad order");
-  }
-  BFA_CUDA(cudaStreamSynchronize(st), "export quads");
   return BFA_OK;
 }
 

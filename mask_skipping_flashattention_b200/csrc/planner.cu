@@ -327,9 +327,7 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
                                                int32_t* __restrict__ order, int32_t* __restrict__ pair_row,
                                                int32_t* __restrict__ pair_cost, int32_t* __restrict__ pair_order,
                                                int32_t* __restrict__ pair_idx, int part_is_pos,
-                                               int2* __restrict__ row_work, int2* __restrict__ pair_work,
-                                               int32_t* __restrict__ quad_row, int32_t* __restrict__ quad_cost,
-                                               int32_t* __restrict__ quad_order, int2* __restrict__ quad_work) {
+                                               int2* __restrict__ row_work, int2* __restrict__ pair_work) {
   extern __shared__ int32_t bucket[];
   __shared__ int32_t small_keys[kSmallOrder];
   __shared__ int32_t warp_sums[32];
@@ -407,34 +405,6 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
       const int pr = pair_row[pair_order[i]];
       pair_work[i] = make_int2(pr, row_group[pr >= 0 ? pr : ~pr]);
     }
-  if (quad_row == nullptr) return;
-
-  // 6. quads (the work unit of a pair of SMs): a row opens a quad when its tile
-  //    index inside its group is a multiple of 4; a quad holds up to 4 rows of
-  //    its group and costs their listed tiles
-  __syncthreads();  // pair_idx is reused as the quad index
-  auto opens4 = [&](int r) {
-    const GroupInfo g = groups[row_group[r]];
-    return ((r - g.row0) & 3) == 0 ? 1 : 0;
-  };
-  const int n_quads = block_exclusive_scan(n_rows, opens4, pair_idx, warp_sums, &carry);
-  for (int r = tid; r < n_rows; r += blockDim.x) {
-    const GroupInfo g = groups[row_group[r]];
-    if (((r - g.row0) & 3) != 0) continue;
-    const int end = min(r + 4, g.row0 + g.nqt);
-    int cost = 0;
-    for (int x = r; x < end; ++x) cost += row_cnt[x];
-    const int qi = pair_idx[r];
-    quad_row[qi] = r;
-    quad_cost[qi] = cost;
-  }
-  __syncthreads();
-  if (n_quads <= kSmallOrder) block_stable_order_desc_small(n_quads, quad_cost, small_keys, quad_order);
-  else block_stable_order_desc(n_quads, quad_cost, 4 * max_nkt, bucket, quad_order);
-  for (int i = tid; i < n_quads; i += blockDim.x) {
-    const int qr = quad_row[quad_order[i]];
-    quad_work[i] = make_int2(qr, row_group[qr]);
-  }
 }
 
 // Transposed lists for the backward's key-tile pass (BinFlash's dK/dV pass over
@@ -827,18 +797,15 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row, int32_t* pair_cost,
                         int32_t* pair_order, int32_t* pair_idx, int part_is_pos, int2* row_work,
-                        int2* pair_work, int32_t* quad_row, int32_t* quad_cost, int32_t* quad_order,
-                        int2* quad_work) {
-  // bucket of the counting sorts: keys up to 2 max_nkt (pairs), 4 max_nkt (quads)
-  const size_t smem = sizeof(int32_t) * static_cast<size_t>((quad_row ? 4 : 2) * max_nkt + 1);
+                        int2* pair_work) {
+  const size_t smem = sizeof(int32_t) * static_cast<size_t>(2 * max_nkt + 1);
   if (smem > 48 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order,
-                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos, row_work, pair_work,
-                               quad_row, quad_cost, quad_order, quad_work);
+                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos, row_work, pair_work);
   return cudaGetLastError();
 }
 

@@ -21,10 +21,6 @@ Readings fixed here (the pages leave them open):
   tile alone when the group has an odd number); pairs are listed group by group,
   stored as their first row (bit-inverted, ~row, for a single-row pair), and
   ordered longest-first by the pair's total listed tiles, ties by pair index;
-* work quads (the unit of a pair of SMs that share one product): inside each
-  group, query tiles (4i .. 4i+3) form one quad (fewer tiles at the group's end);
-  quads are listed group by group, stored as their first row, and ordered
-  longest-first by the quad's total listed tiles, ties by quad index;
 * a plan over several groups (batches, sequences, or BSR head groups) is the
   concatenation of the groups' rows in group order.
 
@@ -107,7 +103,7 @@ def combine_groups(group_plans, BM=128, BN=128):
         parts += rp
         fines += fn
     counts = np.array([len(x) for x in lists], dtype=np.int32)
-    pair_row, pair_cost, quad_row, quad_cost = [], [], [], []
+    pair_row, pair_cost = [], []
     r0 = 0
     for cls in cls_all:
         nqt = cls.shape[0]
@@ -115,9 +111,6 @@ def combine_groups(group_plans, BM=128, BN=128):
             two = i + 1 < nqt
             pair_row.append(r0 + i if two else ~(r0 + i))
             pair_cost.append(int(counts[r0 + i]) + (int(counts[r0 + i + 1]) if two else 0))
-        for i in range(0, nqt, 4):
-            quad_row.append(r0 + i)
-            quad_cost.append(int(counts[r0 + i:r0 + min(i + 4, nqt)].sum()))
         r0 += nqt
     row_ptr = np.zeros(len(lists) + 1, dtype=np.int32)
     row_ptr[1:] = np.cumsum(counts)
@@ -135,8 +128,6 @@ def combine_groups(group_plans, BM=128, BN=128):
         "order": lpt_order(counts),
         "pair_row": np.array(pair_row, dtype=np.int32),
         "pair_order": lpt_order(pair_cost),
-        "quad_row": np.array(quad_row, dtype=np.int32),
-        "quad_order": lpt_order(quad_cost),
     }
 
 

@@ -33,9 +33,6 @@ def assert_plan_equal(got, ref):
     if "pair_row" in got:
         np.testing.assert_array_equal(got["pair_row"], ref["pair_row"], err_msg="pair rows")
         np.testing.assert_array_equal(got["pair_order"], ref["pair_order"], err_msg="pair order")
-    if "quad_row" in got:
-        np.testing.assert_array_equal(got["quad_row"], ref["quad_row"], err_msg="quad rows")
-        np.testing.assert_array_equal(got["quad_order"], ref["quad_order"], err_msg="quad order")
 
 
 def compare_rows(O_gpu, L_gpu, O_ref, L_ref, where=""):

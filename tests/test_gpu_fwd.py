@@ -300,6 +300,24 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     test_default_scale_matches_explicit()
 
 
+def test_max_jump_in_a_later_key_tile():
+    """Scores of some key tiles far above the earlier ones: a row's running max
+    grows by much more than 2^8 after its first tile, so the forward must move
+    its reference max and rescale the O it has accumulated."""
+    B, H, N, D = 1, 4, 1024, 128
+    q, k, v = (_rand((B, N, H, D), 9300 + i) for i in range(3))
+    k = k.float()
+    k[:, 5 * 128:6 * 128] *= 12.0          # key tile 5: scores about 12 x larger
+    k[:, 700:704] *= 20.0                  # and a few keys of tile 5 larger still
+    k = k.to(torch.bfloat16)
+    M = np.tril(np.ones((N, N), dtype=bool))
+    P = bfa.plan_dense(_cuda(M))
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    P.device_status()
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M, None, [(0, h) for h in range(H)], where="max jump")
+
+
 def test_forward_and_backward_give_up_on_a_short_wait_bound():
     """The kernels' own failure path: with the shortest loop-wait bound (1 us) the
     first wait of a block for its scores outlasts the bound (the copies of Q and K

@@ -198,63 +198,6 @@ def _brute_pairs(masks, BM=128, BN=128):
     return pair_row, order
 
 
-def _brute_quads(masks, BM=128, BN=128):
-    """Work quads recomputed from the masks with plain loops: inside each group,
-    query tiles (4i .. 4i + 3) form a quad (fewer at the group's end), stored as
-    its first row; a quad costs the non-empty key tiles of its rows; the order is
-    longest first, ties by quad index (insertion sort, stable)."""
-    quad_row, cost = [], []
-    r0 = 0
-    for M in masks:
-        Sq, Sk = M.shape
-        nqt, nkt = -(-Sq // BM), -(-Sk // BN)
-        i = 0
-        while i < nqt:
-            c = 0
-            for qt in range(i, min(i + 4, nqt)):
-                for kt in range(nkt):
-                    if M[qt * BM:(qt + 1) * BM, kt * BN:(kt + 1) * BN].any():
-                        c += 1
-            quad_row.append(r0 + i)
-            cost.append(c)
-            i += 4
-        r0 += nqt
-    order = []
-    for p in range(len(cost)):
-        pos = len(order)
-        while pos > 0 and cost[order[pos - 1]] < cost[p]:
-            pos -= 1
-        order.insert(pos, p)
-    return quad_row, order
-
-
-@pytest.mark.parametrize("seed", range(3))
-def test_work_quads_match_brute_force(seed):
-    rng = np.random.default_rng(400 + seed)
-    masks = [
-        rng.random((7 * 128 + 3, 700)) < 0.004,         # 8 tiles, ragged last tile
-        np.tril(np.ones((128, 128), dtype=bool)),       # a group of one tile
-        np.zeros((0, 256), dtype=bool),                 # an empty group
-        rng.random((6 * 128, 3 * 128 + 5)) < 0.5,       # 6 tiles: one quad and a half quad
-        np.tril(np.ones((5 * 128 - 1, 5 * 128 - 1), dtype=bool)),
-        np.zeros((300, 260), dtype=bool),
-    ]
-    P = op.plan_masks(masks)
-    quad_row, order = _brute_quads(masks)
-    np.testing.assert_array_equal(P["quad_row"], np.array(quad_row, dtype=np.int32))
-    np.testing.assert_array_equal(P["quad_order"], np.array(order, dtype=np.int32))
-
-
-def test_work_quads_of_the_causal_grid_closed_form():
-    """Causal 8192: quad i holds tiles 4i .. 4i + 3 with 16 i + 10 listed tiles, so
-    the longest-first order is the quads in reverse."""
-    n = 64
-    M = np.tril(np.ones((n * 128, n * 128), dtype=bool))
-    P = op.plan_masks([M])
-    assert P["quad_row"].tolist() == list(range(0, n, 4))
-    assert P["quad_order"].tolist() == list(range(n // 4 - 1, -1, -1))
-
-
 @pytest.mark.parametrize("seed", range(3))
 def test_work_pairs_match_brute_force(seed):
     rng = np.random.default_rng(300 + seed)
