@@ -22,8 +22,11 @@
 namespace bfa {
 
 // kernels (planner.cu, fwd.cu)
+// With `groups` set, the launch also writes the dense plan's single group
+// (*group), its row -> group map and clears the status words.
 cudaError_t launch_dense_classify(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* cls, uint32_t* fine,
-                                  cudaStream_t s);
+                                  cudaStream_t s, GroupInfo* groups = nullptr, const GroupInfo* group = nullptr,
+                                  int32_t* row_group = nullptr, uint32_t* err = nullptr, int32_t* max_width = nullptr);
 cudaError_t launch_blockid_classify(const GroupInfo* groups, int n_groups, int max_tiles_q, int max_tiles_k,
                                     const int32_t* q_blk, const int32_t* k_blk, const uint8_t* q_valid,
                                     const uint8_t* k_valid, int batched, int Sq, int Sk, int window, int copy_ids,
@@ -36,7 +39,8 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row = nullptr, int32_t* pair_cost = nullptr,
                         int32_t* pair_order = nullptr, int32_t* pair_idx = nullptr, int part_is_pos = 0,
-                        int2* row_work = nullptr, int2* pair_work = nullptr);
+                        int2* row_work = nullptr, int2* pair_work = nullptr, int n_groups = 0,
+                        int64_t grid_tiles = -1);
 cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int n_groups,
                                int nqb, int nkb, int wpr, uint32_t* bits, uint32_t* err, cudaStream_t s);
 cudaError_t launch_cols(const GroupInfo* groups, int n_groups, const uint8_t* cls, const int32_t* row_ptr,
@@ -208,8 +212,10 @@ struct SlabLayout {
 };
 
 // Allocate and carve the plan slab; uploads groups and row_group.
+// `init_later`: a regular layout whose group table and status words the
+// caller's first kernel writes (dense plans: the classify launch).
 bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t kid_elems, int64_t kbit_words,
-                      int64_t term_ints = 0) {
+                      int64_t term_ints = 0, bool init_later = false) {
   SlabLayout L;
   const int64_t cap_tiles = std::max<int64_t>(P->grid_tiles, 1);
   const size_t o_groups = L.take<GroupInfo>(std::max(P->n_groups, 1));
@@ -264,7 +270,9 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   P->terms = reinterpret_cast<int32_t*>(base + o_terms);
   P->fine = reinterpret_cast<uint32_t*>(base + o_fine);
 
-  if (P->regular) {
+  if (P->regular && init_later) {
+    // nothing to launch here
+  } else if (P->regular) {
     // the same launch clears the status words (err, max_width)
     e = launch_init_regular_groups(P->groups_h[0], P->n_groups, P->regular_hkv, P->kind == BFA_PLAN_BSR ? 1 : 0,
                                    P->copy_ids ? 1 : 0, P->groups, P->row_group, P->n_rows, P->stream, P->err,
@@ -309,7 +317,8 @@ bfa_status build_rows(bfa_plan* P, int part_is_pos = 0) {
   if (P->max_nkt > kMaxKvTiles) return fail(BFA_ERR_CAPACITY, "too many key tiles per row (%d)", P->max_nkt);
   cudaError_t e = launch_rows(P->groups, P->row_group, P->cls, P->n_rows, P->max_nkt, P->row_cnt, P->row_ptr,
                               P->kv_tile, P->part, P->order, P->stream, P->pair_row, P->pair_cost,
-                              P->pair_order, P->pair_idx, part_is_pos, P->row_work, P->pair_work);
+                              P->pair_order, P->pair_idx, part_is_pos, P->row_work, P->pair_work, P->n_groups,
+                              P->grid_tiles);
   return e == cudaSuccess ? BFA_OK : cuda_fail(e, "plan rows kernel");
 }
 
@@ -480,9 +489,12 @@ BFA_API bfa_status bfa_plan_dense(const uint8_t* mask, int64_t ld, int Sq, int S
   P->regular = true;
   finalize_layout(P);
   if ((s = check_capacity(P, true))) { cleanup(); return s; }
-  if ((s = alloc_plan(P, true, 0, 0, 0))) { cleanup(); return s; }
+  if ((s = alloc_plan(P, true, 0, 0, 0, 0, /*init_later=*/true))) { cleanup(); return s; }
   P->fine_tiles = P->grid_tiles;
-  BFA_CUDA(launch_dense_classify(mask, ld, Sq, Sk, P->cls, P->fine, P->stream), "dense classify kernel");
+  GroupInfo g0 = P->groups_h[0];
+  BFA_CUDA(launch_dense_classify(mask, ld, Sq, Sk, P->cls, P->fine, P->stream, P->groups, &g0, P->row_group, P->err,
+                                 P->max_width),
+           "dense classify kernel");
   if ((s = build_rows(P))) { cleanup(); return s; }
   *out = P;
   return BFA_OK;

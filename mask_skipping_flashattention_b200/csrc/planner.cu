@@ -25,6 +25,7 @@ namespace bfa {
 // with one 16-byte load per row, so each warp instruction reads 512 contiguous
 // mask bytes.  Each warp owns 16 rows.
 constexpr int kDenseTilesPerCta = 4;
+constexpr size_t kRowsStageBytes = 160 * 1024;  // k_rows: largest staged group table + row map + class grid
 
 __device__ __forceinline__ uint32_t nz_bytes4(uint32_t x) {
   // bit k (k < 4) set iff byte k of x is nonzero
@@ -35,20 +36,60 @@ __device__ __forceinline__ uint32_t nz_bytes4(uint32_t x) {
   return ((t * 0x01020408u) >> 24) & 0xFu;
 }
 
+// Optional set-up of a dense plan done by the classify launch itself (one
+// launch fewer): its single group, the row -> group map and the status words.
+struct DenseInit {
+  GroupInfo* groups;  // nullptr: nothing to do
+  GroupInfo group;
+  int32_t* row_group;
+  uint32_t* err;
+  int32_t* max_width;
+};
+
 __global__ void __launch_bounds__(256) k_dense_classify(const uint8_t* __restrict__ mask, int64_t ld, int Sq,
                                                         int Sk, int nkt, uint8_t* __restrict__ cls,
-                                                        uint32_t* __restrict__ fine, int vec_ok) {
+                                                        uint32_t* __restrict__ fine, int vec_ok,
+                                                        const DenseInit init) {
   __shared__ uint32_t words[kDenseTilesPerCta][kTile][kWordsPerTileRow];  // 8 KB
   __shared__ int tile_cnt[kDenseTilesPerCta];
   const int qt = blockIdx.y;
   const int kt0 = blockIdx.x * kDenseTilesPerCta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < kDenseTilesPerCta) tile_cnt[threadIdx.x] = 0;
+  if (init.groups != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+    init.row_group[qt] = 0;
+    if (qt == 0) {
+      *init.groups = init.group;
+      *init.err = 0u;
+      *init.max_width = 0;
+    }
+  }
   const int t = lane >> 3, chunk = lane & 7;
   const int64_t col0 = static_cast<int64_t>(kt0 + t) * kTile + chunk * 16;
   const int rows_here = min(kTile, Sq - qt * kTile);
 
   uint32_t m16[16];
+  // A CTA whose 128 rows x 512 bytes all lie inside the mask (every CTA but those
+  // on the ragged edges) issues its 16 row loads per thread before using any of
+  // them, so that they are all in flight at once; the edge path below checks
+  // each row and column.
+  const bool inside = vec_ok && rows_here == kTile && (kt0 + kDenseTilesPerCta) * kTile <= Sk;
+  if (inside) {
+    uint4 v[16];
+    const uint8_t* base = mask + static_cast<int64_t>(qt * kTile + warp * 16) * ld + col0;
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) v[rr] = __ldg(reinterpret_cast<const uint4*>(base + rr * ld));
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) {
+      const uint4 x = v[rr];
+      if (((x.x | x.y | x.z | x.w) & 0xFEFEFEFEu) == 0u) {
+        m16[rr] = ((x.x * 0x01020408u) >> 24) | (((x.y * 0x01020408u) >> 24) << 4) |
+                  (((x.z * 0x01020408u) >> 24) << 8) | (((x.w * 0x01020408u) >> 24) << 12);
+      } else {
+        m16[rr] = nz_bytes4(x.x) | (nz_bytes4(x.y) << 4) | (nz_bytes4(x.z) << 8) | (nz_bytes4(x.w) << 12);
+      }
+    }
+  } else {
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) {
     const int r = warp * 16 + rr;
@@ -71,6 +112,7 @@ __global__ void __launch_bounds__(256) k_dense_classify(const uint8_t* __restric
       }
     }
     m16[rr] = m;
+  }
   }
   int cnt = 0;
 #pragma unroll
@@ -327,18 +369,51 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
                                                int32_t* __restrict__ order, int32_t* __restrict__ pair_row,
                                                int32_t* __restrict__ pair_cost, int32_t* __restrict__ pair_order,
                                                int32_t* __restrict__ pair_idx, int part_is_pos,
-                                               int2* __restrict__ row_work, int2* __restrict__ pair_work) {
-  extern __shared__ int32_t bucket[];
+                                               int2* __restrict__ row_work, int2* __restrict__ pair_work,
+                                               int n_groups, int64_t grid_tiles, int stage) {
+  extern __shared__ __align__(16) int32_t bucket[];
   __shared__ int32_t small_keys[kSmallOrder];
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const uint32_t lt_mask = (1u << lane) - 1u;
 
+  // 0. with `stage`, the group table, the row -> group map and the class grid are
+  //    copied to shared memory first (coalesced), so that the per-row passes
+  //    below read them there instead of in dependent global loads; the area is
+  //    reused by the sort buckets from step 4 on
+  const GroupInfo* sgroups = groups;
+  const int32_t* srow_group = row_group;
+  const uint8_t* scls = cls;
+  if (stage) {
+    GroupInfo* g_s = reinterpret_cast<GroupInfo*>(bucket);
+    int32_t* rg_s = reinterpret_cast<int32_t*>(g_s + n_groups);
+    uint8_t* c_s = reinterpret_cast<uint8_t*>(rg_s + n_rows);
+    const int32_t* gw = reinterpret_cast<const int32_t*>(groups);
+    int32_t* gws = reinterpret_cast<int32_t*>(g_s);
+    for (int i = tid; i < n_groups * static_cast<int>(sizeof(GroupInfo) / 4); i += blockDim.x) gws[i] = gw[i];
+    for (int i = tid; i < n_rows; i += blockDim.x) rg_s[i] = row_group[i];
+    const int64_t n16 = grid_tiles >> 4;  // the class grid starts 256-byte aligned in the plan slab
+    const uint4* c16 = reinterpret_cast<const uint4*>(cls);
+    for (int64_t i = tid; i < n16; i += blockDim.x) {
+      const uint4 v = c16[i];
+      uint8_t* d = c_s + 16 * i;
+      reinterpret_cast<uint32_t*>(d)[0] = v.x;  // c_s is 4-byte aligned
+      reinterpret_cast<uint32_t*>(d)[1] = v.y;
+      reinterpret_cast<uint32_t*>(d)[2] = v.z;
+      reinterpret_cast<uint32_t*>(d)[3] = v.w;
+    }
+    for (int64_t i = 16 * n16 + tid; i < grid_tiles; i += blockDim.x) c_s[i] = cls[i];
+    __syncthreads();
+    sgroups = g_s;
+    srow_group = rg_s;
+    scls = c_s;
+  }
+
   // 1. count the listed tiles of every row (warp per row, ballot + popc)
   for (int r = warp; r < n_rows; r += nw) {
-    const GroupInfo g = groups[row_group[r]];
-    const uint8_t* c = cls + g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
+    const GroupInfo g = sgroups[srow_group[r]];
+    const uint8_t* c = scls + g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
     int n = 0;
     for (int k0 = 0; k0 < g.nkt; k0 += 32) {
       const int kt = k0 + lane;
@@ -355,9 +430,9 @@ __global__ void __launch_bounds__(1024) k_rows(const GroupInfo* __restrict__ gro
 
   // 3. write each row's ascending list (warp per row)
   for (int r = warp; r < n_rows; r += nw) {
-    const GroupInfo g = groups[row_group[r]];
+    const GroupInfo g = sgroups[srow_group[r]];
     const int64_t rowoff = g.cls_off + static_cast<int64_t>(r - g.row0) * g.nkt;
-    const uint8_t* c = cls + rowoff;
+    const uint8_t* c = scls + rowoff;
     int out = row_ptr[r];
     for (int k0 = 0; k0 < g.nkt; k0 += 32) {
       const int kt = k0 + lane;
@@ -759,11 +834,18 @@ cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int 
 }
 
 cudaError_t launch_dense_classify(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* cls, uint32_t* fine,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, GroupInfo* groups, const GroupInfo* group, int32_t* row_group,
+                                  uint32_t* err, int32_t* max_width) {
   const int nqt = (Sq + kTile - 1) / kTile, nkt = (Sk + kTile - 1) / kTile;
   const int vec_ok = ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (ld & 15) == 0) ? 1 : 0;
+  DenseInit init;
+  init.groups = groups;
+  if (groups != nullptr) init.group = *group;
+  init.row_group = row_group;
+  init.err = err;
+  init.max_width = max_width;
   dim3 grid((nkt + kDenseTilesPerCta - 1) / kDenseTilesPerCta, nqt);
-  k_dense_classify<<<grid, 256, 0, s>>>(mask, ld, Sq, Sk, nkt, cls, fine, vec_ok);
+  k_dense_classify<<<grid, 256, 0, s>>>(mask, ld, Sq, Sk, nkt, cls, fine, vec_ok, init);
   return cudaGetLastError();
 }
 
@@ -797,15 +879,22 @@ cudaError_t launch_rows(const GroupInfo* groups, const int32_t* row_group, const
                         int max_nkt, int32_t* row_cnt, int32_t* row_ptr, int32_t* kv_tile, int32_t* part,
                         int32_t* order, cudaStream_t s, int32_t* pair_row, int32_t* pair_cost,
                         int32_t* pair_order, int32_t* pair_idx, int part_is_pos, int2* row_work,
-                        int2* pair_work) {
-  const size_t smem = sizeof(int32_t) * static_cast<size_t>(2 * max_nkt + 1);
+                        int2* pair_work, int n_groups, int64_t grid_tiles) {
+  // bucket of the counting sorts (keys up to 2 max_nkt), shared with the staged
+  // copies of the group table, the row map and the class grid when they fit
+  const size_t bucket_bytes = sizeof(int32_t) * static_cast<size_t>(2 * max_nkt + 1);
+  const size_t stage_bytes = sizeof(GroupInfo) * static_cast<size_t>(n_groups) +
+                             sizeof(int32_t) * static_cast<size_t>(n_rows) + static_cast<size_t>(grid_tiles);
+  const int stage = (n_groups > 0 && grid_tiles >= 0 && stage_bytes <= kRowsStageBytes) ? 1 : 0;
+  const size_t smem = stage ? (bucket_bytes > stage_bytes ? bucket_bytes : stage_bytes) : bucket_bytes;
   if (smem > 48 * 1024) {
     cudaError_t e =
         cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   k_rows<<<1, 1024, smem, s>>>(groups, row_group, cls, n_rows, max_nkt, row_cnt, row_ptr, kv_tile, part, order,
-                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos, row_work, pair_work);
+                               pair_row, pair_cost, pair_order, pair_idx, part_is_pos, row_work, pair_work, n_groups,
+                               grid_tiles, stage);
   return cudaGetLastError();
 }
 
