@@ -29,9 +29,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-# kernels of one step: k_init_regular_groups, k_dense_classify, k_rows (the plan)
-# and bfa_fwd_kernel<128> (the forward)
-LAUNCHES_PER_STEP = 4
+# kernels of one step: k_dense_classify, k_rows (the plan) and bfa_fwd_kernel<128>
+# (the forward)
+LAUNCHES_PER_STEP = 3
 METRIC = "masked attn fwd TFLOP/s on attended pairs (bf16), % of B200 tensor peak"
 WORKLOAD = dict(workload="causal_8192", B=4, H=32, Hkv=32, N=8192, D=128, mask="dense causal (N,N) bool",
                 plan="bfa_plan_dense per step", layout="BSHD")
@@ -418,7 +418,7 @@ def run_bfa(args, rank, world, local_rank):
                      "traffic": _fwd_traffic(), "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "algorithmic_bytes": algo_bytes},
         "fwd_ms": fwd_ms, "plan_ms": plan_ms,
-        "planner": {"call": "bfa_plan_dense (k_init_regular_groups, k_dense_classify, k_rows)", "bound": "hbm",
+        "planner": {"call": "bfa_plan_dense (k_dense_classify, k_rows)", "bound": "hbm",
                     "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{src} hbm_gbs",
                     "l2": "256 MB written before every timed call", **{
                         k: dict(v, frac=v["gbs"] / peaks["hbm_gbs"]) for k, v in planner.items()}},
@@ -470,12 +470,22 @@ def run_sweep(args):
 
     torch.cuda.set_device(0)
     reps = max(3, args.steps)
+    only = args.workload  # None: every workload
 
     def cuda(x):
         return torch.as_tensor(np.ascontiguousarray(x)).cuda()
 
     def measure(name, P, q, k, v, pairs, D, plan_desc):
+        if only is not None and name != only:
+            return
         out, lse = bfa.fwd(P, q, k, v)
+        if args.fwd_only:  # a few forward calls only (an ncu capture of the forward)
+            for _ in range(reps):
+                bfa.fwd(P, q, k, v, out=out, lse=lse)
+            torch.cuda.synchronize()
+            P.device_status()
+            print(json.dumps({"workload": name, "fwd_calls": reps + 1}), flush=True)
+            return
         g = torch.Generator(device="cuda")
         g.manual_seed(7)
         dout = torch.randn(q.shape, device="cuda", generator=g).to(torch.bfloat16)
@@ -536,6 +546,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-union-planner", action="store_true", help="skip the planner leg on the 268 MB union mask")
     ap.add_argument("--sweep", action="store_true", help="forward/backward on every workload (information)")
+    ap.add_argument("--workload", default=None,
+                    help="with --sweep: only this workload (causal_8192, blockcausal_gqa, 'varlen_16 window=-1', "
+                         "'varlen_16 window=1024', bsr_16384, union_16384)")
+    ap.add_argument("--fwd-only", action="store_true", help="with --sweep: forward calls only, no timing line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

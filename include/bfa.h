@@ -59,7 +59,9 @@ typedef enum bfa_status {
   BFA_ERR_NONCANONICAL_BSR = -4, /* BSR rows not sorted / unique / in range             */
   BFA_ERR_CAPACITY = -5,         /* sizes beyond what the library can index or allocate */
   BFA_ERR_CUDA = -6,             /* a CUDA runtime call failed                          */
-  BFA_ERR_TIMEOUT = -7           /* a device-side wait ran past its bound               */
+  BFA_ERR_TIMEOUT = -7,          /* a device-side wait ran past its bound               */
+  BFA_ERR_BOUNDS = -8            /* checked build only: an index left its array, or the
+                                    guard bytes after a plan array were overwritten      */
 } bfa_status;
 
 enum { BFA_TILE = 128 };
@@ -338,7 +340,13 @@ bfa_status bfa_plan_export_cols(const bfa_plan* plan, int32_t* col_ptr, int32_t*
                                 int32_t* col_order, void* stream);
 
 /* Synchronise `stream` and report BFA_ERR_TIMEOUT if a kernel that used the plan
- * hit its wait bound since the last call (the flag is then cleared). */
+ * hit its wait bound since the last call (the flag is then cleared).
+ * The checked build of the library (libbfa_checked.so, compiled with
+ * -DBFA_CHECKED: a stand-in for a memory checker) also bounds-checks every
+ * plan-indexed access of its kernels, skipping the access and flagging it, and
+ * surrounds every plan array with guard bytes; this call then first verifies the
+ * guard bytes and reports BFA_ERR_BOUNDS if an index left its array or a guard
+ * was overwritten (the flags are then cleared). */
 bfa_status bfa_plan_device_status(const bfa_plan* plan, void* stream);
 
 /* Free a plan in stream order on the stream it was built on.  Work on other

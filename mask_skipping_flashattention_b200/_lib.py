@@ -9,7 +9,10 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libbfa.so")
+# BFA_LIBRARY=checked selects the bounds-checked build (libbfa_checked.so: the
+# same kernels with every plan-indexed access checked and guard bytes around
+# plan arrays, reported by bfa_plan_device_status); the default is libbfa.so.
+LIB_PATH = os.path.join(_HERE, "libbfa_checked.so" if os.environ.get("BFA_LIBRARY") == "checked" else "libbfa.so")
 
 c_i32p = ctypes.POINTER(ctypes.c_int32)
 c_i64p = ctypes.POINTER(ctypes.c_int64)
@@ -20,6 +23,7 @@ c_void = ctypes.c_void_p
 STATUS = {
     0: "BFA_OK", -1: "BFA_ERR_INVALID_ARG", -2: "BFA_ERR_UNSUPPORTED", -3: "BFA_ERR_NOT_DEVICE",
     -4: "BFA_ERR_NONCANONICAL_BSR", -5: "BFA_ERR_CAPACITY", -6: "BFA_ERR_CUDA", -7: "BFA_ERR_TIMEOUT",
+    -8: "BFA_ERR_BOUNDS",
 }
 
 # every entry point declared in include/bfa.h: name -> (restype, argtypes)

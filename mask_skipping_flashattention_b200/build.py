@@ -19,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbfa.so")
+LIB_CHECKED = os.path.join(PKG, "libbfa_checked.so")
 SOURCES = ["planner.cu", "fwd.cu", "bwd.cu", "bfa_host.cu"]
 HEADERS = ["ptx.cuh", "plan_types.cuh", "fwd_params.cuh", "pred.cuh", "tile_mask.cuh", "bwd_params.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -41,16 +42,23 @@ def _stale(target, deps):
 
 
 def build(force=False, verbose=False):
-    os.makedirs(BUILD, exist_ok=True)
+    """Build libbfa.so and its bounds-checked twin libbfa_checked.so (-DBFA_CHECKED)."""
+    lib = _build_one(LIB, BUILD, [], force, verbose)
+    _build_one(LIB_CHECKED, os.path.join(BUILD, "checked"), ["-DBFA_CHECKED"], force, verbose)
+    return lib
+
+
+def _build_one(lib_path, build_dir, defines, force, verbose):
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", "bfa.h")]
     objs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD, src.replace(".cu", ".o"))
+        o = os.path.join(build_dir, src.replace(".cu", ".o"))
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
-            cmd = [nvcc, *ARCH, *FLAGS, "-c", s, "-o", o]
+            cmd = [nvcc, *ARCH, *FLAGS, *defines, "-c", s, "-o", o]
             r = subprocess.run(cmd, capture_output=True, text=True)
             log = r.stdout + r.stderr
             with open(o + ".log", "w") as f:
@@ -60,13 +68,13 @@ def build(force=False, verbose=False):
                 raise RuntimeError(f"nvcc failed on {src}")
             if verbose:
                 sys.stdout.write(log)
-    if force or _stale(LIB, objs):
-        cmd = [nvcc, *ARCH, "-shared", "-o", LIB, *objs, "-cudart", "static"]
+    if force or _stale(lib_path, objs):
+        cmd = [nvcc, *ARCH, "-shared", "-o", lib_path, *objs, "-cudart", "static"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("link of libbfa.so failed")
-    return LIB
+            raise RuntimeError(f"link of {os.path.basename(lib_path)} failed")
+    return lib_path
 
 
 def main():

@@ -62,6 +62,8 @@ cudaError_t launch_pred_classify(const int32_t* terms, int n_terms, const GroupI
 cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int n_hkv, int bsr, int copy_ids,
                                        GroupInfo* groups, int32_t* row_group, int n_rows, cudaStream_t s,
                                        uint32_t* err = nullptr, int32_t* max_width = nullptr);
+cudaError_t launch_check_guards(const void* slab, const uint64_t* offs, int n, uint32_t guard_bytes, int guard_byte,
+                                uint32_t* err, cudaStream_t s);
 
 
 }  // namespace bfa
@@ -117,6 +119,14 @@ struct bfa_plan {
   int32_t* q_tile = nullptr;     // [listed tiles]
   int32_t* tpart = nullptr;      // [listed tiles]
   int32_t* col_order = nullptr;  // [n_cols]
+  // capacities of the id copies (entries), for the checked build's index checks
+  int64_t cap_qid = 1, cap_kid = 1, cap_kbits = 1;
+  // checked build: guard regions after every slab array (offsets into the slab,
+  // held in the slab's last region so that a kernel can verify them)
+  int n_guards = 0, n_col_guards = 0;
+  const uint64_t* guard_offs = nullptr;
+  const uint64_t* col_guard_offs = nullptr;
+  std::vector<uint64_t> guards_h, col_guards_h;
 };
 
 namespace {
@@ -201,15 +211,47 @@ constexpr int kMaxKvTiles = 16384;  // key tiles per row: the row kernel's share
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The checked build places kGuardBytes of guard bytes (kGuardByte) right after
+// every array of a slab; bfa_plan_device_status verifies them.
+constexpr size_t kGuardBytes = 64;
+constexpr int kGuardByte = 0xA5;
+#ifdef BFA_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
 struct SlabLayout {
   size_t off = 0;
+  std::vector<uint64_t> guards;  // checked build: offsets of the guard regions
   template <typename T>
   size_t take(size_t count) {
     const size_t o = off;
-    off = align256(off + count * sizeof(T));
+    const size_t end = off + count * sizeof(T);
+    if (kChecked) {
+      guards.push_back(end);
+      off = align256(end + kGuardBytes);
+    } else {
+      off = align256(end);
+    }
     return o;
   }
+  // checked build: room for the guard offsets at the end of the slab
+  size_t take_guard_table() { return take<uint64_t>(guards.size() + 1); }
 };
+
+// checked build: fill a new slab with the guard byte and upload its guard table
+cudaError_t arm_guards(void* slab, size_t bytes, SlabLayout& L, size_t o_table, std::vector<uint64_t>& keep,
+                       cudaStream_t st) {
+  if (!kChecked) return cudaSuccess;
+  keep = L.guards;
+  keep.pop_back();  // the table's own guard is not listed (it is written by the upload)
+  cudaError_t e = cudaMemsetAsync(slab, kGuardByte, bytes, st);
+  if (e == cudaSuccess && !keep.empty())
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(slab) + o_table, keep.data(), keep.size() * sizeof(uint64_t),
+                        cudaMemcpyHostToDevice, st);
+  return e;
+}
 
 // Allocate and carve the plan slab; uploads groups and row_group.
 // `init_later`: a regular layout whose group table and status words the
@@ -240,6 +282,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   const size_t o_kb = L.take<uint32_t>(std::max<int64_t>(kbit_words, 1));
   const size_t o_terms = L.take<int32_t>(std::max<int64_t>(term_ints, 1));
   const size_t o_fine = L.take<uint32_t>(with_fine ? static_cast<size_t>(cap_tiles) * kFineWordsPerTile : 1);
+  const size_t o_gtab = kChecked ? L.take_guard_table() : 0;
+  P->cap_qid = std::max<int64_t>(qid_elems, 1);
+  P->cap_kid = std::max<int64_t>(kid_elems, 1);
+  P->cap_kbits = std::max<int64_t>(kbit_words, 1);
   cudaMemPool_t pool;
   cudaError_t e = plan_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "plan memory pool");
@@ -247,6 +293,10 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
   if (e != cudaSuccess) return fail(BFA_ERR_CAPACITY, "plan allocation of %zu bytes failed: %s", L.off,
                                     cudaGetErrorString(e));
   uint8_t* base = static_cast<uint8_t*>(P->slab);
+  e = arm_guards(P->slab, L.off, L, o_gtab, P->guards_h, P->stream);
+  if (e != cudaSuccess) return cuda_fail(e, "plan guard bytes");
+  P->n_guards = static_cast<int>(P->guards_h.size());
+  P->guard_offs = reinterpret_cast<const uint64_t*>(base + o_gtab);
   P->groups = reinterpret_cast<GroupInfo*>(base + o_groups);
   P->row_group = reinterpret_cast<int32_t*>(base + o_rowg);
   P->cls = base + o_cls;
@@ -293,7 +343,8 @@ bfa_status alloc_plan(bfa_plan* P, bool with_fine, int64_t qid_elems, int64_t ki
     if (e != cudaSuccess) return cuda_fail(e, "upload plan rows");
   }
   if (!P->regular) {  // regular layouts cleared them in the group-table launch
-    e = cudaMemsetAsync(P->err, 0, 2 * 256, P->stream);  // err and max_width slots
+    e = cudaMemsetAsync(P->err, 0, sizeof(uint32_t), P->stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(P->max_width, 0, sizeof(int32_t), P->stream);
     if (e != cudaSuccess) return cuda_fail(e, "clear plan status");
   }
   return BFA_OK;
@@ -343,6 +394,7 @@ bfa_status ensure_cols(bfa_plan* P, cudaStream_t st) {
   const size_t o_qt = L.take<int32_t>(cap);
   const size_t o_tp = L.take<int32_t>(cap);
   const size_t o_co = L.take<int32_t>(std::max(n_cols, 1));
+  const size_t o_gtab = kChecked ? L.take_guard_table() : 0;
   cudaMemPool_t pool;
   cudaError_t e = plan_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "plan memory pool");
@@ -352,6 +404,10 @@ bfa_status ensure_cols(bfa_plan* P, cudaStream_t st) {
     return fail(BFA_ERR_CAPACITY, "transposed plan allocation of %zu bytes failed: %s", L.off, cudaGetErrorString(e));
   }
   uint8_t* base = static_cast<uint8_t*>(P->cols_slab);
+  e = arm_guards(P->cols_slab, L.off, L, o_gtab, P->col_guards_h, st);
+  if (e != cudaSuccess) return cuda_fail(e, "transposed plan guard bytes");
+  P->n_col_guards = static_cast<int>(P->col_guards_h.size());
+  P->col_guard_offs = reinterpret_cast<const uint64_t*>(base + o_gtab);
   P->col0 = reinterpret_cast<int32_t*>(base + o_c0);
   P->col_group = reinterpret_cast<int32_t*>(base + o_cg);
   P->col_cnt = reinterpret_cast<int32_t*>(base + o_cc);
@@ -416,7 +472,7 @@ bfa_status check_capacity(const bfa_plan* P, bool with_fine) {
 // ----------------------------------------------------------------------------
 // C ABI
 // ----------------------------------------------------------------------------
-BFA_API const char* bfa_version(void) { return "bfa 0.1 (sm_100a)"; }
+BFA_API const char* bfa_version(void) { return kChecked ? "bfa 0.1 (sm_100a, checked)" : "bfa 0.1 (sm_100a)"; }
 
 BFA_API const char* bfa_last_error(void) { return g_err.c_str(); }
 
@@ -918,6 +974,11 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.plan.terms = P->terms;
   p.plan.n_terms = P->n_terms;
   p.plan.err = P->err;
+  p.plan.cap_tiles = std::max<int64_t>(P->grid_tiles, 1);
+  p.plan.cap_fine = std::max<int64_t>(P->fine_tiles, 1);
+  p.plan.cap_qid = P->cap_qid;
+  p.plan.cap_kid = P->cap_kid;
+  p.plan.cap_kbits = P->cap_kbits;
   p.plan.n_rows = P->n_rows;
   p.plan.n_groups = P->n_groups;
   p.plan.mask_mode = P->mask_mode;
@@ -1045,6 +1106,11 @@ bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const
   p.plan.terms = P->terms;
   p.plan.n_terms = P->n_terms;
   p.plan.err = P->err;
+  p.plan.cap_tiles = std::max<int64_t>(P->grid_tiles, 1);
+  p.plan.cap_fine = std::max<int64_t>(P->fine_tiles, 1);
+  p.plan.cap_qid = P->cap_qid;
+  p.plan.cap_kid = P->cap_kid;
+  p.plan.cap_kbits = P->cap_kbits;
   p.plan.n_rows = P->n_rows;
   p.plan.n_groups = P->n_groups;
   p.plan.mask_mode = P->mask_mode;
@@ -1356,8 +1422,22 @@ BFA_API bfa_status bfa_plan_device_status(const bfa_plan* P, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto cleanup = []() {};
   uint32_t err = 0;
+  if (kChecked) {  // the guard bytes after every plan array must be intact
+    BFA_CUDA(launch_check_guards(P->slab, P->guard_offs, P->n_guards, kGuardBytes, kGuardByte, P->err, st),
+             "guard check kernel");
+    if (P->cols_slab)
+      BFA_CUDA(launch_check_guards(P->cols_slab, P->col_guard_offs, P->n_col_guards, kGuardBytes, kGuardByte, P->err,
+                                   st),
+               "guard check kernel");
+  }
   BFA_CUDA(cudaMemcpyAsync(&err, P->err, sizeof(err), cudaMemcpyDeviceToHost, st), "read device status");
   BFA_CUDA(cudaStreamSynchronize(st), "device status");
+  if (err & (DEVERR_BOUNDS | DEVERR_GUARD)) {
+    BFA_CUDA(cudaMemsetAsync(P->err, 0, sizeof(uint32_t), st), "clear device status");
+    BFA_CUDA(cudaStreamSynchronize(st), "device status");
+    return fail(BFA_ERR_BOUNDS, "checked build: %s%s", (err & DEVERR_BOUNDS) ? "an index left its array " : "",
+                (err & DEVERR_GUARD) ? "guard bytes after a plan array were overwritten" : "");
+  }
   if (err & DEVERR_TIMEOUT) {
     BFA_CUDA(cudaMemsetAsync(P->err, 0, sizeof(uint32_t), st), "clear device status");
     BFA_CUDA(cudaStreamSynchronize(st), "device status");

@@ -269,13 +269,24 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     fence_barrier_init();
     int i, j;
     chunked_decode(blockIdx.x, p.plan.n_rows, p.rep, p.head_chunk, i, j);
-    const int2 rw = p.plan.row_work[i];  // {row, its group}, longest first
-    const int r = rw.x;
+    uint32_t* const err = p.plan.err;
+    (void)err;
+    const int2 rw = p.plan.row_work[BFA_IDX(i, p.plan.n_rows, err)];  // {row, its group}, longest first
+    const int r = static_cast<int>(BFA_IDX(rw.x, p.plan.n_rows, err));
     DqWork w;
-    w.g = p.plan.groups[rw.y];
+    w.g = p.plan.groups[BFA_IDX(rw.y, p.plan.n_groups, err)];
     w.r = r;
     w.e0 = p.plan.row_ptr[r];
     w.n = p.plan.row_ptr[r + 1] - w.e0;
+#ifdef BFA_CHECKED
+    // a list outside the plan's arrays, or a row outside its group, is reported and not walked
+    if (!(w.n >= 0 && w.n <= w.g.nkt && w.e0 >= 0 && w.e0 + w.n <= p.plan.cap_tiles && r >= w.g.row0 &&
+          r < w.g.row0 + w.g.nqt && j >= 0 && j < p.rep)) {
+      atomicOr(err, DEVERR_BOUNDS);
+      w.e0 = 0;
+      w.n = 0;
+    }
+#endif
     w.qt = r - w.g.row0;
     w.j = j;
     replica_bh(p, w.g, j, w.b, w.h);
@@ -508,13 +519,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fence_barrier_init();
     int i, jk;
     chunked_decode(blockIdx.x, p.n_cols, p.rep_kv, p.kv_chunk, i, jk);
-    const int c = p.col_order[i];
-    const int grp = p.col_group[c];
+    uint32_t* const err = p.plan.err;
+    (void)err;
+    const int c = static_cast<int>(BFA_IDX(p.col_order[BFA_IDX(i, p.n_cols, err)], p.n_cols, err));
+    const int grp = static_cast<int>(BFA_IDX(p.col_group[c], p.plan.n_groups, err));
     KvWork w;
     w.g = p.plan.groups[grp];
     w.kt = c - p.col0[grp];
     w.e0 = p.col_ptr[c];
     w.nq = p.col_ptr[c + 1] - w.e0;
+#ifdef BFA_CHECKED
+    // a column outside the transposed lists, or a key tile outside its group, is reported and not walked
+    if (!(w.nq >= 0 && w.nq <= w.g.nqt && w.e0 >= 0 && w.e0 + w.nq <= p.plan.cap_tiles && w.kt >= 0 &&
+          w.kt < w.g.nkt && jk >= 0 && jk < p.rep_kv)) {
+      atomicOr(err, DEVERR_BOUNDS);
+      w.e0 = 0;
+      w.nq = 0;
+    }
+#endif
     w.nh = p.H / p.Hkv;
     kv_replica_bh(p, w.g, jk, w.b, w.hk);
     w.steps = w.nq * w.nh;
@@ -555,8 +577,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (s >= kBwdStages && !mbar_wait_fast(bar(BE + st), ((s >> 1) - 1) & 1, cap, &abort_flag)) break;
         const int h = step_head(s);
         const int qt = p.q_tile[step_entry(s)];
+        BFA_CHECK(qt >= 0 && qt < wk.g.nqt, p.plan.err);
         const int r = wk.g.row0 + qt;
         const int64_t wi = (static_cast<int64_t>(replica_of(p, wk.g, wk.b, h)) * p.plan.n_rows + r) * kTile;
+        BFA_CHECK(wi >= 0 && wi + kTile <= static_cast<int64_t>(p.rep) * p.plan.n_rows * kTile, p.plan.err);
         const uint32_t f = bar(BF + st);
         mbar_expect_tx(f, 2 * C::kTileBytes + C::kVecBytes);
         const int qs = wk.g.q_off + qt * kTile;
@@ -638,6 +662,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int st = s & 1;
       const int e = step_entry(s);
       const int qt = p.q_tile[e], part = p.tpart[e];
+      BFA_CHECK(qt >= 0 && qt < wk.g.nqt, p.plan.err);
       uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       const bool masked = part >= 0 || (qt + 1) * kTile > wk.g.q_len;
       if (masked) col_mask_words(p.plan, ctx, kpos, krow, qt, part, am);

@@ -102,24 +102,35 @@ __device__ __forceinline__ void decode_work(const FwdParams& p, int w, Work& wk)
   const int j = static_cast<int>(hg * chunk + rem % gs);
   // the plan lists the work items in longest-first order with their group
   int r0, r1, grp;
+  uint32_t* const err = p.plan.err;
+  (void)err;
   if (p.pair_heads) {
-    const int2 rw = p.plan.row_work[i];
+    const int2 rw = p.plan.row_work[BFA_IDX(i, p.plan.n_rows, err)];
     r0 = r1 = rw.x;
     grp = rw.y;
   } else {
-    const int2 pw = p.plan.pair_work[i];
+    const int2 pw = p.plan.pair_work[BFA_IDX(i, p.plan.n_pairs, err)];
     r0 = pw.x >= 0 ? pw.x : ~pw.x;
     r1 = pw.x >= 0 ? r0 + 1 : -1;
     grp = pw.y;
   }
-  const GroupInfo g = p.plan.groups[grp];
+  const GroupInfo g = p.plan.groups[BFA_IDX(grp, p.plan.n_groups, err)];
   wk.same_row = p.pair_heads;
   wk.row[0] = r0;
   wk.row[1] = r1;
   for (int s = 0; s < 2; ++s) {
     const int r = wk.row[s];
-    wk.e0[s] = r >= 0 ? p.plan.row_ptr[r] : 0;
-    wk.n[s] = r >= 0 ? p.plan.row_ptr[r + 1] - wk.e0[s] : 0;
+    BFA_CHECK(r < 0 || (r >= g.row0 && r < g.row0 + g.nqt), err);
+    wk.e0[s] = r >= 0 ? p.plan.row_ptr[BFA_IDX(r, p.plan.n_rows, err)] : 0;
+    wk.n[s] = r >= 0 ? p.plan.row_ptr[BFA_IDX(r + 1, p.plan.n_rows + 1, err)] - wk.e0[s] : 0;
+#ifdef BFA_CHECKED
+    // a list outside the plan's arrays is reported and not walked
+    if (!(wk.n[s] >= 0 && wk.n[s] <= g.nkt && wk.e0[s] >= 0 && wk.e0[s] + wk.n[s] <= p.plan.cap_tiles)) {
+      atomicOr(err, DEVERR_BOUNDS);
+      wk.e0[s] = 0;
+      wk.n[s] = 0;
+    }
+#endif
     wk.qt[s] = r >= 0 ? r - g.row0 : 0;
   }
   int b, h0, h1;
@@ -154,7 +165,7 @@ struct UnionWalk {
   int ka, kb, ka2, kb2;  // heads of both lists and the entries after them
   bool same;
   __device__ __forceinline__ void init(const FwdParams& p, const Work& wk) {
-    kv = p.plan.kv_tile;
+    kv = p.plan.kv_tile;  // the list bounds were checked when the work item was decoded
     ea = wk.e0[0];
     na = wk.n[0];
     eb = wk.e0[1];
@@ -337,10 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kt, kt_n;
         bool ha, hb;
         walk.next(kt, ha, hb);  // any_tiles: the union has a first tile
+        BFA_CHECK(kt >= 0 && kt * kTile < wk.k_len, p.plan.err);
         load_kv_tile<C::kPanels>(p, wk, &tmK, sK(0), bar(BQ), kt, wk.k_off + kt * kTile);
         int last_f[2] = {-1, -1};  // last step that filled F[0] / F[1]
         for (int j = 0;; ++j) {
           const bool have_next = walk.next(kt_n, ha, hb);
+          BFA_CHECK(!have_next || (kt_n >= 0 && kt_n * kTile < wk.k_len), p.plan.err);
           if (j >= 1 && !mbar_wait_fast(bar(BE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, cap, &abort_flag)) break;
           const uint32_t f = bar(BF + (j & 1));
           mbar_expect_tx(f, (have_next ? 2 : 1) * C::kTileBytes);

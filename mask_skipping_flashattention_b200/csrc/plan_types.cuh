@@ -20,7 +20,33 @@ enum DevErr : uint32_t {
   DEVERR_TIMEOUT = 1u,       // a bounded wait gave up
   DEVERR_BSR_RANGE = 2u,     // BSR offsets out of range / decreasing
   DEVERR_BSR_ORDER = 4u,     // BSR ids unsorted, duplicated or out of range
+  DEVERR_BOUNDS = 8u,        // checked build: an index left its array (the access was skipped)
+  DEVERR_GUARD = 16u,        // checked build: guard bytes after a plan array were overwritten
 };
+
+// Index checks of the checked build (compiled with -DBFA_CHECKED): an index
+// outside [0, n) sets DEVERR_BOUNDS in the plan's error word and is replaced by
+// 0, so that the access stays inside the array; no trap, no assert.  The normal
+// build compiles the index unchanged.
+#ifdef BFA_CHECKED
+__device__ __forceinline__ int64_t checked_index(int64_t i, int64_t n, uint32_t* err) {
+  if (i < 0 || i >= n) {
+    atomicOr(err, DEVERR_BOUNDS);
+    return 0;
+  }
+  return i;
+}
+#define BFA_IDX(i, n, err) (::bfa::checked_index((i), (n), (err)))
+#define BFA_CHECK(cond, err) \
+  do {                       \
+    if (!(cond)) atomicOr((err), ::bfa::DEVERR_BOUNDS); \
+  } while (0)
+#else
+#define BFA_IDX(i, n, err) (i)
+#define BFA_CHECK(cond, err) \
+  do {                       \
+  } while (0)
+#endif
 
 // One row group: a batch (batched plans), a sequence (varlen plans), a
 // (batch, kv head) pair (BSR plans) or the single shared group of a dense plan.
@@ -60,6 +86,9 @@ struct PlanDev {
   const uint32_t* kbits;     // padded k validity bits (block-id plans)
   const int32_t* terms;      // position terms (predicate plans), 6 ints each
   uint32_t* err;             // device error word
+  int64_t cap_tiles;         // entries of kv_tile / part (and of the class grid)
+  int64_t cap_fine;          // tiles of packed fine words behind `fine`
+  int64_t cap_qid, cap_kid, cap_kbits;  // entries of qid / qvalid, kid, kbits
   int32_t n_rows;
   int32_t n_pairs;
   int32_t n_groups;

@@ -833,6 +833,25 @@ cudaError_t launch_init_regular_groups(const GroupInfo& tmpl, int n_groups, int 
   return cudaGetLastError();
 }
 
+// Checked build: every guard region of a plan slab (offsets in `offs`) must
+// still hold the guard byte.
+__global__ void k_check_guards(const uint8_t* __restrict__ slab, const uint64_t* __restrict__ offs, int n,
+                               uint32_t guard_bytes, int guard_byte, uint32_t* err) {
+  for (int g = blockIdx.x; g < n; g += gridDim.x) {
+    const uint8_t* p = slab + offs[g];
+    for (uint32_t i = threadIdx.x; i < guard_bytes; i += blockDim.x)
+      if (p[i] != static_cast<uint8_t>(guard_byte)) atomicOr(err, DEVERR_GUARD);
+  }
+}
+
+cudaError_t launch_check_guards(const void* slab, const uint64_t* offs, int n, uint32_t guard_bytes, int guard_byte,
+                                uint32_t* err, cudaStream_t s) {
+  if (n <= 0 || slab == nullptr) return cudaSuccess;
+  k_check_guards<<<n < 64 ? n : 64, 64, 0, s>>>(static_cast<const uint8_t*>(slab), offs, n, guard_bytes, guard_byte,
+                                                err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dense_classify(const uint8_t* mask, int64_t ld, int Sq, int Sk, uint8_t* cls, uint32_t* fine,
                                   cudaStream_t s, GroupInfo* groups, const GroupInfo* group, int32_t* row_group,
                                   uint32_t* err, int32_t* max_width) {

@@ -22,7 +22,8 @@ __device__ __forceinline__ void row_mask_words(const PlanDev& plan, const Ctx& w
   const int ncols = wk.k_len - kt * kTile;  // in-range columns (may exceed 128)
   if (plan.mask_mode == MASK_BITS) {
     if (part >= 0) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(plan.fine + static_cast<int64_t>(part) * kFineWordsPerTile +
+      const int64_t fp = BFA_IDX(static_cast<int64_t>(part), plan.cap_fine, plan.err);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(plan.fine + fp * kFineWordsPerTile +
                                                            row * kWordsPerTileRow));
       am[0] = v.x; am[1] = v.y; am[2] = v.z; am[3] = v.w;
     } else {
@@ -31,11 +32,22 @@ __device__ __forceinline__ void row_mask_words(const PlanDev& plan, const Ctx& w
   } else if (plan.mask_mode == MASK_BLOCKID) {
     if (part >= 0) {
       // called by whole warps (the tile is the same for the warp's 32 rows)
-      const int32_t qb = plan.qid[wk.qid_off + qpos];
-      const bool qv = plan.qvalid[wk.qid_off + qpos] != 0;
-      const int32_t* kids = plan.kid + wk.kid_off + kt * kTile;
+      const int64_t qi = BFA_IDX(static_cast<int64_t>(wk.qid_off) + qpos, plan.cap_qid, plan.err);
+      const int32_t qb = plan.qid[qi];
+      const bool qv = plan.qvalid[qi] != 0;
+#ifdef BFA_CHECKED
+      const bool kin = kt >= 0 && wk.kid_off + (kt + 1) * kTile <= plan.cap_kid &&
+                       wk.kbit_off + (kt + 1) * kWordsPerTileRow <= plan.cap_kbits;
+      if (!kin) atomicOr(plan.err, DEVERR_BOUNDS);
+      const int64_t k0 = kin ? wk.kid_off + kt * kTile : 0;
+      const int64_t b0 = kin ? wk.kbit_off + kt * kWordsPerTileRow : 0;
+#else
+      const int64_t k0 = wk.kid_off + kt * kTile;
+      const int64_t b0 = wk.kbit_off + kt * kWordsPerTileRow;
+#endif
+      const int32_t* kids = plan.kid + k0;
       const int4* kb4 = reinterpret_cast<const int4*>(kids);
-      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(plan.kbits + wk.kbit_off + kt * kWordsPerTileRow));
+      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(plan.kbits + b0));
       const uint32_t kvw[4] = {kv.x, kv.y, kv.z, kv.w};
       // Key ids non-decreasing across the tile (the usual form: cross columns at
       // INT32_MIN, then running block counts) make {j : k_blk[j] <= q_blk} a prefix

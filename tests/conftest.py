@@ -16,3 +16,29 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(autouse=True)
+def _checked_build_plan_status():
+    """Under the bounds-checked library (BFA_LIBRARY=checked), every plan a test
+    creates is verified after the test: bfa_plan_device_status checks the guard
+    bytes around its arrays and the kernels' index-check flag (BFA_ERR_BOUNDS)."""
+    if os.environ.get("BFA_LIBRARY") != "checked":
+        yield
+        return
+    import mask_skipping_flashattention_b200 as bfa
+    made = []
+    orig = bfa.Plan.__init__
+
+    def init(self, *a, **k):
+        orig(self, *a, **k)
+        made.append(self)
+
+    bfa.Plan.__init__ = init
+    try:
+        yield
+    finally:
+        bfa.Plan.__init__ = orig
+    for P in made:
+        if P._h is not None:
+            P.device_status()

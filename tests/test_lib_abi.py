@@ -27,6 +27,17 @@ def test_library_exports_every_declared_symbol():
     assert set(_declared()) == set(_lib.SIGNATURES), "binding signatures out of sync with bfa.h"
 
 
+def test_checked_library_exports_the_same_symbols():
+    """The bounds-checked build (libbfa_checked.so) is a drop-in twin of libbfa.so."""
+    from mask_skipping_flashattention_b200 import _lib
+    path = os.path.join(os.path.dirname(_lib.LIB_PATH), "libbfa_checked.so")
+    lib = ctypes.CDLL(path)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    lib.bfa_version.restype = ctypes.c_char_p
+    assert b"checked" in lib.bfa_version()
+
+
 def test_library_reports_no_device_without_a_gpu():
     import torch
     import mask_skipping_flashattention_b200 as bfa
