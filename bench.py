@@ -99,7 +99,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
                  "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -531,6 +531,8 @@ def run_sweep(args):
     P = bfa.plan_bsr(cuda(ip), cuda(ix), w["S"], w["S"], w["block"], w["block"], causal=True)
     measure("bsr_16384", P, w["q"].cuda(), w["k"].cuda(), w["v"].cuda(), per_group * (w["H"] // w["Hkv"]), w["D"],
             "BSR, causal inside blocks")
+    # the union workload's q, k, v are the BSR workload's (the same configuration,
+    # shapes and seeds: workloads.qkv(5, ...)), so the tensors above are reused
     u = workloads.union_16384(with_qkv=False)
     measure("union_16384", bfa.plan_dense(u["mask"].cuda()), w["q"].cuda(), w["k"].cuda(), w["v"].cuda(),
             float(u["mask"].sum()) * w["B"] * w["H"], w["D"], "dense")
