@@ -8,7 +8,8 @@ either as ``BFA_ERR_BOUNDS``.  It stands in for a memory checker, which is not
 available here.  This test runs a set of the small forward, backward and plan
 parity tests in a subprocess that loads the checked build; the tests' conftest
 then verifies every plan they create after each test.  They must all pass (the
-outputs still match the oracle) with every plan's status clean.
+outputs still match the oracle) with every plan's status clean, at the small
+sizes and on the full-size workloads, the bench's causal 8192 launch included.
 """
 
 import os
@@ -47,6 +48,14 @@ CASES = [
     "tests/test_gpu_bwd.py::test_predicate_terms",
     "tests/test_gpu_bwd.py::test_general_block_sparse_with_validity",
     "tests/test_gpu_bwd.py::test_varlen_causal_packed",
+    # full-size workloads, the bench's own launch among them
+    "tests/test_gpu_plan.py::test_dense_plan_causal_8192",
+    "tests/test_gpu_plan.py::test_bsr_plan_workload_full_size_every_group",
+    "tests/test_gpu_fwd.py::test_causal_8192_full_size_sampled",
+    "tests/test_gpu_fwd.py::test_varlen_workload",
+    "tests/test_gpu_fwd.py::test_bsr_workload_sampled",
+    "tests/test_gpu_fwd.py::test_union_workload_sampled",
+    "tests/test_gpu_bwd.py::test_bsr_workload_one_kv_group",
 ]
 
 
