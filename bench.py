@@ -428,7 +428,7 @@ def run_bfa(args, rank, world, local_rank):
         "bwd": {"ms_per_step": bwd_ms, "tflops": 2.5 * flops / (bwd_ms * 1e-3) / 1e12,
                 "frac": 2.5 * flops / (bwd_ms * 1e-3) / 1e12 / peak,
                 "flops_counted": "2.5 x the forward's attended-pair flops (dV, dP, dQ, dK and the recomputed S)",
-                "kernels": "k_bwd_prep, k_bwd_dq, k_bwd_dkdv", "steps": bwd_steps},
+                "kernels": "k_bwd_prep, k_bwd_fused, k_bwd_dq_store (fused pass, D = 128)", "steps": bwd_steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
     }

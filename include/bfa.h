@@ -253,9 +253,16 @@ bfa_status bfa_fwd(const bfa_plan* plan, const void* q, const void* k, const voi
  *   GQA dk and dv sum over the query heads of each kv head.  All strides
  *   {batch, token, head} in elements, multiples of 8; bases 16-byte aligned.
  * The first call on a plan builds its transposed lists (bfa_plan_export_cols) on
- * `stream`; a per-call workspace of 8 bytes per (replica, query-tile row) comes
- * from the plan's stream-ordered pool.  Asynchronous; a device-side timeout is
- * reported by bfa_plan_device_status().  Paged caches are not accepted here.
+ * `stream`; a per-call workspace comes from the plan's stream-ordered pool: 8
+ * bytes per (replica, query row of the plan's tiles), plus 4 * D bytes for the
+ * fused pass.  Asynchronous; a device-side timeout is reported by
+ * bfa_plan_device_status().  Paged caches are not accepted here.
+ * Forms: D = 128 runs one fused pass over the key-tile columns (S and dP made
+ * once per pair; dQ summed across key tiles by fp32 reductions into the
+ * workspace, then scaled into dq), whose dq is not bitwise reproducible from run
+ * to run (the order of the fp32 sums varies); dk and dv are.  D = 64, and every D
+ * after bfa_set_bwd_deterministic(1), run the two passes (dK/dV over key-tile
+ * columns, dQ over query-tile rows), bitwise reproducible.
  */
 bfa_status bfa_bwd(const bfa_plan* plan, const void* q, const void* k, const void* v, const void* out,
                    const void* dout, const float* lse, const int64_t q_strides[3], const int64_t k_strides[3],
@@ -365,6 +372,11 @@ void bfa_plan_destroy(bfa_plan* plan);
 #define BFA_WAIT_NS_MIN 1000ull
 #define BFA_WAIT_NS_MAX 60000000000ull
 void bfa_set_wait_timeout_ns(uint64_t ns);
+
+/* Backward form for calls made after this one (process-wide): on != 0 makes
+ * bfa_bwd use the two-pass form for every head dim, so that its results are
+ * bitwise reproducible; 0 (the default) lets D = 128 use the fused pass. */
+void bfa_set_bwd_deterministic(int on);
 
 /* Launch a one-thread-block kernel that waits, with the current bound, on a
  * barrier phase that nothing completes, and synchronise.  Returns

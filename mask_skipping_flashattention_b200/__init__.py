@@ -26,7 +26,7 @@ from ._lib import BfaError, PlanInfo
 __all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_predicate", "plan_bsr", "plan_block_bits",
            "fwd", "bwd", "fwd_paged",
            "make_att_block_ids",
-           "is_available", "load_error", "set_wait_timeout_ns", "selftest_wait_timeout", "library_path"]
+           "is_available", "load_error", "set_wait_timeout_ns", "set_bwd_deterministic", "selftest_wait_timeout", "library_path"]
 
 TILE = 128
 KIND_NAMES = {1: "dense", 2: "blockids", 3: "positional", 4: "bsr", 5: "predicate"}
@@ -69,6 +69,11 @@ def load_error():
 
 def set_wait_timeout_ns(ns):
     _L.bfa_set_wait_timeout_ns(int(ns))
+
+
+def set_bwd_deterministic(on=True):
+    """Two-pass backward for every head dim (bitwise reproducible) when ``on``."""
+    _L.bfa_set_bwd_deterministic(1 if on else 0)
 
 
 def selftest_wait_timeout(stream=None):

@@ -66,6 +66,7 @@ SIGNATURES = {
     "bfa_plan_device_status": (ctypes.c_int, [c_void, c_void]),
     "bfa_plan_destroy": (None, [c_void]),
     "bfa_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
+    "bfa_set_bwd_deterministic": (None, [ctypes.c_int]),
     "bfa_selftest_wait_timeout": (ctypes.c_int, [c_void]),
     "bfa_plan_dense_noalloc": (ctypes.c_int, [c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int, c_void, c_void,
                                               c_void, c_void, c_void, c_void, c_void]),

@@ -133,6 +133,7 @@ namespace {
 
 thread_local std::string g_err;
 uint64_t g_wait_ns = 1000000000ull;
+int g_bwd_deterministic = 0;  // bfa_set_bwd_deterministic
 
 // Device address of the allocation-free planner's scratch array, per device
 // (looked up on that entry point's first call on a device; see below).
@@ -511,6 +512,8 @@ BFA_API void bfa_set_wait_timeout_ns(uint64_t ns) {
   if (ns == 0) ns = 1000000000ull;
   g_wait_ns = std::min<uint64_t>(std::max<uint64_t>(ns, BFA_WAIT_NS_MIN), BFA_WAIT_NS_MAX);
 }
+
+BFA_API void bfa_set_bwd_deterministic(int on) { g_bwd_deterministic = on ? 1 : 0; }
 
 BFA_API bfa_status bfa_make_block_ids(const uint8_t* pad_masks, const uint8_t* att_masks, int B, int N, int n_cross,
                                       const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
@@ -1165,6 +1168,10 @@ bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const
   p.n_cols = n_cols;
   p.wait_ns = g_wait_ns;
   const int64_t ws_rows = static_cast<int64_t>(p.rep) * P->n_rows * kTile;
+  // D = 128 runs the fused pass, which also needs the fp32 dQ sums (D floats a row),
+  // unless reproducible sums were asked for
+  const bool fused = D == 128 && !g_bwd_deterministic;
+  const int64_t ws_floats = ws_rows * (2 + (fused ? D : 0));
   void* ws = nullptr;
   auto cleanup = [&]() {
     if (ws) cudaFreeAsync(ws, st);
@@ -1172,18 +1179,24 @@ bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const
   if (ws_rows > 0) {
     cudaMemPool_t pool;
     BFA_CUDA(plan_pool(&pool), "plan memory pool");
-    cudaError_t e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(ws_rows) * 2 * sizeof(float), pool, st);
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(ws_floats) * sizeof(float), pool, st);
     if (e != cudaSuccess) {
       ws = nullptr;
-      return fail(BFA_ERR_CAPACITY, "backward workspace of %lld bytes: %s", (long long)(ws_rows * 8),
+      return fail(BFA_ERR_CAPACITY, "backward workspace of %lld bytes: %s", (long long)(ws_floats * 4),
                   cudaGetErrorString(e));
     }
     p.ws_lse2 = static_cast<float*>(ws);
     p.ws_d = p.ws_lse2 + ws_rows;
+    p.dq_acc = fused ? p.ws_d + ws_rows : nullptr;
   }
   BFA_CUDA(launch_bwd_prep(p, st), "backward preprocess kernel");
-  BFA_CUDA(launch_bwd_dq(D, tq, tdo, tk, tv, p, static_cast<int64_t>(P->n_rows) * p.rep, st), "dQ kernel");
-  BFA_CUDA(launch_bwd_dkdv(D, tk, tv, tq, tdo, p, static_cast<int64_t>(n_cols) * p.rep_kv, st), "dK/dV kernel");
+  if (fused) {
+    BFA_CUDA(launch_bwd_fused(tk, tv, tq, tdo, p, static_cast<int64_t>(n_cols) * p.rep_kv, st), "fused backward kernel");
+    BFA_CUDA(launch_bwd_dq_store(p, st), "dQ store kernel");
+  } else {
+    BFA_CUDA(launch_bwd_dq(D, tq, tdo, tk, tv, p, static_cast<int64_t>(P->n_rows) * p.rep, st), "dQ kernel");
+    BFA_CUDA(launch_bwd_dkdv(D, tk, tv, tq, tdo, p, static_cast<int64_t>(n_cols) * p.rep_kv, st), "dK/dV kernel");
+  }
   cleanup();
   return BFA_OK;
 }

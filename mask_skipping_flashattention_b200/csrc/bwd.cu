@@ -216,6 +216,11 @@ __global__ void __launch_bounds__(128) k_bwd_prep(const BwdParams p) {
   const int64_t wi = (static_cast<int64_t>(j) * p.plan.n_rows + r) * kTile + threadIdx.x;
   p.ws_lse2[wi] = -lse2;  // stored negated: the tile kernels add them
   p.ws_d[wi] = -dval;
+  if (p.dq_acc) {  // the fused pass sums into this tile's dQ rows (contiguous, D floats a row)
+    float4* z = reinterpret_cast<float4*>(p.dq_acc + (wi - threadIdx.x) * D);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < kTile * D / 4; i += 128) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -787,10 +792,446 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
+// fused pass (D = 128): one CTA per (key-tile column, kv replica), walking the
+// column's query-tile list as k_bwd_dkdv does, and making dQ from the same dS:
+// dQ^T = K^T dS^T runs into the dP^T columns once dK has read dS^T there, and a
+// fourth warpgroup reads it out and sums it into an fp32 workspace.  Each
+// (query tile, key tile) pair then costs five 128 x 128 x 128 products instead
+// of the two passes' seven (S and dP are made once).
+// ----------------------------------------------------------------------------
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
+// issuer, warps 2..3 idle, warps 4..7 the P^T / dS^T rows (one key per thread;
+// dS^T also goes to shared memory as the B operand of dQ^T), warps 8..15 the dQ
+// rows (one head dimension per thread, the TMEM lanes of dQ^T; warps 8..11 take
+// queries [0, 64) and warps 12..15 queries [64, 128): one SM needs eight warps
+// of reductions in flight to reach the rate L2 accepts them at).
+// Shared memory (1024-aligned, nothing static): K, V, Q[2], dO[2], dS^T, the
+// query vectors of two steps, then the barriers and the work item.
+// TMEM (512 columns): S^T [0,128) (P^T over [0,64)), dP^T [128,256) (dS^T over
+// [128,192), then dQ^T), dV [256,384), dK [384,512).
+constexpr int kFusedThreads = 512;
+constexpr int kFusedRegsLaunch = 128;
+constexpr uint32_t kFusedRegsWG0 = 120, kFusedRegsRows = 216, kFusedRegsDq = 88;
+static_assert(128 * (kFusedRegsWG0 + kFusedRegsRows + 2 * kFusedRegsDq) == kFusedThreads * kFusedRegsLaunch,
+              "register split");
+
+struct FCfg {
+  static constexpr int D = 128;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kOffDS = 6 * kTileBytes;
+  static constexpr int kOffVec = 7 * kTileBytes;
+  static constexpr int kOffCtl = kOffVec + kBwdStages * BCfg<D>::kVecBytes;
+  static constexpr int kSmemBytes = kOffCtl + 512;
+  static constexpr uint32_t kIdescQT = idesc_bf16_f32_mn(128, 128);  // A = K^T and B = dS^T, both MN-major
+};
+static_assert(FCfg::kSmemBytes <= 232448, "fused pass shared memory");
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    k_bwd_fused(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
+  constexpr int D = FCfg::D;
+  using C = BCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_fused[];
+  // the swizzled tiles need 1024-byte alignment, which the declaration asks for;
+  // a block that does not get it reports and does nothing
+  if (smem_u32(smem_fused) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.plan.err, DEVERR_BOUNDS);
+    return;
+  }
+  uint8_t* const sK = smem_fused;
+  uint8_t* const sV = smem_fused + C::kTileBytes;
+  uint8_t* const sQ0 = smem_fused + 2 * C::kTileBytes;  // + 2 st tiles: Q(st), dO(st)
+  uint8_t* const sdS = smem_fused + FCfg::kOffDS;
+  float* const sVec0 = reinterpret_cast<float*>(smem_fused + FCfg::kOffVec);
+  // BKV: K and V.  BF / BE [2]: Q, dO and the query vectors of a step full /
+  // free.  BS1 / BS2: S^T / dP^T ready.  BP1 [4]: P^T of one 32-query chunk
+  // written, BP2: dS^T written (TMEM and shared memory; 4 warps each).  BQ: dQ^T
+  // ready, BQR: dQ^T read out (8 warps).  BO: every product done.
+  enum { BKV = 0, BF = 1, BE = 3, BS1 = 5, BS2 = 6, BP1 = 7, BP2 = 11, BQ = 12, BQR = 13, BO = 14, BDONE = 15, NBAR = 16 };
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(smem_fused + FCfg::kOffCtl);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
+  int* const abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  KvWork* const wk_s = reinterpret_cast<KvWork*>(bars + NBAR + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto sQ = [&](int st) { return sQ0 + (2 * st) * C::kTileBytes; };
+  auto sdO = [&](int st) { return sQ0 + (2 * st + 1) * C::kTileBytes; };
+  auto sVec = [&](int st) { return sVec0 + st * 2 * kTile; };  // [lse2 x 128][D x 128]
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i >= BP1 && i <= BP2) ? 4 : (i == BQR ? 8 : 1));
+    fence_barrier_init();
+    int i, jk;
+    chunked_decode(blockIdx.x, p.n_cols, p.rep_kv, p.kv_chunk, i, jk);
+    uint32_t* const err = p.plan.err;
+    (void)err;
+    const int c = static_cast<int>(BFA_IDX(p.col_order[BFA_IDX(i, p.n_cols, err)], p.n_cols, err));
+    const int grp = static_cast<int>(BFA_IDX(p.col_group[c], p.plan.n_groups, err));
+    KvWork w;
+    w.g = p.plan.groups[grp];
+    w.kt = c - p.col0[grp];
+    w.e0 = p.col_ptr[c];
+    w.nq = p.col_ptr[c + 1] - w.e0;
+#ifdef BFA_CHECKED
+    if (!(w.nq >= 0 && w.nq <= w.g.nqt && w.e0 >= 0 && w.e0 + w.nq <= p.plan.cap_tiles && w.kt >= 0 &&
+          w.kt < w.g.nkt && jk >= 0 && jk < p.rep_kv)) {
+      atomicOr(err, DEVERR_BOUNDS);
+      w.e0 = 0;
+      w.nq = 0;
+    }
+#endif
+    w.nh = p.H / p.Hkv;
+    kv_replica_bh(p, w.g, jk, w.b, w.hk);
+    w.steps = w.nq * w.nh;
+    *wk_s = w;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const KvWork& wk = *wk_s;
+  const uint64_t cap = p.wait_ns;
+  const int steps = wk.steps;
+  auto step_head = [&](int s) { return wk.hk * wk.nh + s / wk.nq; };
+  auto step_entry = [&](int s) { return wk.e0 + s % wk.nq; };
+
+  if (warp < 4) {
+    regs_dec<kFusedRegsWG0>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0 && steps > 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmdO);
+        const int ks = wk.g.k_off + wk.kt * kTile;
+        mbar_expect_tx(bar(BKV), 2 * C::kTileBytes);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_4d(smem_u32(sK + pn * 16384), &tmK, bar(BKV), pn * 64, wk.hk, ks, wk.b);
+          tma_load_4d(smem_u32(sV + pn * 16384), &tmV, bar(BKV), pn * 64, wk.hk, ks, wk.b);
+        }
+        int last[kBwdStages] = {-1, -1};
+        for (int s = 0; s < steps; ++s) {
+          const int st = s & 1;
+          if (s >= kBwdStages && !mbar_wait_fast(bar(BE + st), ((s >> 1) - 1) & 1, cap, abort_flag)) break;
+          const int h = step_head(s);
+          const int qt = p.q_tile[step_entry(s)];
+          BFA_CHECK(qt >= 0 && qt < wk.g.nqt, p.plan.err);
+          const int r = wk.g.row0 + qt;
+          const int64_t wi = (static_cast<int64_t>(replica_of(p, wk.g, wk.b, h)) * p.plan.n_rows + r) * kTile;
+          BFA_CHECK(wi >= 0 && wi + kTile <= static_cast<int64_t>(p.rep) * p.plan.n_rows * kTile, p.plan.err);
+          const uint32_t f = bar(BF + st);
+          mbar_expect_tx(f, 2 * C::kTileBytes + C::kVecBytes);
+          const int qs = wk.g.q_off + qt * kTile;
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn) {
+            tma_load_4d(smem_u32(sQ(st) + pn * 16384), &tmQ, f, pn * 64, h, qs, wk.b);
+            tma_load_4d(smem_u32(sdO(st) + pn * 16384), &tmdO, f, pn * 64, h, qs, wk.b);
+          }
+          bulk_load(smem_u32(sVec(st)), p.ws_lse2 + wi, kTile * 4, f);
+          bulk_load(smem_u32(sVec(st) + kTile), p.ws_d + wi, kTile * 4, f);
+          last[st] = s;
+        }
+        mbar_drain(bar(BKV), 0, abort_flag);
+        for (int st = 0; st < kBwdStages; ++st)
+          if (last[st] >= 0) mbar_drain(bar(BF + st), (last[st] >> 1) & 1, abort_flag);
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      // Pipe order: dV(s), S^T(s+1), dK(s), dQ^T(s), dP^T(s+1), dV(s+1), ...
+      // dQ^T(s) goes over dS^T(s) once dK(s) is issued; dP^T(s+1) waits until
+      // the dQ warps hold dQ^T(s) in registers.
+      if (lane == 0 && steps > 0) {
+        const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+        bool ok = mbar_wait_fast(bar(BKV), 0, cap, abort_flag);
+        if (ok) ok = mbar_wait_fast(bar(BF), 0, cap, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_nn<D>(tS, sK, sQ(0));  // S^T = K Q^T
+          umma_commit(bar(BS1));
+          issue_nn<D>(tdP, sV, sdO(0));  // dP^T = V dO^T
+          umma_commit(bar(BS2));
+        }
+        for (int s = 0; ok && s < steps; ++s) {
+          const int st = s & 1, st1 = st ^ 1;
+          // dV += P^T dO, chunk by chunk as the rows write P^T
+          for (int cc = 0; cc < 4; ++cc) {
+            if (!mbar_wait_fast(bar(BP1 + cc), s & 1, cap, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ddo = mn_desc(sdO(st));
+#pragma unroll
+            for (int kk = 2 * cc; kk < 2 * cc + 2; ++kk)
+              umma_ts(tdV, tS + kk * 8, ddo + kk * (2048 >> 4), C::kIdescD, (s > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (!ok) break;
+          if (s + 1 < steps) {
+            if (!mbar_wait_fast(bar(BF + st1), ((s + 1) >> 1) & 1, cap, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_nn<D>(tS, sK, sQ(st1));
+            umma_commit(bar(BS1));
+          }
+          // dK += dS^T Q, then dQ^T = K^T dS^T (both operands MN-major in shared memory)
+          if (!mbar_wait_fast(bar(BP2), s & 1, cap, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t dq = mn_desc(sQ(st));
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tdK, tdP + kk * 8, dq + kk * (2048 >> 4), C::kIdescD, (s > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t dkt = mn_desc(sK), dds = mn_desc(sdS);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ss(tdP, dkt + kk * (2048 >> 4), dds + kk * (2048 >> 4), FCfg::kIdescQT, kk > 0 ? 1u : 0u);
+          umma_commit(bar(BQ));
+          umma_commit(bar(BE + st));
+          if (s + 1 < steps) {
+            if (!mbar_wait_fast(bar(BQR), s & 1, cap, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_nn<D>(tdP, sV, sdO(st1));
+            umma_commit(bar(BS2));
+          }
+        }
+        if (ok) umma_commit(bar(BO));
+        umma_commit(bar(BDONE));
+        mbar_drain(bar(BDONE), 0, abort_flag);
+      }
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P^T, dS^T rows (one key per thread)
+    regs_inc<kFusedRegsRows>();
+    const int quarter = warp & 3;
+    const int krow = quarter * 32 + lane;
+    const int kpos = wk.kt * kTile + krow;
+    const uint32_t tLane = tmem_addr(tmem, quarter * 32, 0);
+    // row krow of the dS^T tile with its swizzle folded in: the row starts on a
+    // 128-byte boundary, so chunk c16 of the row sits at (row ^ (c16 << 4))
+    const uint32_t sdS_row = (smem_u32(sdS) + krow * 128) | ((krow & 7) << 4);
+    const GroupCtx ctx = group_ctx(wk.g);
+    const float c = p.scale_log2;
+    const uint64_t c2 = f2_pack(c, c);
+    // Key rows past the group's keys hold other tokens (the next sequence of a
+    // packed batch); their dS^T must be 0 here, since dQ^T sums over every key
+    // row of the tile.  A tile that runs past the keys is masked on every step.
+    const bool kedge = (wk.kt + 1) * kTile > wk.g.k_len;
+    const bool kout = kpos >= wk.g.k_len;
+    bool ok = true;
+    for (int s = 0; s < steps; ++s) {
+      const int st = s & 1;
+      const int e = step_entry(s);
+      const int qt = p.q_tile[e], part = p.tpart[e];
+      BFA_CHECK(qt >= 0 && qt < wk.g.nqt, p.plan.err);
+      uint32_t am[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      const bool masked = part >= 0 || (qt + 1) * kTile > wk.g.q_len || kedge;
+      if (masked) {
+        col_mask_words(p.plan, ctx, kpos, krow, qt, part, am);
+        if (kout) am[0] = am[1] = am[2] = am[3] = 0u;
+      }
+      const bool gv = mbar_wait(bar(BF + st), (s >> 1) & 1, cap, abort_flag);
+      const bool gs = gv && mbar_wait(bar(BS1), s & 1, cap, abort_flag);
+      if (__any_sync(0xffffffffu, !gs)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sLse = smem_u32(sVec(st)), sDv = smem_u32(sVec(st) + kTile);
+      // phase 1: P^T = 2^(scale log2(e) S^T - LSE log2(e)), kept in fp32 for
+      // phase 2 and written as bf16 over S^T, 32 queries at a time
+      uint64_t pv[64];
+      {
+        uint32_t sA[32], sB[32];
+        tmem_ld_32x32b_x32(tLane, sA);
+        tmem_wait_ld();
+        reg_fence(sA);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t(&sv)[32] = (cc & 1) ? sB : sA;
+          if (cc + 1 < 4) tmem_ld_32x32b_x32(tLane + (cc + 1) * 32, (cc & 1) ? sA : sB);
+          if (masked) {
+            const uint32_t bits = am[cc];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (!((bits >> j) & 1u)) sv[j] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pkp[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 L = ld_shared_f4(sLse + (cc * 32 + q4 * 4) * 4);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int col = q4 * 4 + 2 * h2;
+              const float s0 = __uint_as_float(sv[col]), s1 = __uint_as_float(sv[col + 1]);
+              const uint64_t nl = h2 ? f2_pack(L.z, L.w) : f2_pack(L.x, L.y);
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(s0, s1), c2, nl), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              pv[cc * 16 + 2 * q4 + h2] = f2_pack(p0, p1);
+              pkp[2 * q4 + h2] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st_32x32b_x16(tLane + cc * 16, pkp);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BP1 + cc));
+          if (cc + 1 < 4) {
+            tmem_wait_ld();
+            reg_fence((cc & 1) ? sA : sB);
+          }
+        }
+      }
+      // phase 2: dS^T = P^T * (dP^T - D), as bf16 over dP^T (A operand of dK) and
+      // into shared memory (B operand of dQ^T: row krow, queries contiguous, in
+      // the 128-byte swizzled layout of a tile); the buffer is free: dQ^T of the
+      // previous step was done before dP^T of this one was issued
+      const bool gd = mbar_wait(bar(BS2), s & 1, cap, abort_flag);
+      if (__any_sync(0xffffffffu, !gd)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t dA[32], dB[32];
+        tmem_ld_32x32b_x32(tLane + 128, dA);
+        tmem_wait_ld();
+        reg_fence(dA);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t(&dp)[32] = (cc & 1) ? dB : dA;
+          if (cc + 1 < 4) tmem_ld_32x32b_x32(tLane + 128 + (cc + 1) * 32, (cc & 1) ? dA : dB);
+          uint32_t pks[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 Dv = ld_shared_f4(sDv + (cc * 32 + q4 * 4) * 4);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int col = q4 * 4 + 2 * h2;
+              const uint64_t nd = h2 ? f2_pack(Dv.z, Dv.w) : f2_pack(Dv.x, Dv.y);
+              float d0, d1;
+              f2_unpack(f2_mul(pv[cc * 16 + 2 * q4 + h2],
+                               f2_add(f2_pack(__uint_as_float(dp[col]), __uint_as_float(dp[col + 1])), nd)),
+                        d0, d1);
+              pks[2 * q4 + h2] = pack_bf16x2(d0, d1);
+            }
+          }
+          tmem_st_32x32b_x16(tLane + 128 + cc * 16, pks);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c16 = (cc & 1) * 4 + j;  // 16-byte chunk of the row inside its 64-query panel
+            st_shared_v4((sdS_row ^ (c16 << 4)) + (cc >> 1) * 16384, pks[4 * j], pks[4 * j + 1], pks[4 * j + 2],
+                         pks[4 * j + 3]);
+          }
+          if (cc + 1 < 4) {
+            tmem_wait_ld();
+            reg_fence((cc & 1) ? dA : dB);
+          }
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BP2));
+    }
+    bool done = ok;
+    if (ok && steps > 0) {
+      const bool got = mbar_wait(bar(BO), 0, cap, abort_flag);
+      done = !__any_sync(0xffffffffu, !got);
+    }
+    tc_fence_after();
+    if (done) {
+      const bool store = kpos < wk.g.k_len;
+      const int64_t tok = static_cast<int64_t>(wk.g.k_off) + kpos;
+      __nv_bfloat16* dvp =
+          p.dv + static_cast<int64_t>(wk.b) * p.dv_sb + tok * p.dv_ss + static_cast<int64_t>(wk.hk) * p.dv_sh;
+      __nv_bfloat16* dkp =
+          p.dk + static_cast<int64_t>(wk.b) * p.dk_sb + tok * p.dk_ss + static_cast<int64_t>(wk.hk) * p.dk_sh;
+      store_row<D>(tLane + 256, steps > 0, 1.f, dvp, store);
+      store_row<D>(tLane + 256 + D, steps > 0, p.scale, dkp, store);
+    }
+  } else {
+    // ------------------------------------------------------------ dQ rows (one head dimension per thread)
+    // A warp reads its 64 queries of dQ^T(s) out of TMEM, releases the columns
+    // to dP^T(s+1), then sums them into the workspace: for each query, the 32
+    // lanes add 32 consecutive floats (one 128-byte line).
+    regs_dec<kFusedRegsDq>();
+    const int quarter = warp & 3;
+    const int q0 = warp >= 12 ? 64 : 0;
+    const int dim = quarter * 32 + lane;
+    const uint32_t tQT = tmem_addr(tmem + 128 + q0, quarter * 32, 0);
+    for (int s = 0; s < steps; ++s) {
+      const int h = step_head(s);
+      const int qt = p.q_tile[step_entry(s)];
+      BFA_CHECK(qt >= 0 && qt < wk.g.nqt, p.plan.err);
+      const int64_t wi =
+          (static_cast<int64_t>(replica_of(p, wk.g, wk.b, h)) * p.plan.n_rows + wk.g.row0 + qt) * kTile;
+      BFA_CHECK(wi >= 0 && wi + kTile <= static_cast<int64_t>(p.rep) * p.plan.n_rows * kTile, p.plan.err);
+      const int nvalid = min(kTile, wk.g.q_len - qt * kTile) - q0;  // rows past the sequence stay 0
+      float* const dst = p.dq_acc + (wi + q0) * D + dim;
+      const bool got = mbar_wait(bar(BQ), s & 1, cap, abort_flag);
+      if (__any_sync(0xffffffffu, !got)) break;
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_32x32b_x32(tQT, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld_32x32b_x32(tQT + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      reg_fence(v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BQR));
+#ifdef BFA_CHECKED
+      if (!(wi >= 0 && wi + kTile <= static_cast<int64_t>(p.rep) * p.plan.n_rows * kTile)) continue;
+#endif
+      if (nvalid >= 64) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) red_add_f32(dst + q * D, __uint_as_float(v[q]));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 64; ++q)
+          if (q < nvalid) red_add_f32(dst + q * D, __uint_as_float(v[q]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*static_cast<volatile int*>(abort_flag) && threadIdx.x == 0) atomicOr(p.plan.err, DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// dQ = scale * (the fused pass's fp32 sums) as bf16, per (replica, plan row):
+// a warp converts 32 rows, one 512-byte row per step (4 floats a lane)
+__global__ void __launch_bounds__(128) k_bwd_dq_store(const BwdParams p) {
+  constexpr int D = FCfg::D;
+  const int64_t blk = blockIdx.x;
+  const int r = static_cast<int>(blk % p.plan.n_rows);
+  const int j = static_cast<int>(blk / p.plan.n_rows);
+  const GroupInfo g = p.plan.groups[p.plan.row_group[r]];
+  int b, h;
+  replica_bh(p, g, j, b, h);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t wi = (static_cast<int64_t>(j) * p.plan.n_rows + r) * kTile;
+  __nv_bfloat16* const base = p.dq + static_cast<int64_t>(b) * p.dq_sb + static_cast<int64_t>(h) * p.dq_sh;
+#pragma unroll 4
+  for (int i = 0; i < 32; ++i) {
+    const int row = warp * 32 + i;
+    const int qpos = (r - g.row0) * kTile + row;
+    if (qpos >= g.q_len) break;
+    const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + (wi + row) * D + lane * 4);
+    const int64_t tok = static_cast<int64_t>(g.q_off) + qpos;
+    uint2 o;
+    o.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
+    o.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
+    *reinterpret_cast<uint2*>(base + tok * p.dq_ss + lane * 4) = o;
+  }
+}
+
+// ----------------------------------------------------------------------------
 // launchers (host)
 // ----------------------------------------------------------------------------
 int bwd_smem_bytes(int D) {
-  return D == 64 ? max(BCfg<64>::kSmemBytes, BCfg<64>::kDqSmemBytes) : max(BCfg<128>::kSmemBytes, BCfg<128>::kDqSmemBytes);
+  return D == 64 ? max(BCfg<64>::kSmemBytes, BCfg<64>::kDqSmemBytes) : FCfg::kSmemBytes;
 }
 
 cudaError_t launch_bwd_prep(const BwdParams& p, cudaStream_t s) {
@@ -820,6 +1261,31 @@ cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tdo, 
     if (ready != cudaSuccess) return ready;
     k_bwd_dq<128><<<static_cast<unsigned>(n_work), kDqThreads, BCfg<128>::kDqSmemBytes, s>>>(tq, tdo, tk, tv, p);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_fused(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                             const CUtensorMap& tdo, const BwdParams& p, int64_t n_work, cudaStream_t s) {
+  if (n_work <= 0) return cudaSuccess;
+  if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  // the setmaxnreg split is only safe with exactly kFusedRegsLaunch registers a thread
+  static cudaError_t ready = []() {
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, k_bwd_fused);
+    if (e != cudaSuccess) return e;
+    if (a.numRegs != kFusedRegsLaunch) return cudaErrorInvalidKernelImage;
+    return bwd_prepare(k_bwd_fused, FCfg::kSmemBytes);
+  }();
+  if (ready != cudaSuccess) return ready;
+  k_bwd_fused<<<static_cast<unsigned>(n_work), kFusedThreads, FCfg::kSmemBytes, s>>>(tk, tv, tq, tdo, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dq_store(const BwdParams& p, cudaStream_t s) {
+  const int64_t blocks = static_cast<int64_t>(p.rep) * p.plan.n_rows;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  k_bwd_dq_store<<<static_cast<unsigned>(blocks), 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -36,6 +36,10 @@ struct BwdParams {
   // -D = -dO . O, with rows past a sequence (and rows that attend nothing) 0
   float* ws_lse2;
   float* ws_d;
+  // fused pass (D = 128): fp32 dQ / scale per (replica, plan row, row of the
+  // tile), D values a row; zeroed by the preprocess, summed into by every key
+  // tile of the row's list, then scaled into dq.  nullptr for the two-pass form.
+  float* dq_acc;
   // transposed lists of the plan
   const int32_t* col0;
   const int32_t* col_group;
@@ -52,6 +56,9 @@ cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tdo, 
                           const CUtensorMap& tv, const BwdParams& p, int64_t n_work, cudaStream_t s);
 cudaError_t launch_bwd_dkdv(int D, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                             const CUtensorMap& tdo, const BwdParams& p, int64_t n_work, cudaStream_t s);
+cudaError_t launch_bwd_fused(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                             const CUtensorMap& tdo, const BwdParams& p, int64_t n_work, cudaStream_t s);
+cudaError_t launch_bwd_dq_store(const BwdParams& p, cudaStream_t s);
 int bwd_smem_bytes(int D);
 
 }  // namespace bfa

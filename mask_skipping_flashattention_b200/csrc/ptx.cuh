@@ -295,6 +295,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
          ((M >> 4) << 24);
 }
 
+// the same with the A operand MN-major too (A stored M-contiguous, as a K tile
+// read as K^T)
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(uint32_t M, uint32_t N) {
+  return idesc_bf16_f32(M, N, 1) | (1u << 15);
+}
+
 // D(tmem) (+)= A(smem) * B(smem)
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                         uint32_t accumulate) {
@@ -336,6 +342,11 @@ __device__ __forceinline__ void regs_inc() {
 }
 
 // ---------------------------------------------------------------- math
+// relaxed fp32 reduction into global memory (no return value)
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -306,3 +306,93 @@ def test_bsr_workload_one_kv_group():
                      causal=True)[0, 0]
     _group_bwd_check(dq[b].cpu(), dk[b].cpu(), dv[b].cpu(), w["q"][b], w["k"][b], w["v"][b], do[b], M, g,
                      w["H"] // w["Hkv"], w["scale"], (0, w["S"]), "bsr")
+
+
+class _two_pass:
+    """Backward in the two-pass (bitwise reproducible) form inside the block."""
+
+    def __enter__(self):
+        bfa.set_bwd_deterministic(True)
+
+    def __exit__(self, *exc):
+        bfa.set_bwd_deterministic(False)
+
+
+@pytest.mark.parametrize("case", ["dense_ragged_gqa", "varlen_window", "varlen_single_row_tiles",
+                                  "varlen_cross_full_tiles"])
+def test_fused_and_two_pass_forms_agree(case):
+    # D = 128: the fused pass (default) and the two-pass form both match the
+    # oracle; dK and dV are made by the same products in the same order in both
+    # forms (bit-identical); dQ differs only by the order of its fp32 sums.  The
+    # packed cases put other sequences' tokens in the rows past a sequence's last
+    # key tile: the fused pass sums dQ over every key row of a tile, so those rows
+    # must not count (one valid query and one valid key make a full diagonal tile;
+    # non-causal cross lengths make full tiles that run past their keys).
+    D = 128
+    if case == "dense_ragged_gqa":
+        rng = np.random.default_rng(5)
+        B, H, Hkv, Sq, Sk = 2, 4, 2, 300, 389
+        M = rng.random((Sq, Sk)) < 0.4
+        M[:, :3] = True
+        P = bfa.plan_dense(_cuda(M))
+        q = workloads.randn_bf16((B, Sq, H, D), 51)
+        k = workloads.randn_bf16((B, Sk, Hkv, D), 52)
+        v = workloads.randn_bf16((B, Sk, Hkv, D), 53)
+        do = workloads.randn_bf16((B, Sq, H, D), 54)
+        rq, rk, rv = ob.attention_bwd_bshd(q, k, v, do, lambda b, h: M, None)
+    else:
+        H, Hkv = 4, 2
+        if case == "varlen_cross_full_tiles":
+            cq = np.array([0, 100, 357, 400], dtype=np.int32)
+            ck = np.array([0, 150, 389, 529], dtype=np.int32)
+            # one block id for every token: each query attends all keys of its sequence
+            ids = dict(q_blk=_cuda(np.zeros(cq[-1], np.int32)), k_blk=_cuda(np.zeros(ck[-1], np.int32)))
+            P = bfa.plan_blockids(**ids, cu_seqlens_q=_cuda(cq), cu_seqlens_k=_cuda(ck), max_q=512, max_k=512)
+            M = om.varlen_dense(cq, ck, False, -1)
+        else:
+            cq = ck = (np.array([0, 130, 515, 772, 836], dtype=np.int32) if case == "varlen_window"
+                       else np.array([0, 1, 130, 259], dtype=np.int32))
+            W = 200 if case == "varlen_window" else -1
+            P = bfa.plan_blockids(cu_seqlens_q=_cuda(cq), cu_seqlens_k=_cuda(ck), max_q=512, max_k=512,
+                                  window_left=W)
+            M = om.varlen_dense(cq, ck, True, W)
+        Tq, Tk = int(cq[-1]), int(ck[-1])
+        q = workloads.randn_bf16((Tq, H, D), 61)
+        k = workloads.randn_bf16((Tk, Hkv, D), 62)
+        v = workloads.randn_bf16((Tk, Hkv, D), 63)
+        do = workloads.randn_bf16((Tq, H, D), 64)
+        rq, rk, rv = ob.attention_bwd_thd(q, k, v, do, M)
+    qc, kc, vc, dc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out, lse = bfa.fwd(P, qc, kc, vc)
+    fused = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    with _two_pass():
+        two = bfa.bwd(P, qc, kc, vc, out, dc, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    for grads in (fused, two):
+        _close(grads[0], rq, "dq")
+        _close(grads[1], rk, "dk")
+        _close(grads[2], rv, "dv")
+    assert torch.equal(fused[1], two[1]) and torch.equal(fused[2], two[2])
+    dq_diff = (fused[0].float() - two[0].float()).abs().max().item()
+    assert dq_diff <= 2 ** -7 * two[0].float().abs().max().item() + 1e-3
+
+
+def test_two_pass_form_is_bitwise_reproducible():
+    # the deterministic form repeats itself bit for bit; the fused form repeats
+    # dK and dV bit for bit (its dQ sums may come in another order)
+    B, H, Hkv, N, D = 1, 4, 2, 640, 128
+    M = np.tril(np.ones((N, N), dtype=bool))
+    P = bfa.plan_dense(_cuda(M))
+    q, k, v, do = (workloads.randn_bf16(s, 70 + i).cuda() for i, s in
+                   enumerate([(B, N, H, D), (B, N, Hkv, D), (B, N, Hkv, D), (B, N, H, D)]))
+    out, lse = bfa.fwd(P, q, k, v)
+    with _two_pass():
+        a = bfa.bwd(P, q, k, v, out, do, lse)
+        b = bfa.bwd(P, q, k, v, out, do, lse)
+    f1 = bfa.bwd(P, q, k, v, out, do, lse)
+    f2 = bfa.bwd(P, q, k, v, out, do, lse)
+    torch.cuda.synchronize()
+    P.device_status()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    assert torch.equal(f1[1], f2[1]) and torch.equal(f1[2], f2[2])

@@ -48,6 +48,8 @@ CASES = [
     "tests/test_gpu_bwd.py::test_predicate_terms",
     "tests/test_gpu_bwd.py::test_general_block_sparse_with_validity",
     "tests/test_gpu_bwd.py::test_varlen_causal_packed",
+    "tests/test_gpu_bwd.py::test_fused_and_two_pass_forms_agree",
+    "tests/test_gpu_bwd.py::test_two_pass_form_is_bitwise_reproducible",
     # full-size workloads, the bench's own launch among them
     "tests/test_gpu_plan.py::test_dense_plan_causal_8192",
     "tests/test_gpu_plan.py::test_bsr_plan_workload_full_size_every_group",
