@@ -191,6 +191,21 @@ def block_bits_dense(block_bits, Sq, Skv, q_block_size, kv_block_size, causal=Fa
     return M
 
 
+def gqa_packed_rows(M, heads_per_kv):
+    """Rows of one (batch, kv head) mask in GQA-packed order (flashinfer
+    block_sparse_attention, ``q_block_size``: one physical query tile holds the
+    query tokens of a BSR row for every query head that shares the kv head, which
+    is why the page asks ``q_block_size * Hq / Hkv`` to be a multiple of 8).
+
+    ``M`` is the (Sq, Skv) mask of the kv head.  The result has Sq * heads_per_kv
+    rows; row ``t`` is query position ``t // heads_per_kv`` of the group's query
+    head ``t % heads_per_kv``, and every head of the group attends with the kv
+    head's routing, so row ``t`` is ``M[t // heads_per_kv]``.
+    """
+    M = np.asarray(M, dtype=bool)
+    return np.repeat(M, int(heads_per_kv), axis=0)
+
+
 def bsr_to_block_bits(block_indptr, block_indices, n_kv_blocks):
     """The exact-block bitmap of BSR routing (same selection, bitmask layout)."""
     indptr = np.asarray(block_indptr, dtype=np.int64)

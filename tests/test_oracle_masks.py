@@ -322,3 +322,33 @@ def test_predicate_terms_match_the_page_algebra():
     np.testing.assert_array_equal(om.predicate_dense(PREDICATES["global3_window4"], 20, 20), alg)
     assert om.predicate_dense(PREDICATES["noop"], 4, 6).all()
     assert not om.predicate_dense([], 4, 6).any()
+
+
+def test_gqa_packed_rows_hand_example_and_brute_force():
+    # two positions, two keys, two heads per kv head: each position's row appears
+    # once per head, position-major (row t = position t // 2, head t % 2)
+    M = np.array([[1, 0], [0, 1]], dtype=bool)
+    np.testing.assert_array_equal(om.gqa_packed_rows(M, 2),
+                                  np.array([[1, 0], [1, 0], [0, 1], [0, 1]], dtype=bool))
+    rng = np.random.default_rng(3)
+    A = rng.random((37, 53)) < 0.4
+    for G in (1, 2, 4, 8):
+        P = om.gqa_packed_rows(A, G)
+        assert P.shape == (37 * G, 53)
+        for t in range(P.shape[0]):
+            np.testing.assert_array_equal(P[t], A[t // G])
+    np.testing.assert_array_equal(om.gqa_packed_rows(A, 1), A)
+
+
+def test_gqa_packed_rows_of_a_bsr_routing_follow_the_routing():
+    # packed rows of a BSR mask: row t attends key j exactly when position t // G's
+    # BSR row lists j's block (checked against the routing directly, not via bsr_dense)
+    indptr = np.array([[[0, 2, 3, 5]]], dtype=np.int32)
+    indices = np.array([0, 2, 1, 0, 3], dtype=np.int32)
+    Sq, Skv, qb, kb, G = 12, 32, 4, 8, 4
+    packed = om.gqa_packed_rows(om.bsr_dense(indptr, indices, Sq, Skv, qb, kb)[0, 0], G)
+    for t in range(Sq * G):
+        r = (t // G) // qb
+        blocks = set(indices[indptr[0, 0, r]:indptr[0, 0, r + 1]].tolist())
+        for j in range(Skv):
+            assert packed[t, j] == (j // kb in blocks)
