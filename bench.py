@@ -475,7 +475,7 @@ def run_sweep(args):
     def cuda(x):
         return torch.as_tensor(np.ascontiguousarray(x)).cuda()
 
-    def measure(name, P, q, k, v, pairs, D, plan_desc):
+    def measure(name, P, q, k, v, pairs, D, plan_desc, bwd=True):
         if only is not None and name != only:
             return
         out, lse = bfa.fwd(P, q, k, v)
@@ -491,12 +491,13 @@ def run_sweep(args):
         dout = torch.randn(q.shape, device="cuda", generator=g).to(torch.bfloat16)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         fms = _time_ms(lambda: bfa.fwd(P, q, k, v, out=out, lse=lse), reps)
-        bms = _time_ms(lambda: bfa.bwd(P, q, k, v, out, dout, lse, dq=dq, dk=dk, dv=dv), reps)
+        bms = _time_ms(lambda: bfa.bwd(P, q, k, v, out, dout, lse, dq=dq, dk=dk, dv=dv), reps) if bwd else None
         P.device_status()
         flops = 4.0 * D * pairs
         print(json.dumps({"workload": name, "plan": plan_desc, "attended_pairs": pairs, "fwd_ms": fms,
                           "fwd_tflops": flops / (fms * 1e-3) / 1e12, "bwd_ms": bms,
-                          "bwd_tflops": 2.5 * flops / (bms * 1e-3) / 1e12, "reps": reps}), flush=True)
+                          "bwd_tflops": 2.5 * flops / (bms * 1e-3) / 1e12 if bwd else None, "reps": reps}),
+              flush=True)
 
     w = workloads.causal_8192()
     measure("causal_8192", bfa.plan_dense(w["mask"].cuda()), w["q"].cuda(), w["k"].cuda(), w["v"].cuda(),
@@ -536,6 +537,27 @@ def run_sweep(args):
     u = workloads.union_16384(with_qkv=False)
     measure("union_16384", bfa.plan_dense(u["mask"].cuda()), w["q"].cuda(), w["k"].cuda(), w["v"].cuda(),
             float(u["mask"].sum()) * w["B"] * w["H"], w["D"], "dense")
+    del w, u
+    # 16-token BSR rows with 8 query heads per kv head: GQA-packed tiles (one BSR
+    # row of all 8 heads per tile) against 128-token tiles (the union of 8 rows'
+    # lists); forward only (packed plans have no backward)
+    w = workloads.bsr_16384_q16_gqa8()
+    ip, ix, S, qb, kb = w["block_indptr"], w["block_indices"], w["S"], w["q_block"], w["kv_block"]
+    G = w["H"] // w["Hkv"]
+    per_group = 0.0
+    for b in range(ip.shape[0]):
+        for h in range(ip.shape[1]):
+            for r in range(ip.shape[2] - 1):
+                sel = ix[ip[b, h, r]:ip[b, h, r + 1]]
+                d = (r * qb) // kb
+                t = np.arange(r * qb, min(S, (r + 1) * qb))
+                per_group += float((sel < d).sum()) * t.size * kb + float((t - d * kb + 1).sum())
+    q, k, v = w["q"].cuda(), w["k"].cuda(), w["v"].cuda()
+    for name, plan in (("bsr_16384_q16_gqa8 packed", bfa.plan_bsr_packed(cuda(ip), cuda(ix), S, S, G, qb, kb,
+                                                                         causal=True)),
+                       ("bsr_16384_q16_gqa8 unpacked", bfa.plan_bsr(cuda(ip), cuda(ix), S, S, qb, kb, causal=True))):
+        measure(name, plan, q, k, v, per_group * G, w["D"], "BSR, 16-token rows, causal inside blocks", bwd=False)
+        del plan
     return 0
 
 
@@ -550,7 +572,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="forward/backward on every workload (information)")
     ap.add_argument("--workload", default=None,
                     help="with --sweep: only this workload (causal_8192, blockcausal_gqa, 'varlen_16 window=-1', "
-                         "'varlen_16 window=1024', bsr_16384, union_16384)")
+                         "'varlen_16 window=1024', bsr_16384, union_16384, 'bsr_16384_q16_gqa8 packed', "
+                         "'bsr_16384_q16_gqa8 unpacked')")
     ap.add_argument("--fwd-only", action="store_true", help="with --sweep: forward calls only, no timing line")
     args = ap.parse_args()
     if args.warmup < 3:

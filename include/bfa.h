@@ -106,6 +106,9 @@ typedef struct bfa_plan_info {
   int32_t packed_fine;    /* 1: partial tiles carry packed fine masks (bfa_plan_export fills fine) */
   int32_t n_cols;         /* key-tile columns (sum over groups of their key tiles): the backward's
                              dK/dV work units, see bfa_plan_export_cols                         */
+  int32_t heads_per_kv;   /* bfa_plan_bsr_packed: query heads packed into each row's tiles; else 1;
+                             with packing, sq counts query positions and the groups' rows count
+                             positions x heads_per_kv                                           */
 } bfa_plan_info;
 
 /* Library version string. */
@@ -206,6 +209,24 @@ bfa_status bfa_plan_predicate(const bfa_mask_term* terms, int n_terms, int B, in
 bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
                         int Sq, int Skv, int q_block, int kv_block, int causal, const uint32_t* kv_valid_bits,
                         bfa_plan** out, void* stream);
+
+/*
+ * bfa_plan_bsr with GQA-packed query tiles (flashinfer block_sparse_attention,
+ * q_block_size: one physical query tile holds the query tokens of BSR rows for
+ * every query head of a kv head, so it never straddles two rows' lists when
+ * q_block * heads_per_kv is a multiple of 128).  Plan row t of the (b, hkv)
+ * routing slice is query position t / heads_per_kv of query head
+ * hkv * heads_per_kv + t % heads_per_kv; a 128-row tile is 128 / heads_per_kv
+ * positions of all heads_per_kv heads.  heads_per_kv = H / Hkv of the calls that
+ * use the plan: a power of two up to 128, with q_block * heads_per_kv a multiple
+ * of 8 (the page's rule); other arguments as for bfa_plan_bsr.  Only bfa_fwd,
+ * bfa_fwd_approx and bfa_fwd_paged take these plans (a batched (B, Sq, H, D) query
+ * layout with heads of one kv head adjacent, as BSHD has them); bfa_bwd returns
+ * BFA_ERR_UNSUPPORTED for them.
+ */
+bfa_status bfa_plan_bsr_packed(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
+                               int heads_per_kv, int Sq, int Skv, int q_block, int kv_block, int causal,
+                               const uint32_t* kv_valid_bits, bfa_plan** out, void* stream);
 
 /*
  * Plan from an exact-block bitmap (flashinfer block_sparse_attention,

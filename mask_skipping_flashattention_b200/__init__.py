@@ -23,7 +23,8 @@ import torch
 from . import _lib
 from ._lib import BfaError, PlanInfo
 
-__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_predicate", "plan_bsr", "plan_block_bits",
+__all__ = ["Plan", "BfaError", "plan_dense", "plan_blockids", "plan_predicate", "plan_bsr", "plan_bsr_packed",
+           "plan_block_bits",
            "fwd", "bwd", "fwd_paged",
            "make_att_block_ids",
            "is_available", "load_error", "set_wait_timeout_ns", "set_bwd_deterministic", "selftest_wait_timeout", "library_path"]
@@ -276,6 +277,22 @@ def plan_bsr(block_indptr, block_indices, Sq, Skv, q_block_size=TILE, kv_block_s
     _lib.check(_L.bfa_plan_bsr(_ptr(ip), _ptr(ix) if ix.numel() else None, ix.numel(), B, Hkv, int(Sq), int(Skv),
                                int(q_block_size), int(kv_block_size), 1 if causal else 0, _ptr(kv),
                                ctypes.byref(h), st))
+    return Plan(h, st)
+
+
+def plan_bsr_packed(block_indptr, block_indices, Sq, Skv, heads_per_kv, q_block_size=TILE, kv_block_size=TILE,
+                    causal=False, kv_valid_bits=None, stream=None):
+    """BSR plan with GQA-packed query tiles: each tile holds 128 / heads_per_kv query
+    positions of all ``heads_per_kv`` query heads of a kv head (forward only)."""
+    ip = block_indptr.to(torch.int32).contiguous()
+    ix = block_indices.to(torch.int32).contiguous()
+    kv = kv_valid_bits.contiguous() if kv_valid_bits is not None else None
+    B, Hkv, _ = ip.shape
+    h = ctypes.c_void_p()
+    st = _stream(stream)
+    _lib.check(_L.bfa_plan_bsr_packed(_ptr(ip), _ptr(ix) if ix.numel() else None, ix.numel(), B, Hkv,
+                                      int(heads_per_kv), int(Sq), int(Skv), int(q_block_size), int(kv_block_size),
+                                      1 if causal else 0, _ptr(kv), ctypes.byref(h), st))
     return Plan(h, st)
 
 

@@ -43,6 +43,9 @@ SIGNATURES = {
     "bfa_plan_bsr": (ctypes.c_int, [c_void, c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, c_void,
                                     ctypes.POINTER(c_void), c_void]),
+    "bfa_plan_bsr_packed": (ctypes.c_int, [c_void, c_void, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           c_void, ctypes.POINTER(c_void), c_void]),
     "bfa_plan_block_bits": (ctypes.c_int, [c_void, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, c_void,
                                            ctypes.POINTER(c_void), c_void]),
@@ -78,7 +81,8 @@ class PlanInfo(ctypes.Structure):
                 ("n_rows", ctypes.c_int32), ("grid_tiles", ctypes.c_int64), ("batch", ctypes.c_int32),
                 ("hkv", ctypes.c_int32), ("sq", ctypes.c_int32), ("sk", ctypes.c_int32),
                 ("max_kv_tiles", ctypes.c_int32), ("window_left", ctypes.c_int32), ("causal", ctypes.c_int32),
-                ("n_pairs", ctypes.c_int32), ("packed_fine", ctypes.c_int32), ("n_cols", ctypes.c_int32)]
+                ("n_pairs", ctypes.c_int32), ("packed_fine", ctypes.c_int32), ("n_cols", ctypes.c_int32),
+                ("heads_per_kv", ctypes.c_int32)]
 
 
 class MaskTerm(ctypes.Structure):

@@ -48,12 +48,12 @@ cudaError_t launch_cols(const GroupInfo* groups, int n_groups, const uint8_t* cl
                         int32_t* col_group, int32_t* col_cnt, int32_t* col_ptr, int32_t* q_tile, int32_t* tpart,
                         int32_t* col_order, cudaStream_t s);
 cudaError_t launch_bits_classify(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
-                                 int q_block, int kv_block, int causal, const GroupInfo* groups, int n_groups,
-                                 int nqt, uint8_t* cls, cudaStream_t s);
+                                 int q_block, int kv_block, int causal, int g_pack, const GroupInfo* groups,
+                                 int n_groups, int nqt, uint8_t* cls, cudaStream_t s);
 cudaError_t launch_bits_fine(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
-                             int q_block, int kv_block, int causal, const GroupInfo* groups, const int32_t* row_group,
-                             int n_rows, const int32_t* row_ptr, const int32_t* kv_tile, const int32_t* part,
-                             uint32_t* fine, cudaStream_t s);
+                             int q_block, int kv_block, int causal, int g_pack, const GroupInfo* groups,
+                             const int32_t* row_group, int n_rows, const int32_t* row_ptr, const int32_t* kv_tile,
+                             const int32_t* part, uint32_t* fine, cudaStream_t s);
 cudaError_t launch_make_block_ids(const uint8_t* pad, const uint8_t* att, int B, int N, int n_cross,
                                   const uint8_t* cross_pad, int32_t* q_blk, int32_t* k_blk, uint8_t* q_valid,
                                   uint8_t* k_valid, cudaStream_t s);
@@ -75,6 +75,9 @@ using namespace bfa;
 // ----------------------------------------------------------------------------
 struct bfa_plan {
   int kind = 0, varlen = 0, batch = 0, hkv = 0, sq = 0, sk = 0, window = -1, causal = 0;
+  // GQA-packed query rows (bfa_plan_bsr_packed): plan row t of a (batch, kv head)
+  // group is query position t / pack_g of head t % pack_g of the kv head; 1: off
+  int pack_g = 1;
   int n_groups = 0, n_rows = 0, n_pairs = 0, max_nkt = 0, max_nqt = 0, mask_mode = MASK_BITS;
   int64_t grid_tiles = 0;
   int64_t fine_tiles = 0;       // tiles of packed fine words held in `fine`
@@ -681,7 +684,8 @@ bool kv_block_ok(int kv_block) { return kv_block == 8 || kv_block == 16 || kv_bl
 // reduced to tile classes plus packed fine words for the partial tiles.
 bfa_status plan_block_sparse(const int32_t* indptr, const int32_t* indices, int64_t n_indices,
                              const uint32_t* block_bits, const uint32_t* kv_valid, int B, int Hkv, int Sq, int Skv,
-                             int q_block, int kv_block, int causal, bfa_plan** out, cudaStream_t st) {
+                             int q_block, int kv_block, int causal, bfa_plan** out, cudaStream_t st,
+                             int g_pack = 1) {
   bfa_plan* P = new bfa_plan();
   uint32_t* tmp_bits = nullptr;
   auto cleanup = [&]() {
@@ -698,8 +702,10 @@ bfa_status plan_block_sparse(const int32_t* indptr, const int32_t* indices, int6
   P->sq = Sq;
   P->sk = Skv;
   P->stream = st;
+  P->pack_g = g_pack;
+  // packed: each group's plan rows are its Sq positions x g_pack heads
   for (int b = 0; b < B; ++b)
-    for (int h = 0; h < Hkv; ++h) P->groups_h.push_back(make_group(0, Sq, 0, Skv, b, h));
+    for (int h = 0; h < Hkv; ++h) P->groups_h.push_back(make_group(0, Sq * g_pack, 0, Skv, b, h));
   P->regular = true;
   P->regular_hkv = Hkv;
   finalize_layout(P);
@@ -728,7 +734,7 @@ bfa_status plan_block_sparse(const int32_t* indptr, const int32_t* indices, int6
     }
     bits = tmp_bits;
   }
-  BFA_CUDA(launch_bits_classify(bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, P->causal, P->groups,
+  BFA_CUDA(launch_bits_classify(bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, P->causal, g_pack, P->groups,
                                 P->n_groups, P->max_nqt, P->cls, st),
            "block-sparse classify kernel");
   if ((s = build_rows(P, 1))) { cleanup(); return s; }
@@ -743,8 +749,8 @@ bfa_status plan_block_sparse(const int32_t* indptr, const int32_t* indices, int6
            "fine-mask allocation");
   P->fine = static_cast<uint32_t*>(P->fine_extra);
   P->fine_tiles = nnz;
-  BFA_CUDA(launch_bits_fine(bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, P->causal, P->groups, P->row_group,
-                            P->n_rows, P->row_ptr, P->kv_tile, P->part, P->fine, st),
+  BFA_CUDA(launch_bits_fine(bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, P->causal, g_pack, P->groups,
+                            P->row_group, P->n_rows, P->row_ptr, P->kv_tile, P->part, P->fine, st),
            "block-sparse fine-mask kernel");
   if (tmp_bits) {
     cudaFreeAsync(tmp_bits, st);
@@ -852,6 +858,31 @@ BFA_API bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, i
   return BFA_OK;
 }
 
+BFA_API bfa_status bfa_plan_bsr_packed(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B,
+                                       int Hkv, int heads_per_kv, int Sq, int Skv, int q_block, int kv_block,
+                                       int causal, const uint32_t* kv_valid_bits, bfa_plan** out, void* stream) {
+  if (!out) return fail(BFA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (B <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || n_indices < 0)
+    return fail(BFA_ERR_INVALID_ARG, "bad sizes B=%d Hkv=%d Sq=%d Skv=%d n_indices=%lld", B, Hkv, Sq, Skv,
+                (long long)n_indices);
+  const int G = heads_per_kv;
+  if (G <= 0 || G > kTile || (G & (G - 1)) != 0)
+    return fail(BFA_ERR_INVALID_ARG, "heads_per_kv=%d must be a power of two up to %d", G, kTile);
+  if (q_block <= 0 || (static_cast<int64_t>(q_block) * G) % 8 != 0)
+    return fail(BFA_ERR_INVALID_ARG, "q_block=%d times heads_per_kv=%d must be a positive multiple of 8", q_block, G);
+  if (static_cast<int64_t>(Sq) * G >= (int64_t(1) << 31))
+    return fail(BFA_ERR_CAPACITY, "Sq * heads_per_kv = %lld exceeds int32", (long long)Sq * G);
+  if (!kv_block_ok(kv_block))
+    return fail(BFA_ERR_INVALID_ARG, "kv_block=%d: allowed sizes are 8, 16, 32 and the multiples of 64", kv_block);
+  bfa_status s;
+  if ((s = need_device(indptr, "block_indptr"))) return s;
+  if (n_indices > 0 && (s = need_device(indices, "block_indices"))) return s;
+  if ((s = need_device(kv_valid_bits, "kv_valid_bits", true))) return s;
+  return plan_block_sparse(indptr, indices, n_indices, nullptr, kv_valid_bits, B, Hkv, Sq, Skv, q_block, kv_block,
+                           causal, out, static_cast<cudaStream_t>(stream), G);
+}
+
 BFA_API bfa_status bfa_plan_block_bits(const uint32_t* block_bits, int B, int Hkv, int Sq, int Skv, int q_block,
                                        int kv_block, int causal, const uint32_t* kv_valid_bits, bfa_plan** out,
                                        void* stream) {
@@ -923,6 +954,37 @@ bool make_tmap(CUtensorMap* m, const void* base, int D, int heads, int64_t token
   return true;
 }
 
+// 5-D map over (d, head in group, kv head, token, batch) of a bf16 (B, S, H, D)
+// tensor whose G heads of a kv head are adjacent: box = 64 d x G heads x 1 kv head
+// x 128 / G tokens x 1 batch, so a box is one 128-row tile of GQA-packed rows
+// (position-major, head-minor), 128-byte swizzle.
+bool make_tmap_packed(CUtensorMap* m, const void* base, int D, int G, int hkv, int64_t tokens, int batch,
+                      int64_t s_head, int64_t s_tok, int64_t s_batch, std::string* why) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  if (s_batch == 0 || batch == 1) s_batch = std::max<int64_t>(s_tok * std::max<int64_t>(tokens, 1), 8);
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(hkv),
+                        static_cast<cuuint64_t>(tokens), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(s_head) * 2, static_cast<cuuint64_t>(s_head) * G * 2,
+                           static_cast<cuuint64_t>(s_tok) * 2, static_cast<cuuint64_t>(s_batch) * 2};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(G), 1, static_cast<cuuint32_t>(kTile / G), 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "packed tensor map rejected (CUresult %d) for strides (%lld, %lld, %lld)", (int)r,
+             (long long)s_head, (long long)s_tok, (long long)s_batch);
+    *why = buf;
+    return false;
+  }
+  return true;
+}
+
 int sm_count() {
   static int n = 0;
   if (!n) {
@@ -945,10 +1007,22 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
                                  void* out, const int64_t* os, float* lse, uint64_t wait_ns, cudaStream_t st,
                                  std::string* why, const PagedKV& pg = PagedKV(), float skip_log2 = 0.f) {
   const int bq = P->varlen ? 1 : B;
+  const int G = P->pack_g;
   CUtensorMap tq, tk, tv, to;
-  if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why)) return cudaErrorInvalidValue;
-  // the output with the query layout: whole in-range tiles leave through TMA stores
-  if (!make_tmap(&to, out, D, H, P->sq, bq, os[2], os[1], P->varlen ? 0 : os[0], why)) return cudaErrorInvalidValue;
+  if (G > 1) {  // GQA-packed tiles: the plan was made for G heads per kv head
+    if (H != Hkv * G) {
+      *why = "the plan packs " + std::to_string(G) + " query heads per kv head; H / Hkv = " +
+             std::to_string(H / Hkv);
+      return cudaErrorInvalidValue;
+    }
+    if (!make_tmap_packed(&tq, q, D, G, Hkv, P->sq, bq, qs[2], qs[1], qs[0], why) ||
+        !make_tmap_packed(&to, out, D, G, Hkv, P->sq, bq, os[2], os[1], os[0], why))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], why)) return cudaErrorInvalidValue;
+    // the output with the query layout: whole in-range tiles leave through TMA stores
+    if (!make_tmap(&to, out, D, H, P->sq, bq, os[2], os[1], P->varlen ? 0 : os[0], why)) return cudaErrorInvalidValue;
+  }
   if (pg.page_size == 0) {
     if (!make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], why) ||
         !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], why))
@@ -992,14 +1066,18 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   p.H = H;
   p.Hkv = Hkv;
   p.D = D;
-  p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? H / Hkv : H);
+  // packed plans hold every head of a kv head in their rows: one replica per row
+  p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? (G > 1 ? 1 : H / Hkv) : H);
+  p.pack_g = G;
+  p.pack_shift = 0;
+  while ((1 << p.pack_shift) < G) ++p.pack_shift;
   p.plan.pair_row = P->pair_row;
   p.plan.pair_order = P->pair_order;
   p.plan.n_pairs = P->n_pairs;
   // A CTA runs two query tiles that share K/V: two heads of one kv head on the
   // same row when the GQA group is even (identical key lists), else two
   // consecutive query tiles of one head.
-  p.pair_heads = ((H / Hkv) % 2 == 0) ? 1 : 0;
+  p.pair_heads = (G == 1 && (H / Hkv) % 2 == 0) ? 1 : 0;
   const int64_t units = p.pair_heads ? P->n_rows : P->n_pairs;
   const int64_t items = p.pair_heads ? p.rep / 2 : p.rep;
   // Keep enough replica units of a row together to fill about two waves of
@@ -1008,7 +1086,7 @@ cudaError_t fwd_launch_from_host(const bfa_plan* P, const void* q, const void* k
   int64_t chunk = std::min<int64_t>(items, std::max<int64_t>(1, (waves + units - 1) / std::max<int64_t>(units, 1)));
   const int64_t kv_head_bytes = std::max<int64_t>(1, static_cast<int64_t>(P->sk) * D * 4);
   const int64_t l2_kv_heads = std::max<int64_t>(1, (64LL << 20) / kv_head_bytes);
-  const int64_t units_per_kv_head = p.pair_heads ? std::max(1, (H / Hkv) / 2) : std::max(1, H / Hkv);
+  const int64_t units_per_kv_head = G > 1 ? 1 : (p.pair_heads ? std::max(1, (H / Hkv) / 2) : std::max(1, H / Hkv));
   chunk = std::max<int64_t>(1, std::min<int64_t>(chunk, l2_kv_heads * units_per_kv_head));
   p.head_chunk = static_cast<int>(chunk);
   p.varlen = P->varlen;
@@ -1218,6 +1296,8 @@ BFA_API bfa_status bfa_bwd(const bfa_plan* Pc, const void* q, const void* k, con
     return fail(BFA_ERR_INVALID_ARG, "B=%d does not match the plan's %d", B, P->batch);
   if (P->kind == BFA_PLAN_BSR && Hkv != P->hkv)
     return fail(BFA_ERR_INVALID_ARG, "Hkv=%d does not match the BSR routing's %d", Hkv, P->hkv);
+  if (P->pack_g > 1)
+    return fail(BFA_ERR_UNSUPPORTED, "the backward takes plans without GQA-packed query tiles (bfa_plan_bsr)");
   if (!lse) return fail(BFA_ERR_INVALID_ARG, "lse is required by the backward");
   bfa_status s;
   if ((s = need_device(q, "q")) || (s = need_device(k, "k")) || (s = need_device(v, "v")) ||
@@ -1327,6 +1407,7 @@ BFA_API bfa_status bfa_plan_get_info(const bfa_plan* P, bfa_plan_info* info) {
   info->n_pairs = P->n_pairs;
   info->packed_fine = P->mask_mode == MASK_BITS ? 1 : 0;
   info->n_cols = plan_n_cols(P);
+  info->heads_per_kv = P->pack_g;
   return BFA_OK;
 }
 

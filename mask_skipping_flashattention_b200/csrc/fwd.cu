@@ -314,8 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qs = wk_s.q_off + wk_s.qt[s] * kTile;
         uint8_t* dq = s ? sQ1 : sQ0;
 #pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk_s.h[s], qs, wk_s.b);
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          if (p.pack_g > 1)  // 128 >> pack_shift positions of every head of the kv head
+            tma_load_5d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, 0, wk_s.hk, qs >> p.pack_shift, wk_s.b);
+          else
+            tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk_s.h[s], qs, wk_s.b);
+        }
       }
     }
   }
@@ -574,6 +578,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool store = qpos < wk.q_len;  // TMEM loads below stay whole-warp; only stores are per row
       const int h = slot ? wk.h[1] : wk.h[0];
+      // the row's query head and position (GQA-packed tiles: rows position-major over the kv head's heads)
+      const int hrow = p.pack_g > 1 ? (wk.hk << p.pack_shift) + (qpos & (p.pack_g - 1)) : h;
+      const int prow = p.pack_g > 1 ? qpos >> p.pack_shift : qpos;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       const int qt0 = (slot ? wk.qt[1] : wk.qt[0]) * kTile;  // first row of the tile in its group
       if (qt0 + kTile <= wk.q_len) {
@@ -612,14 +619,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (quarter == 0 && lane == 0 && ok && !*static_cast<volatile int*>(&abort_flag)) {
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_store_4d(&tmO, stg + pn * 16384, pn * 64, h, wk.q_off + qt0, wk.b);
+            if (p.pack_g > 1)
+              tma_store_5d(&tmO, stg + pn * 16384, pn * 64, 0, wk.hk, (wk.q_off + qt0) >> p.pack_shift, wk.b);
+            else
+              tma_store_4d(&tmO, stg + pn * 16384, pn * 64, h, wk.q_off + qt0, wk.b);
           bulk_commit_group();
           bulk_wait_group_read0();
         }
       } else if (ok) {
-        const int64_t tok = static_cast<int64_t>(wk.q_off) + qpos;
+        const int64_t tok = static_cast<int64_t>(wk.q_off) + prow;
         __nv_bfloat16* op =
-            p.out + static_cast<int64_t>(wk.b) * p.o_sb + tok * p.o_ss + static_cast<int64_t>(h) * p.o_sh;
+            p.out + static_cast<int64_t>(wk.b) * p.o_sb + tok * p.o_ss + static_cast<int64_t>(hrow) * p.o_sh;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -644,11 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (ok) {
-        const int64_t tok = static_cast<int64_t>(wk.q_off) + qpos;
+        const int64_t tok = static_cast<int64_t>(wk.q_off) + prow;
         if (p.lse && store) {
           const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-          const int64_t li = p.varlen ? static_cast<int64_t>(h) * p.Sq_lse + tok
-                                      : (static_cast<int64_t>(wk.b) * p.H + h) * p.Sq_lse + qpos;
+          const int64_t li = p.varlen ? static_cast<int64_t>(hrow) * p.Sq_lse + tok
+                                      : (static_cast<int64_t>(wk.b) * p.H + hrow) * p.Sq_lse + prow;
           p.lse[li] = lse;
         }
       }

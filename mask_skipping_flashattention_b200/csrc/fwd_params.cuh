@@ -32,6 +32,11 @@ struct FwdParams {
   // approximate mode: a tile whose scores all lie more than skip_log2 (log2 units)
   // below the rows' running maxima is dropped; <= 0 keeps the exact computation
   float skip_log2;
+  // GQA-packed query tiles: row t of a plan tile is query position t >> pack_shift
+  // of head (kv head << pack_shift) + (t & (pack_g - 1)); Q and O move through
+  // 5-D maps.  pack_g = 1: rows are positions of one head.
+  int32_t pack_g;
+  int32_t pack_shift;
 };
 
 int fwd_smem_bytes(int D);

@@ -611,6 +611,9 @@ struct BlockSparseArgs {
   const uint32_t* kv_valid;  // [batch][kv_wpb] token validity bits, or null
   int nqb, wpr, kv_wpb;
   int q_block, kv_block, causal;
+  // GQA-packed query rows: plan row t of a group is query position t / g_pack of
+  // head t % g_pack of its kv head (1: rows are positions)
+  int g_pack;
 };
 
 // attend-bits of query position i (row of query block qb) over the 32 columns
@@ -648,8 +651,9 @@ __global__ void __launch_bounds__(128) k_bits_classify(BlockSparseArgs a, const 
   const int qt = blockIdx.y;
   if (qt >= g.nqt) return;
   const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
-  const int i = qt * kTile + r;
-  const bool in = i < g.q_len;
+  const int t = qt * kTile + r;  // plan row
+  const bool in = t < g.q_len;
+  const int i = t / a.g_pack;    // query position
   const uint32_t* rowbits = a.bits + (static_cast<int64_t>(blockIdx.x) * a.nqb + (in ? i / a.q_block : 0)) * a.wpr;
   const uint32_t* kvrow = a.kv_valid ? a.kv_valid + static_cast<int64_t>(g.b) * a.kv_wpb : nullptr;
   const int rows_in = min(kTile, g.q_len - qt * kTile);
@@ -683,8 +687,9 @@ __global__ void __launch_bounds__(128) k_bits_fine(BlockSparseArgs a, const Grou
   const int grp = row_group[row];
   const GroupInfo g = groups[grp];
   const int qt = row - g.row0, r = threadIdx.x;
-  const int i = qt * kTile + r;
-  const bool in = i < g.q_len;
+  const int t = qt * kTile + r;  // plan row
+  const bool in = t < g.q_len;
+  const int i = t / a.g_pack;    // query position
   const uint32_t* rowbits = a.bits + (static_cast<int64_t>(grp) * a.nqb + (in ? i / a.q_block : 0)) * a.wpr;
   const uint32_t* kvrow = a.kv_valid ? a.kv_valid + static_cast<int64_t>(g.b) * a.kv_wpb : nullptr;
   for (int e = row_ptr[row]; e < row_ptr[row + 1]; ++e) {
@@ -942,20 +947,20 @@ cudaError_t launch_bsr_to_bits(const int32_t* indptr, const int32_t* indices, in
 }
 
 cudaError_t launch_bits_classify(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
-                                 int q_block, int kv_block, int causal, const GroupInfo* groups, int n_groups,
-                                 int nqt, uint8_t* cls, cudaStream_t s) {
+                                 int q_block, int kv_block, int causal, int g_pack, const GroupInfo* groups,
+                                 int n_groups, int nqt, uint8_t* cls, cudaStream_t s) {
   if (n_groups <= 0 || nqt <= 0) return cudaSuccess;
-  BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal};
+  BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal, g_pack};
   k_bits_classify<<<dim3(n_groups, nqt), 128, 0, s>>>(a, groups, cls);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bits_fine(const uint32_t* bits, const uint32_t* kv_valid, int nqb, int wpr, int kv_wpb,
-                             int q_block, int kv_block, int causal, const GroupInfo* groups, const int32_t* row_group,
-                             int n_rows, const int32_t* row_ptr, const int32_t* kv_tile, const int32_t* part,
-                             uint32_t* fine, cudaStream_t s) {
+                             int q_block, int kv_block, int causal, int g_pack, const GroupInfo* groups,
+                             const int32_t* row_group, int n_rows, const int32_t* row_ptr, const int32_t* kv_tile,
+                             const int32_t* part, uint32_t* fine, cudaStream_t s) {
   if (n_rows <= 0) return cudaSuccess;
-  BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal};
+  BlockSparseArgs a{bits, kv_valid, nqb, wpr, kv_wpb, q_block, kv_block, causal, g_pack};
   k_bits_fine<<<n_rows, 128, 0, s>>>(a, groups, row_group, row_ptr, kv_tile, part, fine);
   return cudaGetLastError();
 }

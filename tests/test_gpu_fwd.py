@@ -524,3 +524,51 @@ def test_block_skipping_with_huge_threshold_is_exact():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     with pytest.raises(bfa.BfaError):
         bfa.fwd(P, q.cuda(), k.cuda(), v.cuda(), softmax_threshold=-1.0)
+
+
+# ---------------------------------------------------------------- GQA-packed BSR query tiles
+@pytest.mark.parametrize("qb,kb,G,causal,D", [
+    (16, 128, 8, False, 128), (16, 64, 8, True, 128), (32, 128, 4, True, 128), (64, 32, 2, False, 128),
+    (16, 128, 8, True, 64),
+])
+def test_bsr_packed_forward(qb, kb, G, causal, D):
+    # a tile holds 128 / G positions of every head of a kv head; outputs and LSE
+    # against the oracle per head, and the unpacked plan of the same routing agrees
+    from test_gpu_plan import _routing, _valid_bits
+    B, Hkv, Sq, Skv = 2, 2, 300, 520
+    H = Hkv * G
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    indptr, indices = _routing(B, Hkv, nqb, nkb, 500 + qb + G)
+    kvb = _valid_bits(B, Skv, 11)
+    P = bfa.plan_bsr_packed(_cuda(indptr), _cuda(indices), Sq, Skv, G, qb, kb, causal=causal,
+                            kv_valid_bits=_cuda(kvb.view(np.int32)))
+    q, k, v = _rand((B, Sq, H, D), 61), _rand((B, Skv, Hkv, D), 62), _rand((B, Skv, Hkv, D), 63)
+    out, lse = bfa.fwd(P, q.cuda(), k.cuda(), v.cuda())
+    Pu = bfa.plan_bsr(_cuda(indptr), _cuda(indices), Sq, Skv, qb, kb, causal=causal,
+                      kv_valid_bits=_cuda(kvb.view(np.int32)))
+    out_u, lse_u = bfa.fwd(Pu, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    P.device_status()
+    M = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=causal,
+                            kv_valid_bits=kvb)
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    check_bshd(out.cpu(), lse.cpu(), q, k, v, lambda b, h: M[b, h // G], None, pairs, where="packed bsr")
+    assert (out.float() - out_u.float()).abs().max().item() <= 2e-2
+    fin = torch.isfinite(lse_u)
+    assert torch.equal(fin, torch.isfinite(lse)) and (lse - lse_u)[fin].abs().max().item() <= 2e-3
+
+
+def test_bsr_packed_forward_rejects_other_head_counts_and_the_backward():
+    from test_gpu_plan import _routing
+    B, Hkv, Sq, Skv, D, G = 1, 2, 256, 256, 128, 4
+    indptr, indices = _routing(B, Hkv, Sq // 32, Skv // 128, 9)
+    P = bfa.plan_bsr_packed(_cuda(indptr), _cuda(indices), Sq, Skv, G, 32, 128)
+    k, v = _rand((B, Skv, Hkv, D), 2).cuda(), _rand((B, Skv, Hkv, D), 3).cuda()
+    with pytest.raises(bfa.BfaError) as e:   # H / Hkv = 2 against the plan's 4
+        bfa.fwd(P, _rand((B, Sq, 2 * Hkv, D), 1).cuda(), k, v)
+    assert e.value.status == "BFA_ERR_INVALID_ARG"
+    q = _rand((B, Sq, G * Hkv, D), 1).cuda()
+    out, lse = bfa.fwd(P, q, k, v)
+    with pytest.raises(bfa.BfaError) as e:
+        bfa.bwd(P, q, k, v, out, out, lse)
+    assert e.value.status == "BFA_ERR_UNSUPPORTED"

@@ -358,3 +358,32 @@ def test_transposed_lists_block_bits_and_predicates():
     Pp = bfa.plan_predicate(terms, B=2, Sq=700, Sk=650)
     Mp = om.predicate_dense(terms, 700, 650)
     _assert_cols_equal(Pp, [Mp, Mp])
+
+
+# ---------------------------------------------------------------- GQA-packed BSR plans
+@pytest.mark.parametrize("qb,kb,G,causal,valid", [
+    (16, 128, 8, False, False), (16, 64, 8, True, True), (32, 128, 4, True, False), (64, 32, 2, False, True),
+    (8, 16, 16, True, False), (100, 128, 2, False, False),
+])
+def test_bsr_packed_plans(qb, kb, G, causal, valid):
+    # the plan of each (batch, kv head) group over its packed rows (position-major,
+    # every head of the kv head), bit for bit against the oracle's plan of the same rows
+    B, Hkv, Sq, Skv = 2, 2, 300, 520
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    indptr, indices = _routing(B, Hkv, nqb, nkb, qb * 100 + kb + G)
+    kvb = _valid_bits(B, Skv, G) if valid else None
+    P = bfa.plan_bsr_packed(_cuda(indptr), _cuda(indices), Sq, Skv, G, qb, kb, causal=causal,
+                            kv_valid_bits=_cuda(kvb.view(np.int32)) if valid else None)
+    assert P.info["heads_per_kv"] == G and P.info["sq"] == Sq
+    M = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=causal,
+                            kv_valid_bits=kvb)
+    ref = oracle_plan_for_groups([om.gqa_packed_rows(M[b, h], G) for b in range(B) for h in range(Hkv)])
+    assert_plan_equal(P.export(), ref)
+
+
+def test_bsr_packed_rejects_bad_packing():
+    indptr, indices = _routing(1, 1, 4, 4, 5)
+    for qb, G in ((64, 3), (64, 256), (3, 2), (64, 0)):
+        with pytest.raises(bfa.BfaError) as e:
+            bfa.plan_bsr_packed(_cuda(indptr), _cuda(indices), 4 * qb, 512, G, qb, 128)
+        assert e.value.status == "BFA_ERR_INVALID_ARG"

@@ -134,6 +134,39 @@ def bsr_routing(B, Hkv, n_blocks, seed):
     return indptr, np.concatenate(idx).astype(np.int32)
 
 
+def bsr_rows_routing(B, Hkv, Sq, q_block, kv_block, seed):
+    """BSR rows of q_block query tokens: the key block holding the row's first
+    token plus floor(d / 4) distinct earlier key blocks (d = that block's index),
+    drawn independently for every row."""
+    rng = np.random.default_rng(seed)
+    nqb = -(-Sq // q_block)
+    indptr = np.zeros((B, Hkv, nqb + 1), dtype=np.int32)
+    idx = []
+    pos = 0
+    for b in range(B):
+        for h in range(Hkv):
+            indptr[b, h, 0] = pos
+            for r in range(nqb):
+                d = (r * q_block) // kv_block
+                n_prev = d // 4
+                prev = rng.choice(d, size=n_prev, replace=False) if n_prev else np.zeros(0, np.int64)
+                row = np.sort(np.concatenate([prev, [d]])).astype(np.int32)
+                idx.append(row)
+                pos += row.size
+                indptr[b, h, r + 1] = pos
+    return indptr, np.concatenate(idx).astype(np.int32)
+
+
+def bsr_16384_q16_gqa8(B=2, H=32, Hkv=4, S=16384, D=128, q_block=16, kv_block=128, with_qkv=True):
+    """BSR routing with 16-token query rows and 8 query heads per kv head (GQA)."""
+    indptr, indices = bsr_rows_routing(B, Hkv, S, q_block, kv_block, 1000 * 5 + 7)
+    out = dict(name="bsr_16384_q16_gqa8", B=B, H=H, Hkv=Hkv, S=S, D=D, q_block=q_block, kv_block=kv_block,
+               block_indptr=indptr, block_indices=indices, causal=True, scale=D ** -0.5)
+    if with_qkv:
+        out["q"], out["k"], out["v"] = qkv(6, (B, S, H, D), (B, S, Hkv, D))
+    return out
+
+
 def bsr_16384(B=2, H=32, Hkv=8, S=16384, D=128, block=128, with_qkv=True):
     indptr, indices = bsr_routing(B, Hkv, -(-S // block), 1000 * 5 + 3)
     out = dict(name="bsr_16384", B=B, H=H, Hkv=Hkv, S=S, D=D, block=block,
