@@ -270,8 +270,9 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint8_t* sV, 
 }
 
 // kSkip: approximate mode (content-based block skipping); the exact kernel is
-// compiled without any of its code.
-template <int D, bool kSkip>
+// compiled without any of its code.  kPacked: GQA-packed query tiles (5-D Q / O
+// boxes, rows mapped to (position, head)); the other kernels hold none of it.
+template <int D, bool kSkip, bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
     bfa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dq = s ? sQ1 : sQ0;
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn) {
-          if (p.pack_g > 1)  // 128 >> pack_shift positions of every head of the kv head
+          if constexpr (kPacked)  // 128 >> pack_shift positions of every head of the kv head
             tma_load_5d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, 0, wk_s.hk, qs >> p.pack_shift, wk_s.b);
           else
             tma_load_4d(smem_u32(dq + pn * 16384), &tmQ, bar(BQ), pn * 64, wk_s.h[s], qs, wk_s.b);
@@ -579,8 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = qpos < wk.q_len;  // TMEM loads below stay whole-warp; only stores are per row
       const int h = slot ? wk.h[1] : wk.h[0];
       // the row's query head and position (GQA-packed tiles: rows position-major over the kv head's heads)
-      const int hrow = p.pack_g > 1 ? (wk.hk << p.pack_shift) + (qpos & (p.pack_g - 1)) : h;
-      const int prow = p.pack_g > 1 ? qpos >> p.pack_shift : qpos;
+      const int hrow = kPacked ? (wk.hk << p.pack_shift) + (qpos & (p.pack_g - 1)) : h;
+      const int prow = kPacked ? qpos >> p.pack_shift : qpos;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       const int qt0 = (slot ? wk.qt[1] : wk.qt[0]) * kTile;  // first row of the tile in its group
       if (qt0 + kTile <= wk.q_len) {
@@ -619,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (quarter == 0 && lane == 0 && ok && !*static_cast<volatile int*>(&abort_flag)) {
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
-            if (p.pack_g > 1)
+            if constexpr (kPacked)
               tma_store_5d(&tmO, stg + pn * 16384, pn * 64, 0, wk.hk, (wk.q_off + qt0) >> p.pack_shift, wk.b);
             else
               tma_store_4d(&tmO, stg + pn * 16384, pn * 64, h, wk.q_off + qt0, wk.b);
@@ -706,23 +707,32 @@ static cudaError_t prepare(K kernel, int smem) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
-template <int D, bool kSkip>
+template <int D, bool kSkip, bool kPacked>
 static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const CUtensorMap& to, const FwdParams& p, int64_t n_work, cudaStream_t s) {
-  static cudaError_t ready = prepare(bfa_fwd_kernel<D, kSkip>, Cfg<D>::kSmemBytes);
+  static cudaError_t ready = prepare(bfa_fwd_kernel<D, kSkip, kPacked>, Cfg<D>::kSmemBytes);
   if (ready != cudaSuccess) return ready;
-  bfa_fwd_kernel<D, kSkip><<<static_cast<unsigned>(n_work), kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+  bfa_fwd_kernel<D, kSkip, kPacked><<<static_cast<unsigned>(n_work), kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv,
+                                                                                                       to, p);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& to, const FwdParams& p, int64_t n_work, cudaStream_t s) {
+  const bool approx = p.skip_log2 > 0.f, packed = p.pack_g > 1;
+  if (packed)
+    return approx ? launch_one<D, true, true>(tq, tk, tv, to, p, n_work, s)
+                  : launch_one<D, false, true>(tq, tk, tv, to, p, n_work, s);
+  return approx ? launch_one<D, true, false>(tq, tk, tv, to, p, n_work, s)
+                : launch_one<D, false, false>(tq, tk, tv, to, p, n_work, s);
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int64_t n_work, cudaStream_t s) {
   if (n_work <= 0) return cudaSuccess;
   if (n_work > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const bool approx = p.skip_log2 > 0.f;
-  if (D == 64)
-    return approx ? launch_one<64, true>(tq, tk, tv, to, p, n_work, s) : launch_one<64, false>(tq, tk, tv, to, p, n_work, s);
-  return approx ? launch_one<128, true>(tq, tk, tv, to, p, n_work, s) : launch_one<128, false>(tq, tk, tv, to, p, n_work, s);
+  return D == 64 ? launch_d<64>(tq, tk, tv, to, p, n_work, s) : launch_d<128>(tq, tk, tv, to, p, n_work, s);
 }
 
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s) {
@@ -732,10 +742,12 @@ cudaError_t launch_wait_selftest(uint32_t* err, uint64_t cap, cudaStream_t s) {
 
 cudaError_t probe_fwd_kernels() {
   cudaFuncAttributes a;
-  cudaError_t e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, false>);
-  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, false>);
-  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, true>);
-  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, true>);
+  cudaError_t e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, false, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, false, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, true, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, true, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<128, false, true>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, bfa_fwd_kernel<64, false, true>);
   return e;
 }
 
