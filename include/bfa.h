@@ -219,10 +219,11 @@ bfa_status bfa_plan_bsr(const int32_t* indptr, const int32_t* indices, int64_t n
  * hkv * heads_per_kv + t % heads_per_kv; a 128-row tile is 128 / heads_per_kv
  * positions of all heads_per_kv heads.  heads_per_kv = H / Hkv of the calls that
  * use the plan: a power of two up to 128, with q_block * heads_per_kv a multiple
- * of 8 (the page's rule); other arguments as for bfa_plan_bsr.  Only bfa_fwd,
- * bfa_fwd_approx and bfa_fwd_paged take these plans (a batched (B, Sq, H, D) query
- * layout with heads of one kv head adjacent, as BSHD has them); bfa_bwd returns
- * BFA_ERR_UNSUPPORTED for them.
+ * of 8 (the page's rule); other arguments as for bfa_plan_bsr.  Every call takes
+ * these plans (bfa_fwd, bfa_fwd_approx, bfa_fwd_paged, bfa_bwd) with H = Hkv *
+ * heads_per_kv and a batched (B, Sq, H, D) query layout whose heads of one kv head
+ * are adjacent, as BSHD has them; q, out, dout and dq move as 5-D boxes of all
+ * the kv head's heads.
  */
 bfa_status bfa_plan_bsr_packed(const int32_t* indptr, const int32_t* indices, int64_t n_indices, int B, int Hkv,
                                int heads_per_kv, int Sq, int Skv, int q_block, int kv_block, int causal,

@@ -1161,9 +1161,13 @@ bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const
                                 const int64_t* dks, const int64_t* dvs, cudaStream_t st) {
   std::string why;
   const int bq = P->varlen ? 1 : B;
+  const int G = P->pack_g;
   CUtensorMap tq, tdo, tk, tv;
-  if (!make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], &why) ||
-      !make_tmap(&tdo, dout, D, H, P->sq, bq, dos[2], dos[1], dos[0], &why) ||
+  const bool qmaps = G > 1 ? (make_tmap_packed(&tq, q, D, G, Hkv, P->sq, bq, qs[2], qs[1], qs[0], &why) &&
+                              make_tmap_packed(&tdo, dout, D, G, Hkv, P->sq, bq, dos[2], dos[1], dos[0], &why))
+                           : (make_tmap(&tq, q, D, H, P->sq, bq, qs[2], qs[1], qs[0], &why) &&
+                              make_tmap(&tdo, dout, D, H, P->sq, bq, dos[2], dos[1], dos[0], &why));
+  if (!qmaps ||
       !make_tmap(&tk, k, D, Hkv, P->sk, bq, ks[2], ks[1], ks[0], &why) ||
       !make_tmap(&tv, v, D, Hkv, P->sk, bq, vs[2], vs[1], vs[0], &why))
     return fail(BFA_ERR_INVALID_ARG, "%s", why.c_str());
@@ -1202,8 +1206,12 @@ bfa_status bwd_launch_from_host(bfa_plan* P, const void* q, const void* k, const
   p.H = H;
   p.Hkv = Hkv;
   p.D = D;
-  p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? H / Hkv : H);
+  // packed plans hold every head of a kv head in their rows: one replica per row
+  p.rep = P->kind == BFA_PLAN_DENSE ? B * H : (P->kind == BFA_PLAN_BSR ? (G > 1 ? 1 : H / Hkv) : H);
   p.rep_kv = P->kind == BFA_PLAN_DENSE ? B * Hkv : (P->kind == BFA_PLAN_BSR ? 1 : Hkv);
+  p.pack_g = G;
+  p.pack_shift = 0;
+  while ((1 << p.pack_shift) < G) ++p.pack_shift;
   const int n_cols = plan_n_cols(P);
   const int64_t waves = 2LL * sm_count();
   auto chunk_for = [&](int64_t units, int64_t items) {
@@ -1296,8 +1304,8 @@ BFA_API bfa_status bfa_bwd(const bfa_plan* Pc, const void* q, const void* k, con
     return fail(BFA_ERR_INVALID_ARG, "B=%d does not match the plan's %d", B, P->batch);
   if (P->kind == BFA_PLAN_BSR && Hkv != P->hkv)
     return fail(BFA_ERR_INVALID_ARG, "Hkv=%d does not match the BSR routing's %d", Hkv, P->hkv);
-  if (P->pack_g > 1)
-    return fail(BFA_ERR_UNSUPPORTED, "the backward takes plans without GQA-packed query tiles (bfa_plan_bsr)");
+  if (P->pack_g > 1 && H != Hkv * P->pack_g)
+    return fail(BFA_ERR_INVALID_ARG, "the plan packs %d query heads per kv head; H / Hkv = %d", P->pack_g, H / Hkv);
   if (!lse) return fail(BFA_ERR_INVALID_ARG, "lse is required by the backward");
   bfa_status s;
   if ((s = need_device(q, "q")) || (s = need_device(k, "k")) || (s = need_device(v, "v")) ||

@@ -98,6 +98,32 @@ __device__ __forceinline__ int replica_of(const BwdParams& p, const GroupInfo& g
   return h;
 }
 
+// plan row `qpos` of a query tile -> its query position and head, for the row's
+// base head h (GQA-packed plans: rows position-major over the kv head's heads)
+__device__ __forceinline__ void row_pos_head(const BwdParams& p, int qpos, int h, int& prow, int& hrow) {
+  if (p.pack_g > 1) {
+    prow = qpos >> p.pack_shift;
+    hrow = h + (qpos & (p.pack_g - 1));
+  } else {
+    prow = qpos;
+    hrow = h;
+  }
+}
+
+// one 128-row tile of Q or dO: a 4-D box of one head, or a 5-D box of every head
+// of the kv head (GQA-packed plans)
+template <int kPanels>
+__device__ __forceinline__ void load_q_tile(const BwdParams& p, const CUtensorMap* map, uint8_t* dst, uint32_t bar,
+                                            int h, int hk, int qs, int b) {
+#pragma unroll
+  for (int pn = 0; pn < kPanels; ++pn) {
+    if (p.pack_g > 1)
+      tma_load_5d(smem_u32(dst + pn * 16384), map, bar, pn * 64, 0, hk, qs >> p.pack_shift, b);
+    else
+      tma_load_4d(smem_u32(dst + pn * 16384), map, bar, pn * 64, h, qs, b);
+  }
+}
+
 // kv replica index -> (batch, kv head) of a key-tile column
 __device__ __forceinline__ void kv_replica_bh(const BwdParams& p, const GroupInfo& g, int j, int& b, int& hk) {
   if (p.plan.kind == 1) {
@@ -184,12 +210,14 @@ __global__ void __launch_bounds__(128) k_bwd_prep(const BwdParams p) {
   const int r = static_cast<int>(blk % p.plan.n_rows);
   const int j = static_cast<int>(blk / p.plan.n_rows);
   const GroupInfo g = p.plan.groups[p.plan.row_group[r]];
-  int b, h;
-  replica_bh(p, g, j, b, h);
+  int b, h0;
+  replica_bh(p, g, j, b, h0);
   const int qpos = (r - g.row0) * kTile + threadIdx.x;
+  int prow, h;
+  row_pos_head(p, qpos, h0, prow, h);
   float dval = 0.f, lse2 = 0.f;
   if (qpos < g.q_len) {
-    const int64_t tok = static_cast<int64_t>(g.q_off) + qpos;
+    const int64_t tok = static_cast<int64_t>(g.q_off) + prow;
     const uint4* o4 = reinterpret_cast<const uint4*>(p.out + static_cast<int64_t>(b) * p.o_sb + tok * p.o_ss +
                                                      static_cast<int64_t>(h) * p.o_sh);
     const uint4* d4 = reinterpret_cast<const uint4*>(p.dout + static_cast<int64_t>(b) * p.do_sb + tok * p.do_ss +
@@ -209,7 +237,7 @@ __global__ void __launch_bounds__(128) k_bwd_prep(const BwdParams p) {
     }
     dval = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     const int64_t li = p.varlen ? static_cast<int64_t>(h) * p.Sq_lse + tok
-                                : (static_cast<int64_t>(b) * p.H + h) * p.Sq_lse + qpos;
+                                : (static_cast<int64_t>(b) * p.H + h) * p.Sq_lse + prow;
     const float L = p.lse[li];
     lse2 = (L == -INFINITY) ? 0.f : L * 1.4426950408889634f;  // a row that attends nothing has no listed pair
   }
@@ -319,11 +347,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       prefetch_tmap(&tmV);
       const int qs = wk.g.q_off + wk.qt * kTile;
       mbar_expect_tx(bar(BQ), 2 * C::kTileBytes);
-#pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_4d(smem_u32(sQ + pn * 16384), &tmQ, bar(BQ), pn * 64, wk.h, qs, wk.b);
-        tma_load_4d(smem_u32(sdO + pn * 16384), &tmdO, bar(BQ), pn * 64, wk.h, qs, wk.b);
-      }
+      load_q_tile<C::kPanels>(p, &tmQ, sQ, bar(BQ), wk.h, wk.hk, qs, wk.b);
+      load_q_tile<C::kPanels>(p, &tmdO, sdO, bar(BQ), wk.h, wk.hk, qs, wk.b);
       const int32_t* kv = p.plan.kv_tile + wk.e0;
       int last[kBwdStages] = {-1, -1};
       int kt_next = kv[0];
@@ -466,9 +491,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
     tc_fence_after();
     if (done) {
-      const int64_t tok = static_cast<int64_t>(wk.g.q_off) + qpos;
+      int prow, hrow;
+      row_pos_head(p, qpos, wk.h, prow, hrow);
+      const int64_t tok = static_cast<int64_t>(wk.g.q_off) + prow;
       __nv_bfloat16* dst =
-          p.dq + static_cast<int64_t>(wk.b) * p.dq_sb + tok * p.dq_ss + static_cast<int64_t>(wk.h) * p.dq_sh;
+          p.dq + static_cast<int64_t>(wk.b) * p.dq_sb + tok * p.dq_ss + static_cast<int64_t>(hrow) * p.dq_sh;
       // each half of the warps writes half of the row's D columns
       store_row<D / 2>(tLane + 256 + half * (D / 2), n > 0, p.scale, dst + half * (D / 2), qpos < wk.g.q_len);
     }
@@ -542,7 +569,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       w.nq = 0;
     }
 #endif
-    w.nh = p.H / p.Hkv;
+    w.nh = p.pack_g > 1 ? 1 : p.H / p.Hkv;  // packed tiles hold every head of the kv head
     kv_replica_bh(p, w.g, jk, w.b, w.hk);
     w.steps = w.nq * w.nh;
     wk_s = w;
@@ -558,8 +585,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const KvWork& wk = wk_s;
   const uint64_t cap = p.wait_ns;
   const int steps = wk.steps;
-  // step s -> query head and list entry
-  auto step_head = [&](int s) { return wk.hk * wk.nh + s / wk.nq; };
+  // step s -> query head (packed plans: the base head of the kv head) and list entry
+  auto step_head = [&](int s) { return (wk.hk * wk.nh + s / wk.nq) << p.pack_shift; };
   auto step_entry = [&](int s) { return wk.e0 + s % wk.nq; };
 
   if (warp == 0) {
@@ -589,11 +616,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t f = bar(BF + st);
         mbar_expect_tx(f, 2 * C::kTileBytes + C::kVecBytes);
         const int qs = wk.g.q_off + qt * kTile;
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_4d(smem_u32(sQ(st) + pn * 16384), &tmQ, f, pn * 64, h, qs, wk.b);
-          tma_load_4d(smem_u32(sdO(st) + pn * 16384), &tmdO, f, pn * 64, h, qs, wk.b);
-        }
+        load_q_tile<C::kPanels>(p, &tmQ, sQ(st), f, h, wk.hk, qs, wk.b);
+        load_q_tile<C::kPanels>(p, &tmdO, sdO(st), f, h, wk.hk, qs, wk.b);
         bulk_load(smem_u32(sVec(st)), p.ws_lse2 + wi, kTile * 4, f);
         bulk_load(smem_u32(sVec(st) + kTile), p.ws_d + wi, kTile * 4, f);
         last[st] = s;
@@ -881,7 +905,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       w.nq = 0;
     }
 #endif
-    w.nh = p.H / p.Hkv;
+    w.nh = p.pack_g > 1 ? 1 : p.H / p.Hkv;  // packed tiles hold every head of the kv head
     kv_replica_bh(p, w.g, jk, w.b, w.hk);
     w.steps = w.nq * w.nh;
     *wk_s = w;
@@ -897,7 +921,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const KvWork& wk = *wk_s;
   const uint64_t cap = p.wait_ns;
   const int steps = wk.steps;
-  auto step_head = [&](int s) { return wk.hk * wk.nh + s / wk.nq; };
+  auto step_head = [&](int s) { return (wk.hk * wk.nh + s / wk.nq) << p.pack_shift; };
   auto step_entry = [&](int s) { return wk.e0 + s % wk.nq; };
 
   if (warp < 4) {
@@ -929,11 +953,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           const uint32_t f = bar(BF + st);
           mbar_expect_tx(f, 2 * C::kTileBytes + C::kVecBytes);
           const int qs = wk.g.q_off + qt * kTile;
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn) {
-            tma_load_4d(smem_u32(sQ(st) + pn * 16384), &tmQ, f, pn * 64, h, qs, wk.b);
-            tma_load_4d(smem_u32(sdO(st) + pn * 16384), &tmdO, f, pn * 64, h, qs, wk.b);
-          }
+          load_q_tile<C::kPanels>(p, &tmQ, sQ(st), f, h, wk.hk, qs, wk.b);
+          load_q_tile<C::kPanels>(p, &tmdO, sdO(st), f, h, wk.hk, qs, wk.b);
           bulk_load(smem_u32(sVec(st)), p.ws_lse2 + wi, kTile * 4, f);
           bulk_load(smem_u32(sVec(st) + kTile), p.ws_d + wi, kTile * 4, f);
           last[st] = s;
@@ -1212,18 +1233,20 @@ __global__ void __launch_bounds__(128) k_bwd_dq_store(const BwdParams p) {
   replica_bh(p, g, j, b, h);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t wi = (static_cast<int64_t>(j) * p.plan.n_rows + r) * kTile;
-  __nv_bfloat16* const base = p.dq + static_cast<int64_t>(b) * p.dq_sb + static_cast<int64_t>(h) * p.dq_sh;
+  __nv_bfloat16* const base = p.dq + static_cast<int64_t>(b) * p.dq_sb;
 #pragma unroll 4
   for (int i = 0; i < 32; ++i) {
     const int row = warp * 32 + i;
     const int qpos = (r - g.row0) * kTile + row;
     if (qpos >= g.q_len) break;
     const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + (wi + row) * D + lane * 4);
-    const int64_t tok = static_cast<int64_t>(g.q_off) + qpos;
+    int prow, hrow;
+    row_pos_head(p, qpos, h, prow, hrow);
+    const int64_t tok = static_cast<int64_t>(g.q_off) + prow;
     uint2 o;
     o.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
     o.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
-    *reinterpret_cast<uint2*>(base + tok * p.dq_ss + lane * 4) = o;
+    *reinterpret_cast<uint2*>(base + tok * p.dq_ss + static_cast<int64_t>(hrow) * p.dq_sh + lane * 4) = o;
   }
 }
 

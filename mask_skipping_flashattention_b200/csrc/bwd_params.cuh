@@ -40,6 +40,11 @@ struct BwdParams {
   // tile), D values a row; zeroed by the preprocess, summed into by every key
   // tile of the row's list, then scaled into dq.  nullptr for the two-pass form.
   float* dq_acc;
+  // GQA-packed query tiles (bfa_plan_bsr_packed): plan row t of a tile is query
+  // position t >> pack_shift of head (kv head << pack_shift) + (t & (pack_g - 1));
+  // Q and dO move through 5-D maps.  pack_g = 1: rows are positions of one head.
+  int32_t pack_g;
+  int32_t pack_shift;
   // transposed lists of the plan
   const int32_t* col0;
   const int32_t* col_group;

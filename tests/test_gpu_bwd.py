@@ -396,3 +396,31 @@ def test_two_pass_form_is_bitwise_reproducible():
     P.device_status()
     assert all(torch.equal(x, y) for x, y in zip(a, b))
     assert torch.equal(f1[1], f2[1]) and torch.equal(f1[2], f2[2])
+
+
+@pytest.mark.parametrize("qb,kb,G,causal,D,form", [
+    (16, 128, 8, False, 128, "fused"), (32, 64, 4, True, 128, "fused"), (32, 64, 4, True, 128, "two_pass"),
+    (16, 128, 8, True, 64, "two_pass"),
+])
+def test_bsr_packed_backward(qb, kb, G, causal, D, form):
+    # GQA-packed plans: a tile's rows are positions x every head of a kv head; the
+    # gradients against the oracle per head, dK / dV summing the group's heads
+    from test_gpu_plan import _routing, _valid_bits
+    B, Hkv, Sq, Skv = 2, 2, 300, 520
+    H = Hkv * G
+    nqb, nkb = -(-Sq // qb), -(-Skv // kb)
+    indptr, indices = _routing(B, Hkv, nqb, nkb, 900 + qb + G)
+    kvb = _valid_bits(B, Skv, 13)
+    P = bfa.plan_bsr_packed(_cuda(indptr), _cuda(indices), Sq, Skv, G, qb, kb, causal=causal,
+                            kv_valid_bits=_cuda(kvb.view(np.int32)))
+    M = om.block_bits_dense(om.bsr_to_block_bits(indptr, indices, nkb), Sq, Skv, qb, kb, causal=causal,
+                            kv_valid_bits=kvb)
+    q = workloads.randn_bf16((B, Sq, H, D), 81)
+    k = workloads.randn_bf16((B, Skv, Hkv, D), 82)
+    v = workloads.randn_bf16((B, Skv, Hkv, D), 83)
+    do = workloads.randn_bf16((B, Sq, H, D), 84)
+    if form == "two_pass":
+        with _two_pass():
+            _run_bshd(P, q, k, v, do, lambda b, h: M[b, h // G])
+    else:
+        _run_bshd(P, q, k, v, do, lambda b, h: M[b, h // G])

@@ -52,6 +52,7 @@ CASES = [
     "tests/test_gpu_bwd.py::test_two_pass_form_is_bitwise_reproducible",
     "tests/test_gpu_plan.py::test_bsr_packed_plans",
     "tests/test_gpu_fwd.py::test_bsr_packed_forward",
+    "tests/test_gpu_bwd.py::test_bsr_packed_backward",
     # full-size workloads, the bench's own launch among them
     "tests/test_gpu_plan.py::test_dense_plan_causal_8192",
     "tests/test_gpu_plan.py::test_bsr_plan_workload_full_size_every_group",

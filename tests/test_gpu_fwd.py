@@ -558,7 +558,7 @@ def test_bsr_packed_forward(qb, kb, G, causal, D):
     assert torch.equal(fin, torch.isfinite(lse)) and (lse - lse_u)[fin].abs().max().item() <= 2e-3
 
 
-def test_bsr_packed_forward_rejects_other_head_counts_and_the_backward():
+def test_bsr_packed_plans_reject_other_head_counts():
     from test_gpu_plan import _routing
     B, Hkv, Sq, Skv, D, G = 1, 2, 256, 256, 128, 4
     indptr, indices = _routing(B, Hkv, Sq // 32, Skv // 128, 9)
@@ -569,6 +569,7 @@ def test_bsr_packed_forward_rejects_other_head_counts_and_the_backward():
     assert e.value.status == "BFA_ERR_INVALID_ARG"
     q = _rand((B, Sq, G * Hkv, D), 1).cuda()
     out, lse = bfa.fwd(P, q, k, v)
+    q2 = _rand((B, Sq, 2 * Hkv, D), 4).cuda()
     with pytest.raises(bfa.BfaError) as e:
-        bfa.bwd(P, q, k, v, out, out, lse)
-    assert e.value.status == "BFA_ERR_UNSUPPORTED"
+        bfa.bwd(P, q2, k, v, q2, q2, lse)
+    assert e.value.status == "BFA_ERR_INVALID_ARG"
