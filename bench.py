@@ -540,7 +540,7 @@ def run_sweep(args):
     del w, u
     # 16-token BSR rows with 8 query heads per kv head: GQA-packed tiles (one BSR
     # row of all 8 heads per tile) against 128-token tiles (the union of 8 rows'
-    # lists); forward only (packed plans have no backward)
+    # lists)
     w = workloads.bsr_16384_q16_gqa8()
     ip, ix, S, qb, kb = w["block_indptr"], w["block_indices"], w["S"], w["q_block"], w["kv_block"]
     G = w["H"] // w["Hkv"]
@@ -556,7 +556,7 @@ def run_sweep(args):
     for name, plan in (("bsr_16384_q16_gqa8 packed", bfa.plan_bsr_packed(cuda(ip), cuda(ix), S, S, G, qb, kb,
                                                                          causal=True)),
                        ("bsr_16384_q16_gqa8 unpacked", bfa.plan_bsr(cuda(ip), cuda(ix), S, S, qb, kb, causal=True))):
-        measure(name, plan, q, k, v, per_group * G, w["D"], "BSR, 16-token rows, causal inside blocks", bwd=False)
+        measure(name, plan, q, k, v, per_group * G, w["D"], "BSR, 16-token rows, causal inside blocks")
         del plan
     return 0
 
