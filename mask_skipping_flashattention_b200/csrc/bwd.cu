@@ -10,9 +10,15 @@
 // D_i = dO_i . O_i, the score gradient is dS = P * (dP - D), and
 //   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
 //
-// Three kernels:
+// Kernels:
 //   k_bwd_prep  per query row: D = dO . O and LSE * log2(e) into a workspace
-//               padded to whole tiles (HBM-bound, one pass over O and dO);
+//               padded to whole tiles (HBM-bound, one pass over O and dO); for
+//               the fused pass it also zeroes the fp32 dQ sums;
+//   k_bwd_fused (D = 128, the default) one pass over the key-tile columns: the
+//               k_bwd_dkdv pass below plus dQ^T = K^T dS^T from the same dS,
+//               summed across key tiles by fp32 reductions; k_bwd_dq_store then
+//               scales the sums into dq (S and dP are made once per tile pair);
+// and the two passes (D = 64, or bitwise-reproducible results on request):
 //   k_bwd_dq    one CTA per (plan row, replica), walking the row's key-tile list:
 //               S = Q K^T and dP = dO V^T (SS), dS into TMEM as bf16, dQ += dS K
 //               (TS); the next tile's S and dP run while this tile's dS is made

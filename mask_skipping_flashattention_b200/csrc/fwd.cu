@@ -2,7 +2,8 @@
 //
 // Each CTA runs two 128-row query tiles ("slots") that share their keys and
 // values: either two heads of one kv head on the same query tile (GQA with an
-// even group), or two consecutive query tiles of one head.  The CTA walks the
+// even group), or two consecutive query tiles of one head, or (GQA-packed plans,
+// kPacked) two consecutive tiles of 128 / G positions x all G heads of a kv head.  The CTA walks the
 // union of the two tiles' plan lists (BinFlash: walk each query block's sorted list of
 // non-empty key blocks, run all-True blocks with no mask loads, apply the mask on
 // partial blocks only, skip all-False blocks).  Work items are taken in the
