@@ -573,3 +573,25 @@ def test_bsr_packed_plans_reject_other_head_counts():
     with pytest.raises(bfa.BfaError) as e:
         bfa.bwd(P, q2, k, v, q2, q2, lse)
     assert e.value.status == "BFA_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("page_size", [16, 128])
+def test_bsr_packed_paged_and_approximate(page_size):
+    # packed tiles with keys / values in a paged cache give the contiguous result bit
+    # for bit, and the approximate mode with a threshold that drops nothing gives the
+    # exact result bit for bit
+    from test_gpu_plan import _routing
+    B, Hkv, G, Sq, Skv, D, qb, kb = 2, 2, 4, 256, 384, 128, 32, 64
+    H = Hkv * G
+    indptr, indices = _routing(B, Hkv, -(-Sq // qb), -(-Skv // kb), 41)
+    P = bfa.plan_bsr_packed(_cuda(indptr), _cuda(indices), Sq, Skv, G, qb, kb, causal=True)
+    q = _rand((B, Sq, H, D), 91).cuda()
+    kc, vc, table, ks, vs = _paged_cache([Skv] * B, page_size, Hkv, D, 95 + page_size)
+    k, v = torch.stack(ks).cuda(), torch.stack(vs).cuda()
+    o1, l1 = bfa.fwd(P, q, k, v)
+    o2, l2 = bfa.fwd_paged(P, q, kc.cuda(), vc.cuda(), _cuda(table))
+    o3, l3 = bfa.fwd(P, q, k, v, softmax_threshold=1e9)
+    torch.cuda.synchronize()
+    P.device_status()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
