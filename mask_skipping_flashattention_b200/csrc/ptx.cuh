@@ -196,7 +196,7 @@ __device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, uint32_t sr
       "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
       : "memory");
 }
-// 1-D bulk copy global -> shared (no tensor map, no multicast): both addresses
+// 1-D bulk copy global -> this CTA's shared memory (no tensor map): both addresses
 // 16-byte aligned, bytes a multiple of 16; completes `bytes` on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
