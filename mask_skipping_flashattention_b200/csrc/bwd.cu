@@ -824,8 +824,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ----------------------------------------------------------------------------
 // fused pass (D = 128): one CTA per (key-tile column, kv replica), walking the
 // column's query-tile list as k_bwd_dkdv does, and making dQ from the same dS:
-// dQ^T = K^T dS^T runs into the dP^T columns once dK has read dS^T there, and a
-// fourth warpgroup reads it out and sums it into an fp32 workspace.  Each
+// dQ^T = K^T dS^T runs into the dP^T columns once dK has read dS^T there, and
+// two more warpgroups read it out and sum it into an fp32 workspace.  Each
 // (query tile, key tile) pair then costs five 128 x 128 x 128 products instead
 // of the two passes' seven (S and dP are made once).
 // ----------------------------------------------------------------------------
@@ -833,8 +833,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // issuer, warps 2..3 idle, warps 4..7 the P^T / dS^T rows (one key per thread;
 // dS^T also goes to shared memory as the B operand of dQ^T), warps 8..15 the dQ
 // rows (one head dimension per thread, the TMEM lanes of dQ^T; warps 8..11 take
-// queries [0, 64) and warps 12..15 queries [64, 128): one SM needs eight warps
-// of reductions in flight to reach the rate L2 accepts them at).
+// queries [0, 64) and warps 12..15 queries [64, 128): on its own, one SM needs
+// eight warps of scalar reductions in flight to reach the rate L2 accepts them
+// at; inside this pass four and eight warps measured the same).
 // Shared memory (1024-aligned, nothing static): K, V, Q[2], dO[2], dS^T, the
 // query vectors of two steps, then the barriers and the work item.
 // TMEM (512 columns): S^T [0,128) (P^T over [0,64)), dP^T [128,256) (dS^T over
