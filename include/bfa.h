@@ -60,8 +60,10 @@ typedef enum bfa_status {
   BFA_ERR_CAPACITY = -5,         /* sizes beyond what the library can index or allocate */
   BFA_ERR_CUDA = -6,             /* a CUDA runtime call failed                          */
   BFA_ERR_TIMEOUT = -7,          /* a device-side wait ran past its bound               */
-  BFA_ERR_BOUNDS = -8            /* checked build only: an index left its array, or the
-                                    guard bytes after a plan array were overwritten      */
+  BFA_ERR_BOUNDS = -8            /* checked build: an index left its array, or the guard
+                                    bytes after a plan array were overwritten; any build:
+                                    a block of the fused backward was given shared memory
+                                    that is not 1024-byte aligned and did no work         */
 } bfa_status;
 
 enum { BFA_TILE = 128 };
