@@ -322,8 +322,9 @@ def test_forward_and_backward_give_up_on_a_short_wait_bound():
     """The kernels' own failure path: with the shortest loop-wait bound (1 us) the
     first wait of a block for its scores outlasts the bound (the copies of Q and K
     alone take longer), so blocks stop their work, drain the copies and products
-    they issued, release tensor memory and report BFA_ERR_TIMEOUT through the plan.
-    Afterwards the default bound gives oracle-exact results on the same plan."""
+    they issued, release tensor memory and report BFA_ERR_TIMEOUT through the plan
+    (forward, fused backward, two-pass backward).  Afterwards the default bound
+    gives oracle-exact results on the same plan."""
     B, H, N, D = 2, 8, 2048, 128
     M = np.tril(np.ones((N, N), dtype=bool))
     q, k, v = (_rand((B, N, H, D), 9100 + i) for i in range(3))
@@ -337,13 +338,16 @@ def test_forward_and_backward_give_up_on_a_short_wait_bound():
             P.device_status()
         assert e.value.status == "BFA_ERR_TIMEOUT"
         dout = _rand((B, N, H, D), 9199).cuda()
-        bfa.bwd(P, qc, kc, vc, out, dout, lse)
-        torch.cuda.synchronize()
-        with pytest.raises(bfa.BfaError) as e:
-            P.device_status()
-        assert e.value.status == "BFA_ERR_TIMEOUT"
+        for deterministic in (False, True):  # the fused pass, then the two passes
+            bfa.set_bwd_deterministic(deterministic)
+            bfa.bwd(P, qc, kc, vc, out, dout, lse)
+            torch.cuda.synchronize()
+            with pytest.raises(bfa.BfaError) as e:
+                P.device_status()
+            assert e.value.status == "BFA_ERR_TIMEOUT"
     finally:
         bfa.set_wait_timeout_ns(0)
+        bfa.set_bwd_deterministic(False)
     out, lse = bfa.fwd(P, qc, kc, vc)
     torch.cuda.synchronize()
     P.device_status()
