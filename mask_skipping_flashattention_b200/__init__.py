@@ -283,7 +283,8 @@ def plan_bsr(block_indptr, block_indices, Sq, Skv, q_block_size=TILE, kv_block_s
 def plan_bsr_packed(block_indptr, block_indices, Sq, Skv, heads_per_kv, q_block_size=TILE, kv_block_size=TILE,
                     causal=False, kv_valid_bits=None, stream=None):
     """BSR plan with GQA-packed query tiles: each tile holds 128 / heads_per_kv query
-    positions of all ``heads_per_kv`` query heads of a kv head (forward only)."""
+    positions of all ``heads_per_kv`` query heads of a kv head (H = Hkv * heads_per_kv
+    in the calls that use it, forward and backward)."""
     ip = block_indptr.to(torch.int32).contiguous()
     ix = block_indices.to(torch.int32).contiguous()
     kv = kv_valid_bits.contiguous() if kv_valid_bits is not None else None

@@ -352,3 +352,19 @@ def test_gqa_packed_rows_of_a_bsr_routing_follow_the_routing():
         blocks = set(indices[indptr[0, 0, r]:indptr[0, 0, r + 1]].tolist())
         for j in range(Skv):
             assert packed[t, j] == (j // kb in blocks)
+
+
+def test_short_row_bsr_routing_is_canonical_and_follows_its_rule():
+    # the 16-token-row routing of the packed-tile workload: canonical rows, each the key
+    # block of its first token plus floor(d / 4) distinct earlier blocks
+    import workloads
+    Sq, qb, kb = 1000, 16, 128
+    ip, ix = workloads.bsr_rows_routing(2, 3, Sq, qb, kb, 11)
+    assert ip.shape == (2, 3, -(-Sq // qb) + 1)
+    assert om.bsr_is_canonical(ip, ix, -(-Sq // kb))
+    for b in range(2):
+        for h in range(3):
+            for r in range(ip.shape[2] - 1):
+                row = ix[ip[b, h, r]:ip[b, h, r + 1]]
+                d = (r * qb) // kb
+                assert row[-1] == d and row.size == d // 4 + 1 and (row[:-1] < d).all()
